@@ -1,0 +1,373 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other than
+itself -- the numbers the pages print, closed forms, library routines for a
+special case, and brute force on tiny inputs.  CPU only."""
+
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import indexer_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
+
+
+def _facts():
+    with open(GOLDEN) as f:
+        return json.load(f)["facts"]
+
+
+def _printed(n, fact):
+    """Round n to the number of significant digits the page prints."""
+    return round(n / fact["scale"], fact["digits"] - len(str(int(fact["mantissa"])))) == fact["mantissa"]
+
+
+# ---------------------------------------------------------------- page numbers
+
+def test_shapes_follow_the_pages():
+    f = _facts()
+    shapes = oracle.parameter_shapes(f["model_width"]["value"], f["q_latent_dim"]["value"],
+                                     f["indexer_heads"]["value"], f["indexer_head_dim"]["value"])
+    assert shapes["W_q"] == (f["q_latent_dim"]["value"], f["q_projection_out"]["value"])
+    assert shapes["W_w"] == (f["weight_projection_in"]["value"], f["weight_projection_out"]["value"])
+    assert shapes["W_k"][1] == f["key_dim"]["value"]
+    assert f["indexer_heads"]["value"] * f["indexer_head_dim"]["value"] == f["q_projection_out"]["value"]
+    assert f["index_rope_dim"]["value"] == 0  # the oracle applies no rotary step at all
+
+
+def test_parameter_count_matches_printed_figures():
+    f = _facts()
+    n = oracle.parameter_count()
+    assert n == 7_438_592
+    assert _printed(n, f["params_per_layer_printed"])
+    assert _printed(f["indexer_layers"]["value"] * n, f["params_total_printed"])
+
+
+def test_parameter_count_rejects_biased_projections():
+    # Bias vectors on the three projections (4,096 + 128 + 32 per layer) still
+    # print as 7.44M per layer but not as 178.5M over 24 layers.
+    f = _facts()
+    biased = oracle.parameter_count() + 4096 + 128 + 32
+    assert _printed(biased, f["params_per_layer_printed"])
+    assert not _printed(f["indexer_layers"]["value"] * biased, f["params_total_printed"])
+
+
+def test_project_consumes_exactly_the_counted_parameters():
+    rng = np.random.default_rng(0)
+    T, hd, ql, H, D = 3, 16, 8, 2, 4
+    shapes = oracle.parameter_shapes(hd, ql, H, D)
+    ws = {k: rng.standard_normal(s) for k, s in shapes.items()}
+    q, k, w = oracle.project(rng.standard_normal((T, hd)), rng.standard_normal((T, ql)),
+                             ws["W_q"], ws["W_k"], ws["W_w"], ws["ln_gamma"], ws["ln_beta"],
+                             n_heads=H, head_dim=D)
+    assert q.shape == (T, H, D) and k.shape == (T, D) and w.shape == (T, H)
+    bad = dict(ws)
+    bad["W_k"] = np.concatenate([ws["W_k"], np.zeros((1, D))])  # a bias row folded in
+    with pytest.raises(ValueError):
+        oracle.project(rng.standard_normal((T, hd)), rng.standard_normal((T, ql)),
+                       bad["W_q"], bad["W_k"], bad["W_w"], bad["ln_gamma"], bad["ln_beta"],
+                       n_heads=H, head_dim=D)
+
+
+# ---------------------------------------------------------------- bf16 rounding
+
+def test_bf16_round_matches_torch_conversion_of_fp32_values():
+    rng = np.random.default_rng(1)
+    mant = rng.uniform(1.0, 2.0, 200_000)
+    expo = rng.integers(-149, 128, 200_000)
+    sign = rng.choice([-1.0, 1.0], 200_000)
+    x32 = (sign * np.ldexp(mant, expo)).astype(np.float32)   # includes fp32 subnormals and near-max values
+    x32 = x32[np.isfinite(x32)]
+    ref = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.bf16_round(x32.astype(np.float64))
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_bf16_round_ties_go_to_even():
+    ulp = 2.0 ** -7
+    assert oracle.bf16_round(1.0 + ulp / 2) == 1.0                 # tie, 1.0 is even
+    assert oracle.bf16_round(1.0 + 3 * ulp / 2) == 1.0 + 2 * ulp   # tie, goes up to even
+    assert oracle.bf16_round(1.0 + ulp / 2 + 2.0 ** -30) == 1.0 + ulp
+    assert oracle.bf16_round(-(1.0 + ulp / 2)) == -1.0
+    assert oracle.bf16_round(2.0 ** 128 * (1 - 2.0 ** -9)) == np.inf  # rounds past the largest finite bf16
+    assert oracle.bf16_round(0.0) == 0.0
+
+
+def test_bf16_bits_round_trip():
+    bits = np.arange(0, 0x7F80, 7, dtype=np.uint16)
+    vals = oracle.bf16_bits_to_float64(bits)
+    np.testing.assert_array_equal(oracle.float64_to_bf16_bits(vals), bits)
+    np.testing.assert_array_equal(oracle.bf16_round(vals), vals)
+
+
+# ---------------------------------------------------------------- LayerNorm
+
+def test_layer_norm_matches_torch_float64():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((64, 128)) * 3 + 0.5
+    g = 1 + 0.02 * rng.standard_normal(128)
+    b = 0.02 * rng.standard_normal(128)
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (128,), torch.from_numpy(g),
+                                         torch.from_numpy(b), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.layer_norm(x, g, b, 1e-6), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_layer_norm_closed_form():
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((32, 128)) * 0.1
+    eps = 1e-3
+    y = oracle.layer_norm(x, np.ones(128), np.zeros(128), eps)
+    v = x.var(axis=1)
+    np.testing.assert_allclose(y.mean(axis=1), 0.0, atol=1e-12)
+    np.testing.assert_allclose(y.var(axis=1), v / (v + eps), rtol=1e-12)
+    # scale invariance up to eps, and the affine part is applied after normalising
+    np.testing.assert_allclose(oracle.layer_norm(7 * x, np.ones(128), np.zeros(128), 0.0),
+                               oracle.layer_norm(x, np.ones(128), np.zeros(128), 0.0), rtol=1e-10)
+    g = rng.standard_normal(128)
+    b = rng.standard_normal(128)
+    np.testing.assert_allclose(oracle.layer_norm(x, g, b, eps), y * g + b, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- projections, brute force
+
+def _py_project(hidden, q_latent, Wq, Wk, Ww, gamma, beta, eps, H, D):
+    """Pure-Python loops, dyadic inputs (every sum exact in float64)."""
+    T = len(hidden)
+    q = [[[sum(q_latent[t][i] * Wq[i][h * D + d] for i in range(len(Wq))) for d in range(D)]
+          for h in range(H)] for t in range(T)]
+    kraw = [[sum(hidden[t][i] * Wk[i][d] for i in range(len(Wk))) for d in range(D)] for t in range(T)]
+    k = []
+    for row in kraw:
+        mu = sum(row) / D
+        var = sum((v - mu) ** 2 for v in row) / D
+        k.append([(row[d] - mu) / (var + eps) ** 0.5 * gamma[d] + beta[d] for d in range(D)])
+    w = [[sum(hidden[t][i] * Ww[i][h] for i in range(len(Ww))) for h in range(H)] for t in range(T)]
+    return np.array(q), np.array(k), np.array(w)
+
+
+def test_project_matches_python_loops_on_tiny_dyadic_inputs():
+    rng = np.random.default_rng(4)
+    T, hd, ql, H, D = 5, 12, 10, 3, 4
+    hidden = rng.integers(-4, 5, (T, hd)).astype(np.float64)
+    q_latent = rng.integers(-4, 5, (T, ql)).astype(np.float64)
+    Wq = rng.integers(-8, 9, (ql, H * D)) / 8.0
+    Wk = rng.integers(-8, 9, (hd, D)) / 8.0
+    Ww = rng.integers(-8, 9, (hd, H)) / 8.0
+    gamma = 1 + rng.integers(-4, 5, D) / 64.0
+    beta = rng.integers(-4, 5, D) / 64.0
+    eps = 2.0 ** -10
+    q, k, w = oracle.project(hidden, q_latent, Wq, Wk, Ww, gamma, beta, eps, H, D)
+    pq, pk, pw = _py_project(hidden.tolist(), q_latent.tolist(), Wq.tolist(), Wk.tolist(),
+                             Ww.tolist(), gamma.tolist(), beta.tolist(), eps, H, D)
+    np.testing.assert_array_equal(q, oracle.bf16_round(pq))       # sums are exact, one rounding
+    np.testing.assert_allclose(k, oracle.bf16_round(pk), rtol=2.0 ** -8)  # sqrt may differ in the last fp64 bit
+    np.testing.assert_array_equal(w, pw.astype(np.float32).astype(np.float64))
+    # q head h is columns h*D .. h*D+D-1 of the projection
+    np.testing.assert_array_equal(q.reshape(T, H * D), oracle.bf16_round(q_latent @ Wq))
+
+
+# ---------------------------------------------------------------- score and selection, brute force
+
+def _py_scores(q_t, w_t, keys):
+    out = []
+    for k in keys:
+        tot = 0.0
+        for h in range(len(q_t)):
+            dot = sum(q_t[h][d] * k[d] for d in range(len(k)))
+            tot += w_t[h] * max(0.0, dot)
+        out.append(tot)
+    return out
+
+
+@pytest.mark.parametrize("H,D,top_k", [(1, 2, 1), (1, 4, 3), (2, 2, 3), (2, 4, 1), (2, 4, 3)])
+def test_topk_matches_bruteforce_on_tiny_inputs(H, D, top_k):
+    rng = np.random.default_rng(100 + 10 * H + D + top_k)
+    T = 12
+    q = rng.integers(-3, 4, (T, H, D)).astype(np.float64)
+    w = rng.integers(-2, 3, (T, H)) / 2.0
+    keys = rng.integers(-3, 4, (T, D)).astype(np.float64)
+    pos = np.arange(T)
+    offs = np.array([0, T])
+    idx, sc = oracle.topk(q, w, pos, offs, keys, offs, top_k=top_k)
+    for t in range(T):
+        I = _py_scores(q[t].tolist(), w[t].tolist(), keys[: t + 1].tolist())
+        n = t + 1
+        if n <= top_k:
+            assert idx[t].tolist() == list(range(n)) + [-1] * (top_k - n)
+            continue
+        sel = idx[t].tolist()
+        assert len(set(sel)) == top_k and all(0 <= s <= t for s in sel)   # causal, inclusive
+        # the chosen set is a best set: it maximises the sum and the minimum over all subsets
+        best_sum = max(sum(I[s] for s in c) for c in itertools.combinations(range(n), top_k))
+        best_min = max(min(I[s] for s in c) for c in itertools.combinations(range(n), top_k))
+        assert sum(I[s] for s in sel) == best_sum
+        assert min(I[s] for s in sel) == best_min
+        # order: score descending, position ascending
+        keyed = [(-I[s], s) for s in sel]
+        assert keyed == sorted(keyed)
+        # ties at the boundary go to the lower positions
+        thr = min(I[s] for s in sel)
+        unsel = [s for s in range(n) if s not in sel]
+        assert all(I[s] < thr or s > max(x for x in sel if I[x] == thr) for s in unsel)
+        np.testing.assert_array_equal(sc[t], [I[s] for s in sel])
+
+
+def test_scores_match_python_loops():
+    rng = np.random.default_rng(5)
+    q = rng.integers(-5, 6, (4, 8)).astype(np.float64)
+    w = rng.integers(-4, 5, 4) / 4.0
+    keys = rng.integers(-5, 6, (30, 8)).astype(np.float64)
+    I, A = oracle.index_scores(q, w, keys)
+    np.testing.assert_array_equal(I, _py_scores(q.tolist(), w.tolist(), keys.tolist()))
+    np.testing.assert_array_equal(A, [sum(abs(w[h] * (q[h] @ k)) for h in range(4)) for k in keys])
+
+
+# ---------------------------------------------------------------- invariants and special cases
+
+def _rand_case(seed, T=40, H=4, D=8):
+    rng = np.random.default_rng(seed)
+    q = oracle.bf16_round(rng.standard_normal((T, H, D)))
+    w = rng.standard_normal((T, H)).astype(np.float32).astype(np.float64)
+    keys = oracle.bf16_round(rng.standard_normal((T, D)))
+    return q, w, keys
+
+
+def test_zero_head_weights_give_zero_scores():
+    q, w, keys = _rand_case(6)
+    I, A = oracle.index_scores(q[0], np.zeros(4), keys)
+    assert np.all(I == 0.0)
+
+
+def test_relu_terms_nonnegative_for_nonnegative_weights():
+    q, w, keys = _rand_case(7)
+    for t in range(10):
+        I, A = oracle.index_scores(q[t], np.abs(w[t]), keys)
+        assert np.all(I >= 0.0)
+        assert np.all(I <= A + 1e-12)
+    # every head term alone carries the sign of its weight
+    for h in range(4):
+        wh = np.zeros(4)
+        wh[h] = -abs(w[0, h]) - 0.5
+        I, _ = oracle.index_scores(q[0], wh, keys)
+        assert np.all(I <= 0.0)
+
+
+def test_single_head_unit_weight_is_textbook_relu_topk():
+    rng = np.random.default_rng(8)
+    D, n, k = 16, 500, 37
+    q = oracle.bf16_round(rng.standard_normal((1, D)))
+    keys = oracle.bf16_round(rng.standard_normal((n, D)))
+    I, _ = oracle.index_scores(q, np.ones(1), keys)
+    relu = np.maximum(keys @ q[0], 0)
+    np.testing.assert_array_equal(I, relu)
+    sel = oracle.select_topk(I, k)
+    ref = np.argpartition(-relu, k - 1)[:k]
+    np.testing.assert_array_equal(np.sort(relu[sel]), np.sort(relu[ref]))
+
+
+def test_short_prefix_selects_everything_in_position_order():
+    q, w, keys = _rand_case(9, T=40)
+    pos = np.arange(40)
+    offs = np.array([0, 40])
+    idx, sc = oracle.topk(q, w, pos, offs, keys, offs, top_k=16)
+    for t in range(16):
+        assert idx[t].tolist() == list(range(t + 1)) + [-1] * (15 - t)
+        assert np.all(np.isneginf(sc[t, t + 1:]))
+    for t in range(16, 40):
+        assert np.all(idx[t] >= 0) and np.all(idx[t] <= t)
+
+
+def test_future_keys_do_not_matter():
+    q, w, keys = _rand_case(10, T=40)
+    pos = np.arange(40)
+    offs = np.array([0, 40])
+    a = oracle.topk(q, w, pos, offs, keys, offs, top_k=8)[0]
+    for t in (5, 20, 33):
+        keys2 = keys.copy()
+        keys2[t + 1:] = oracle.bf16_round(np.random.default_rng(t).standard_normal(keys2[t + 1:].shape)) * 9
+        b = oracle.topk(q[t:t + 1], w[t:t + 1], pos[t:t + 1], np.array([0, 1]), keys2, offs, top_k=8)[0]
+        np.testing.assert_array_equal(a[t], b[0])
+
+
+def test_permuting_visible_keys_permutes_indices():
+    q, w, keys = _rand_case(11, T=60)
+    perm = np.random.default_rng(12).permutation(60)
+    t = 59
+    one = np.array([0, 1])
+    offs = np.array([0, 60])
+    a = oracle.topk(q[t:t + 1], w[t:t + 1], np.array([59]), one, keys, offs, top_k=10)[0][0]
+    b = oracle.topk(q[t:t + 1], w[t:t + 1], np.array([59]), one, keys[perm], offs, top_k=10)[0][0]
+    assert set(perm[b].tolist()) == set(a.tolist())
+
+
+def test_positive_weight_scale_keeps_the_set():
+    q, w, keys = _rand_case(13, T=60)
+    pos = np.arange(60)
+    offs = np.array([0, 60])
+    a = oracle.topk(q, w, pos, offs, keys, offs, top_k=9)[0]
+    b = oracle.topk(q, w * 8.0, pos, offs, keys, offs, top_k=9)[0]
+    np.testing.assert_array_equal(a, b)
+
+
+def test_sequences_are_independent():
+    q, w, keys = _rand_case(14, T=40)
+    # sequence 0: tokens 0..24 at positions 0..24; sequence 1: tokens 25..39 at positions 0..14
+    pos = np.concatenate([np.arange(25), np.arange(15)])
+    qoff = np.array([0, 25, 40])
+    coff = np.array([0, 25, 40])
+    idx, _ = oracle.topk(q, w, pos, qoff, keys, coff, top_k=6)
+    a = oracle.topk(q[:25], w[:25], pos[:25], np.array([0, 25]), keys[:25], np.array([0, 25]), top_k=6)[0]
+    b = oracle.topk(q[25:], w[25:], pos[25:], np.array([0, 15]), keys[25:], np.array([0, 15]), top_k=6)[0]
+    np.testing.assert_array_equal(idx, np.concatenate([a, b]))
+
+
+def test_sorted_order_helper():
+    I = np.array([0.5, 2.0, 2.0, -1.0, 3.0])
+    assert oracle.sort_selected(np.array([0, 1, 2, 4, -1]), I).tolist() == [4, 1, 2, 0, -1]
+
+
+# ---------------------------------------------------------------- planted mistakes are caught
+
+def _bruteforce_ok(score_fn):
+    rng = np.random.default_rng(200)
+    q = rng.integers(-3, 4, (8, 2, 4)).astype(np.float64)
+    w = rng.integers(-2, 3, (8, 2)) / 2.0
+    keys = rng.integers(-3, 4, (8, 4)).astype(np.float64)
+    for t in range(8):
+        I, _ = score_fn(q[t], w[t], keys[: t + 1])
+        if not np.array_equal(I, _py_scores(q[t].tolist(), w[t].tolist(), keys[: t + 1].tolist())):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("mistake", ["no_relu", "relu_after_weight", "transposed_heads", "abs_weight"])
+def test_planted_score_mistakes_fail_the_bruteforce_pin(mistake):
+    def wrong(q_t, w_t, keys):
+        logits = keys @ q_t.T
+        if mistake == "no_relu":
+            I = logits @ w_t
+        elif mistake == "relu_after_weight":
+            I = np.maximum(logits * w_t, 0).sum(axis=1)
+        elif mistake == "transposed_heads":
+            I = np.maximum(logits, 0) @ w_t[::-1]
+        else:
+            I = np.maximum(logits, 0) @ np.abs(w_t)
+        return I, np.abs(logits) @ np.abs(w_t)
+    assert _bruteforce_ok(O.index_scores)
+    assert not _bruteforce_ok(wrong)
+
+
+def test_planted_layernorm_mistakes_fail_the_closed_form():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((16, 128))
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (128,), eps=1e-6).numpy()
+    ones, zeros = np.ones(128), np.zeros(128)
+    unbiased = (x - x.mean(1, keepdims=True)) / np.sqrt(x.var(1, ddof=1, keepdims=True) + 1e-6)
+    rms = x / np.sqrt((x ** 2).mean(1, keepdims=True) + 1e-6)
+    assert np.allclose(oracle.layer_norm(x, ones, zeros, 1e-6), ref, atol=1e-10)
+    assert not np.allclose(unbiased, ref, atol=1e-6)
+    assert not np.allclose(rms, ref, atol=1e-6)

@@ -1,0 +1,162 @@
+"""Seeded generators for the indexer's five workloads (random draws only).
+
+Shapes and value distributions:
+  * weights: W_q [1536, 4096], W_k [7168, 128], W_w [7168, 32], bf16, each
+    N(0, 1/fan_in); LayerNorm gain 1 + N(0, 0.02^2) and bias N(0, 0.02^2), bf16.
+  * prefill activations: hidden [T, 7168] and query latent [T, 1536], bf16
+    N(0, 1); token positions 0..n_b-1 per sequence (or a chunk's offset).
+  * decode: 64 sequences with cache lengths uniform in [16384, 131072]; the
+    pre-norm key rows of every cached token are fp32 N(0, 1) (the key cache is
+    the LayerNorm of these rows, computed by whichever side consumes them).
+
+Each tensor is drawn from its own torch CPU generator whose seed is derived
+from (workload seed, stream id), so that no two tensors share a random stream.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+# Kimi K3.1 Pro indexer dimensions ('Sparse / compressed attn' row of the
+# archdiff.com compare pages): hidden width 7,168, query latent 1,536,
+# 32 heads x 128 dims, top 2,048 tokens per query.
+MODEL_DIMS = dict(hidden_dim=7168, q_latent_dim=1536, n_heads=32, head_dim=128, top_k=2048)
+
+# The five workloads: three single-shot prefills, one decode step, one chunked
+# long-context prefill.
+WORKLOADS = {
+    "prefill_3k": dict(kind="prefill", seq_lens=[3072], weight_seed=0, act_seed=0),
+    "prefill_8k": dict(kind="prefill", seq_lens=[8192], weight_seed=1, act_seed=2),
+    "prefill_2x32k_heavy": dict(kind="prefill", seq_lens=[32768, 32768], weight_seed=3,
+                                act_seed=4, heavy_frac=0.01, heavy_scale=4.0),
+    "decode_64": dict(kind="decode", batch=64, L_min=16384, L_max=131072, weight_seed=5,
+                      act_seed=5),
+    "chunked_128k": dict(kind="chunked", seq_len=131072, chunk=8192, weight_seed=6, act_seed=7),
+}
+
+# stream ids: one per tensor kind
+_S_WQ, _S_WK, _S_WW, _S_GAMMA, _S_BETA = 1, 2, 3, 4, 5
+_S_HIDDEN, _S_QLAT, _S_LENS, _S_RAWK, _S_HEAVY = 11, 12, 13, 14, 15
+
+
+def _gen(seed: int, stream: int, sub: int = 0) -> torch.Generator:
+    g = torch.Generator()
+    g.manual_seed((int(seed) * 1_000_003 + stream * 7919 + int(sub) * 104_729) & 0x7FFF_FFFF_FFFF)
+    return g
+
+
+def _normal(g: torch.Generator, shape, std: float = 1.0, mean: float = 0.0) -> torch.Tensor:
+    x = torch.randn(shape, generator=g, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    if mean != 0.0:
+        x.add_(mean)
+    return x
+
+
+@dataclass
+class Weights:
+    W_q: torch.Tensor      # bf16 [q_latent_dim, n_heads*head_dim]   (in x out)
+    W_k: torch.Tensor      # bf16 [hidden_dim, head_dim]
+    W_w: torch.Tensor      # bf16 [hidden_dim, n_heads]
+    gamma: torch.Tensor    # bf16 [head_dim]
+    beta: torch.Tensor     # bf16 [head_dim]
+
+
+@dataclass
+class PrefillBatch:
+    hidden: torch.Tensor         # bf16 [T, hidden_dim]
+    q_latent: torch.Tensor       # bf16 [T, q_latent_dim]
+    positions: torch.Tensor      # int32 [T], position of each query token in its sequence
+    q_seq_offsets: torch.Tensor  # int32 [B+1], token ranges of the B sequences
+    cache_offsets: torch.Tensor  # int64 [B+1], key-cache row ranges of the B sequences
+    extra: dict = field(default_factory=dict)
+
+
+@dataclass
+class DecodeBatch:
+    lengths: torch.Tensor        # int64 [B], cached tokens per sequence (incl. the new one)
+    raw_keys: torch.Tensor       # fp32 [sum L, head_dim], pre-norm key rows of every cached token
+    hidden: torch.Tensor         # bf16 [B, hidden_dim], the new token of each sequence
+    q_latent: torch.Tensor       # bf16 [B, q_latent_dim]
+    positions: torch.Tensor      # int32 [B] = L_b - 1
+    q_seq_offsets: torch.Tensor  # int32 [B+1] = 0..B
+    cache_offsets: torch.Tensor  # int64 [B+1]
+
+
+def make_weights(seed: int, hidden_dim: int = 7168, q_latent_dim: int = 1536,
+                 n_heads: int = 32, head_dim: int = 128) -> Weights:
+    """Random-init weights of one indexer layer, N(0, 1/fan_in), bf16."""
+    W_q = _normal(_gen(seed, _S_WQ), (q_latent_dim, n_heads * head_dim), q_latent_dim ** -0.5)
+    W_k = _normal(_gen(seed, _S_WK), (hidden_dim, head_dim), hidden_dim ** -0.5)
+    W_w = _normal(_gen(seed, _S_WW), (hidden_dim, n_heads), hidden_dim ** -0.5)
+    gamma = _normal(_gen(seed, _S_GAMMA), (head_dim,), 0.02, 1.0)
+    beta = _normal(_gen(seed, _S_BETA), (head_dim,), 0.02)
+    bf = torch.bfloat16
+    return Weights(W_q.to(bf), W_k.to(bf), W_w.to(bf), gamma.to(bf), beta.to(bf))
+
+
+def make_prefill(seed: int, seq_lens, start_positions=None, cache_lens=None,
+                 hidden_dim: int = 7168, q_latent_dim: int = 1536, sub: int = 0) -> PrefillBatch:
+    """B sequences of query tokens.  Sequence b has seq_lens[b] tokens at
+    positions start_b .. start_b+n_b-1 and owns cache_lens[b] key-cache rows
+    (default start_b + n_b, i.e. exactly the causal prefix of its last token)."""
+    seq_lens = [int(n) for n in seq_lens]
+    B = len(seq_lens)
+    starts = [0] * B if start_positions is None else [int(s) for s in start_positions]
+    clens = [s + n for s, n in zip(starts, seq_lens)] if cache_lens is None else [int(c) for c in cache_lens]
+    for s, n, c in zip(starts, seq_lens, clens):
+        if s + n > c:
+            raise ValueError("a sequence's positions must fit inside its cache rows")
+    T = sum(seq_lens)
+    hidden = _normal(_gen(seed, _S_HIDDEN, sub), (T, hidden_dim)).to(torch.bfloat16)
+    q_latent = _normal(_gen(seed, _S_QLAT, sub), (T, q_latent_dim)).to(torch.bfloat16)
+    positions = torch.cat([torch.arange(s, s + n, dtype=torch.int32) for s, n in zip(starts, seq_lens)]) \
+        if T > 0 else torch.zeros(0, dtype=torch.int32)
+    q_seq_offsets = torch.zeros(B + 1, dtype=torch.int32)
+    q_seq_offsets[1:] = torch.cumsum(torch.tensor(seq_lens, dtype=torch.int64), 0).to(torch.int32)
+    cache_offsets = torch.zeros(B + 1, dtype=torch.int64)
+    cache_offsets[1:] = torch.cumsum(torch.tensor(clens, dtype=torch.int64), 0)
+    return PrefillBatch(hidden, q_latent, positions, q_seq_offsets, cache_offsets)
+
+
+def make_decode(seed: int, batch: int = 64, L_min: int = 16384, L_max: int = 131072,
+                hidden_dim: int = 7168, q_latent_dim: int = 1536, head_dim: int = 128,
+                lengths=None) -> DecodeBatch:
+    """One new query token per sequence; sequence b holds L_b cached tokens
+    (the new token is the last, at position L_b - 1)."""
+    if lengths is None:
+        lengths = torch.randint(L_min, L_max + 1, (batch,), generator=_gen(seed, _S_LENS), dtype=torch.int64)
+    else:
+        lengths = torch.as_tensor(lengths, dtype=torch.int64)
+        batch = int(lengths.numel())
+    total = int(lengths.sum())
+    raw_keys = _normal(_gen(seed, _S_RAWK), (total, head_dim))
+    hidden = _normal(_gen(seed, _S_HIDDEN), (batch, hidden_dim)).to(torch.bfloat16)
+    q_latent = _normal(_gen(seed, _S_QLAT), (batch, q_latent_dim)).to(torch.bfloat16)
+    positions = (lengths - 1).to(torch.int32)
+    q_seq_offsets = torch.arange(batch + 1, dtype=torch.int32)
+    cache_offsets = torch.zeros(batch + 1, dtype=torch.int64)
+    cache_offsets[1:] = torch.cumsum(lengths, 0)
+    return DecodeBatch(lengths, raw_keys, hidden, q_latent, positions, q_seq_offsets, cache_offsets)
+
+
+def heavy_hitter_rows(seed: int, cache_offsets: torch.Tensor, frac: float = 0.01) -> torch.Tensor:
+    """Global key-cache rows to scale (round(frac * L_b) per sequence, drawn
+    without replacement).  Scaling a bf16 row by 4 is exact."""
+    rows = []
+    g = _gen(seed, _S_HEAVY)
+    offs = [int(v) for v in cache_offsets.tolist()]
+    for b in range(len(offs) - 1):
+        L = offs[b + 1] - offs[b]
+        m = int(round(frac * L))
+        if m > 0:
+            rows.append(torch.randperm(L, generator=g)[:m] + offs[b])
+    return torch.cat(rows).to(torch.int64) if rows else torch.zeros(0, dtype=torch.int64)
+
+
+def causal_pairs(positions: torch.Tensor) -> int:
+    """Number of (query, key) pairs a causal pass scores: sum over queries of pos + 1."""
+    return int(positions.to(torch.int64).sum()) + int(positions.numel())
