@@ -1,0 +1,469 @@
+#!/usr/bin/env python3
+"""Benchmark of the DSA lightning indexer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the hot path over one batch: the projections
+(dsa_indexer_project) and the score + top-2,048 (dsa_indexer_topk).  The
+headline workload is the 8,192-token single-sequence prefill; the decode step
+(64 sequences, caches of 16K..128K tokens) is measured in the same run and
+reported under "decode".  Inputs are seeded synthetic tensors resident in HBM;
+L2 is flushed (256 MB write) between timed steps, outside the timed events.
+
+With N > 1 (torchrun), every rank runs its own independent batch (weak
+scaling, no collective on the data path); times are the max over ranks.
+--impl reference times the CPU oracle on a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "indexer score+top-2048 Gpairs/s (prefill), decode GB/s; % of roofline"
+FLOP_PER_PAIR = 2 * 32 * 128           # one (query, key) pair: 32 heads x 128-dim dot products
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------------------------------ helpers
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def _profile_traffic(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summaries
+    (profiles/traffic.txt lines 'key: bytes source_hash'), or None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    from dsa_lightning_indexer_03_b200 import build as B
+    src_hash = B.source_hash()
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        key, _, rest = line.partition(":")
+        parts = rest.split()
+        if key.strip() == kernel_key and len(parts) >= 2 and parts[1] == src_hash:
+            return float(parts[0])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _flush_l2(buf):
+    buf.add_(1)
+
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------------ GPU arm
+
+def _setup_prefill(d, name, seed_offset, device):
+    cfg = W.WORKLOADS[name]
+    wts = W.make_weights(cfg["weight_seed"])
+    batch = W.make_prefill(cfg["act_seed"] + seed_offset, cfg["seq_lens"])
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    ix = d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta),
+                   max_tokens=max(batch.hidden.shape[0], 256))
+    T = batch.hidden.shape[0]
+    rows = int(batch.cache_offsets[-1])
+    st = dict(ix=ix, T=T, host=batch,
+              hidden=to(batch.hidden), q_latent=to(batch.q_latent), positions=to(batch.positions),
+              qoff=to(batch.q_seq_offsets), coff=to(batch.cache_offsets),
+              cache=torch.zeros((rows, 128), dtype=torch.bfloat16, device=device),
+              q=torch.empty((T, 32, 128), dtype=torch.bfloat16, device=device),
+              w=torch.empty((T, 32), dtype=torch.float32, device=device),
+              idx=torch.empty((T, 2048), dtype=torch.int32, device=device),
+              score=torch.empty((T, 2048), dtype=torch.float32, device=device),
+              pairs=W.causal_pairs(batch.positions))
+    return st
+
+
+def _prefill_step(st, ev=None):
+    ix = st["ix"]
+    ix.project(st["hidden"], st["q_latent"], st["positions"], st["qoff"], st["cache"], st["coff"],
+               q_out=st["q"], w_out=st["w"])
+    if ev is not None:
+        ev[0].record()
+    ix.topk(st["q"], st["w"], st["positions"], st["qoff"], st["cache"], st["coff"], idx_out=st["idx"],
+            score_out=st["score"])
+    if ev is not None:
+        ev[1].record()
+
+
+def _setup_decode(d, seed_offset, device):
+    cfg = W.WORKLOADS["decode_64"]
+    wts = W.make_weights(cfg["weight_seed"])
+    g = torch.Generator().manual_seed(1000 + seed_offset)
+    lengths = torch.randint(cfg["L_min"], cfg["L_max"] + 1, (cfg["batch"],), generator=g)
+    batch = W.make_decode(cfg["act_seed"] + seed_offset, lengths=torch.ones_like(lengths))  # new tokens only
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    ix = d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta), max_tokens=256)
+    B = cfg["batch"]
+    total = int(lengths.sum())
+    coff = torch.zeros(B + 1, dtype=torch.int64)
+    coff[1:] = torch.cumsum(lengths, 0)
+    # cached keys: LayerNorm (through the library) of N(0,1) pre-norm rows drawn on the device
+    gd = torch.Generator(device=device).manual_seed(2000 + seed_offset)
+    cache = torch.empty((total, 128), dtype=torch.bfloat16, device=device)
+    step = 1 << 20
+    for s in range(0, total, step):
+        n = min(step, total - s)
+        raw = torch.randn((n, 128), generator=gd, device=device, dtype=torch.float32)
+        ix.key_norm(raw, out=cache[s:s + n])
+    torch.cuda.synchronize()
+    positions = (lengths - 1).to(torch.int32)
+    st = dict(ix=ix, T=B, hidden=to(batch.hidden), q_latent=to(batch.q_latent), positions=to(positions),
+              qoff=to(torch.arange(B + 1, dtype=torch.int32)), coff=to(coff), cache=cache,
+              q=torch.empty((B, 32, 128), dtype=torch.bfloat16, device=device),
+              w=torch.empty((B, 32), dtype=torch.float32, device=device),
+              idx=torch.empty((B, 2048), dtype=torch.int32, device=device),
+              score=torch.empty((B, 2048), dtype=torch.float32, device=device),
+              total_keys=total)
+    # algorithmic bytes of the score + top-k: every cached key once, q/w once, indices+scores out
+    st["bytes"] = total * 128 * 2 + B * (32 * 128 * 2 + 32 * 4) + B * 2048 * (4 + 4)
+    return st
+
+
+def _time_steps(fn, steps, flush):
+    """Per-step CUDA events (L2 flushed between steps, outside the events);
+    returns (step ms list, inner ms list)."""
+    outer, inner = [], []
+    for _ in range(steps):
+        flush()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        fn((e[1], e[2]))
+        e[3].record()
+        outer.append(e)
+    torch.cuda.synchronize()
+    return ([a[0].elapsed_time(a[3]) for a in outer], [a[1].elapsed_time(a[2]) for a in outer])
+
+
+def _e2e_prefill(st, steps):
+    """Same metric through the public API with host buffers: pinned host inputs
+    copied in, indices copied out, every step."""
+    h = st["host"]
+    pin = {k: getattr(h, k).pin_memory() for k in ("hidden", "q_latent", "positions", "q_seq_offsets",
+                                                    "cache_offsets")}
+    out = torch.empty((st["T"], 2048), dtype=torch.int32).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in pin.values())
+    bo = out.numel() * out.element_size()
+    ts = []
+    for _ in range(steps):
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        st["hidden"].copy_(pin["hidden"], non_blocking=True)
+        st["q_latent"].copy_(pin["q_latent"], non_blocking=True)
+        st["positions"].copy_(pin["positions"], non_blocking=True)
+        st["qoff"].copy_(pin["q_seq_offsets"], non_blocking=True)
+        st["coff"].copy_(pin["cache_offsets"], non_blocking=True)
+        _prefill_step(st)
+        out.copy_(st["idx"], non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    return statistics.mean(ts), bi, bo
+
+
+def gpu_arm(args, rank, world, local_rank, dist):
+    import dsa_lightning_indexer_03_b200 as d
+    from dsa_lightning_indexer_03_b200 import build as B
+    B.build()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    peaks = _peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    flush = lambda: _flush_l2(flush_buf)  # noqa: E731
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # ---------------- prefill (headline)
+    st = _setup_prefill(d, args.workload, rank, device)
+    fn = lambda ev: _prefill_step(st, ev)  # noqa: E731
+    _time_steps(fn, args.warmup, flush)
+    barrier()
+    with ClockSampler(device.index) as clk:
+        step_ms, topk_ms = _time_steps(fn, args.steps, flush)
+    barrier()
+    clocks = clk.summary()
+    ms = max_over_ranks(statistics.mean(step_ms))
+    topk_avg = max_over_ranks(statistics.mean(topk_ms))
+    pairs = st["pairs"]
+    value = pairs * world / (ms * 1e-3) / 1e9
+    achieved_tflops = pairs * FLOP_PER_PAIR / (topk_avg * 1e-3) / 1e12
+    traffic = _profile_traffic(f"score_topk:{args.workload}")
+    e2e_ms, bi, bo = _e2e_prefill(st, max(2, min(args.steps, 5)))
+    e2e_ms = max_over_ranks(e2e_ms)
+    st["ix"].device_error()
+
+    # ---------------- decode (second half of the metric)
+    dec = None
+    if not args.skip_decode:
+        del st
+        torch.cuda.empty_cache()
+        ds = _setup_decode(d, rank, device)
+
+        def dfn(ev):
+            ix = ds["ix"]
+            ix.project(ds["hidden"], ds["q_latent"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"],
+                       q_out=ds["q"], w_out=ds["w"])
+            if ev is not None:
+                ev[0].record()
+            ix.topk(ds["q"], ds["w"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"], idx_out=ds["idx"],
+                    score_out=ds["score"])
+            if ev is not None:
+                ev[1].record()
+
+        _time_steps(dfn, args.warmup, flush)
+        barrier()
+        dstep, dtopk = _time_steps(dfn, args.steps, flush)
+        barrier()
+        dms = max_over_ranks(statistics.mean(dtopk))
+        dstep_ms = max_over_ranks(statistics.mean(dstep))
+        gbs = ds["bytes"] / (dms * 1e-3) / 1e9
+        dec = {"workload": "decode_64", "metric": "decode GB/s", "value": round(gbs * world, 2), "unit": "GB/s",
+               "ms_score_topk": round(dms, 4), "ms_per_step": round(dstep_ms, 4),
+               "keys_scanned": ds["total_keys"], "algorithmic_bytes": ds["bytes"],
+               "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(gbs / peaks["hbm_gbs"], 4),
+                            "traffic": _profile_traffic("score_topk:decode_64")}}
+        ds["ix"].device_error()
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "Gpairs/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) random-init weights)",
+        "config": {"workload": args.workload, "batch": len(W.WORKLOADS[args.workload]["seq_lens"]),
+                   "seq_len": W.WORKLOADS[args.workload]["seq_lens"][0], "heads": 32, "head_dim": 128,
+                   "top_k": 2048, "causal_pairs_per_gpu": pairs, "parallelism": f"independent replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(achieved_tflops / peaks["bf16_tflops"], 4),
+                     "traffic": traffic, "kernel": "score_topk (dsa_indexer_topk: prep + score)",
+                     "ms_per_launch": round(topk_avg, 4), "peak_source": peaks["source"] + " burst bf16"},
+        "e2e": {"value": round(pairs * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "Gpairs/s",
+                "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
+        "clocks": clocks,
+        "gpu_launches": args.steps * 4,
+    }
+    if dec is not None:
+        line["decode"] = dec
+    return line
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle arm
+
+def cpu_oracle_sample(name, n_rows=24, seed=0):
+    """The oracle as it stands on a bounded sample of the workload: keys of the
+    whole prefix plus q/w/top-k of n_rows query rows spread over the positions.
+    Returns (Gpairs/s, description)."""
+    import numpy as np
+
+    import oracle
+    cfg = W.WORKLOADS[name]
+    wts = W.make_weights(cfg["weight_seed"])
+    batch = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
+    T = batch.hidden.shape[0]
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(T, size=min(n_rows, T), replace=False))
+    f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    t0 = time.perf_counter()
+    max_pos = int(batch.positions[rows].max())
+    _, k, _ = oracle.project(f(batch.hidden[:max_pos + 1]), f(batch.q_latent[:max_pos + 1]), f(wts.W_q), f(wts.W_k),
+                             f(wts.W_w), f(wts.gamma), f(wts.beta))
+    q, _, w = oracle.project(f(batch.hidden[rows]), f(batch.q_latent[rows]), f(wts.W_q), f(wts.W_k), f(wts.W_w),
+                             f(wts.gamma), f(wts.beta))
+    qq = np.zeros((T, 32, 128))
+    ww = np.zeros((T, 32))
+    qq[rows] = q
+    ww[rows] = w
+    oracle.topk(qq, ww, batch.positions.numpy(), batch.q_seq_offsets.numpy(), k, np.array([0, k.shape[0]]),
+                rows=rows)
+    dt = time.perf_counter() - t0
+    pairs = int((batch.positions[rows].to(torch.int64) + 1).sum())
+    return pairs / dt / 1e9, f"{len(rows)} query rows of {name} (keys of their whole prefix projected), {dt:.1f} s"
+
+
+def reference_arm(args):
+    vals = []
+    desc = ""
+    for _ in range(args.warmup):
+        cpu_oracle_sample(args.workload, n_rows=4)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        v, desc = cpu_oracle_sample(args.workload, n_rows=8, seed=i)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.mean(vals)
+    cores = _cpu_threads()
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "Gpairs/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(wall / max(args.steps, 1) * 1e3, 2),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": len(W.WORKLOADS[args.workload]["seq_lens"]),
+                   "seq_len": W.WORKLOADS[args.workload]["seq_lens"][0], "top_k": 2048},
+        "cpu_baseline": {"value": round(value, 6), "unit": "Gpairs/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------------------------------ main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_8k", choices=["prefill_3k", "prefill_8k", "prefill_2x32k_heavy"])
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    line = gpu_arm(args, rank, world, local_rank, dist)
+    if rank == 0 and not args.no_cpu_baseline:
+        v, desc = cpu_oracle_sample(args.workload, n_rows=24)
+        line["cpu_baseline"] = {"value": round(v, 6), "unit": "Gpairs/s", "cores": _cpu_threads(), "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

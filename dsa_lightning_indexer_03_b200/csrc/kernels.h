@@ -1,0 +1,100 @@
+// kernels.h -- launchers of the library's CUDA kernels (internal to the .so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace dsa {
+
+// ---------------------------------------------------------------- projections
+struct ProjKwEpilogue {
+  int M;                          // tokens
+  __nv_bfloat16* key_cache;       // [cache_rows, 128]
+  int64_t cache_rows;
+  float* w_out;                   // [M, 32]
+  const int32_t* positions;       // [M]
+  const int32_t* q_seq_offsets;   // [B+1]
+  int B;
+  const int64_t* cache_offsets;   // [B+1]
+  const float* gamma;             // [128]
+  const float* beta;              // [128]
+  float eps;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+// q_out[M, 4096] = bf16(A[M,K] * Bt[4096,K]^T); tmA box {64,128}, tmB box {64,256}
+cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N,
+                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s);
+
+// [k~ | w] = A[M,K] * Bt[160,K]^T with the key LayerNorm / scatter epilogue; tmB box {64,160}
+cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K, const ProjKwEpilogue& e,
+                           cudaStream_t s);
+
+cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,
+                            const float* beta, float eps, cudaStream_t s);
+
+// dst[N, K] = src[K, N]^T (bf16), dst row stride K, written at row offset dst_row0
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, int K, int N, __nv_bfloat16* dst, int dst_row0,
+                                  cudaStream_t s);
+
+// ---------------------------------------------------------------- score + top-k
+constexpr int kCandCap = 4096;                 // candidates a query may hold before compaction
+constexpr int kCandStride = kCandCap + kTopK;  // + staging area for the compaction
+constexpr int kMaxChunks = 16;                 // key chunks per query on the split-key path
+constexpr int kMinChunk = 8192;                // shortest key chunk on the split-key path
+constexpr int kSplitMaxTokens = 256;           // split-key path is offered up to this many queries
+constexpr int kPrefillQ = 8;                   // queries per work item on the prefill path
+
+struct WorkItem {
+  int32_t t0;       // first query token
+  int32_t nq;       // queries in the item
+  int32_t b;        // sequence
+  int32_t k_begin;  // first key position scored (multiple of 128)
+  int32_t k_end;    // one past the last key position any query of the item scores
+  int32_t chunk;    // -1: writes the output rows; >= 0: key chunk of a split query (writes partials)
+  int32_t pad0, pad1;
+};
+
+struct TopkWorkspace {
+  WorkItem* items;
+  int max_items;
+  int* n_items;
+  int* work_counter;
+  int* seq_base;     // [max(B, T) + 2]
+  int* pos_eff;      // [T] validated positions, -1 for an invalid query
+  int* tok_nchunks;  // [T] key chunks of each query on the split-key path
+  uint32_t* cand_keys;
+  int32_t* cand_idx;
+  int cand_slots;    // CTA slots (x kPrefillQ queries each)
+  uint32_t* part_keys;
+  int32_t* part_idx;
+  int part_tokens;
+  int* err;
+};
+
+struct TopkArgs {
+  int T, B;
+  int64_t cache_rows;
+  const __nv_bfloat16* q;
+  const float* w;
+  const int32_t* positions;
+  const int32_t* q_seq_offsets;
+  const __nv_bfloat16* key_cache;
+  const int64_t* cache_offsets;
+  int32_t* idx_out;
+  float* score_out;
+  bool split;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtensorMap& tmQ1, const CUtensorMap& tmQ8,
+                        const CUtensorMap& tmK, int num_sms, cudaStream_t s);
+
+cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace dsa

@@ -1,0 +1,342 @@
+// proj.cu -- the indexer's three projections on the tcgen05 tensor cores.
+//
+// 'Sparse / compressed attn' row (Kimi K3.1 Pro): queries from the 1,536-dim
+// query latent (1,536 -> 4,096 = 32 heads x 128), one shared 128-dim key from
+// the hidden state with a LayerNorm, per-head weights from a 7,168 -> 32
+// projection.  The key and weight projections read the same hidden row, so
+// they run as one GEMM with N = 128 + 32 = 160 whose epilogue applies the
+// LayerNorm to columns 0..127 (one TMEM lane = one token, so each epilogue
+// thread owns its whole 128-wide row), casts to bf16 and scatters the row to
+// its key-cache slot, and stores columns 128..159 as fp32 head weights.
+//
+// Kernel shape: one 128-row output tile per CTA; warp 0 issues TMA loads of
+// 64-wide K slices of A and B into a STAGES-deep ring (128-byte swizzle),
+// warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator,
+// warps 2..5 drain TMEM (tcgen05.ld 32x32b) in the epilogue.
+
+#include "kernels.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kABytes = kBM * kBK * 2;  // 16 KB per stage
+constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
+
+enum { EPI_Q = 0, EPI_KW = 1 };
+
+struct ProjParams {
+  int M, K;
+  __nv_bfloat16* q_out;  // EPI_Q
+  int ldq;
+  ProjKwEpilogue kw;     // EPI_KW
+  int* err;
+  uint64_t timeout_ns;
+};
+
+template <int BN, int STAGES>
+struct ProjSmem {
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarOff = STAGES * kStageBytes;
+  static constexpr int kMiscOff = kBarOff + 8 * (2 * STAGES + 2);
+  static constexpr int kGammaOff = (kMiscOff + 16 + 15) / 16 * 16;
+  static constexpr int kTotal = kGammaOff + 2 * 128 * 4 + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// waits without looking at the abort flag (used only to drain in-flight work)
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (global_timer_ns() - t0 > kDrainNs) break;
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    proj_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     ProjParams p) {
+  using L = ProjSmem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = BN <= 32 ? 32 : BN <= 64 ? 64 : BN <= 128 ? 128 : 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  float* s_gamma = reinterpret_cast<float*>(smem + L::kGammaOff);
+  float* s_beta = s_gamma + 128;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kBM;
+  const int n0 = blockIdx.x * BN;
+  const int nk = p.K / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (EPI == EPI_KW && threadIdx.x >= 64) {
+    const int i = threadIdx.x - 64;
+    s_gamma[i] = p.kw.gamma[i];
+    s_beta[i] = p.kw.beta[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{p.err, abort_flag, p.timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+        tma_load_2d(sA + s * kABytes, &tmA, &full[s], kb * kBK, m0);
+        tma_load_2d(sB + s * L::kBBytes, &tmB, &full[s], kb * kBK, n0);
+        issued = kb + 1;
+      }
+      if (*abort_flag) {  // let the loads still in flight land before the CTA exits
+        for (int kb = (issued > STAGES ? issued - STAGES : 0); kb < issued; ++kb)
+          drain_wait(&full[kb % STAGES], (kb / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES;
+        if (!mbar_wait(&full[s], (kb / STAGES) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * kABytes);
+        const uint32_t b = smem_u32(sB + s * L::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          umma_bf16(tmem, umma_desc_sw128(a + kk * 32), umma_desc_sw128(b + kk * 32), idesc, (kb | kk) != 0);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+      umma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+  } else {
+    // epilogue: warps 2..5; TMEM lane quadrant = warp % 4
+    const int qd = warp & 3;
+    const int row = m0 + qd * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, wc));
+    tc_fence_after();
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    if (ok) {
+      if constexpr (EPI == EPI_Q) {
+        __nv_bfloat16* dst = p.q_out + static_cast<size_t>(row) * p.ldq + n0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32cols(tbase + c * 32, r);
+          tmem_ld_wait(r);
+          if (row < p.M) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 pk;
+              pk.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              pk.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              pk.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              pk.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              d4[v] = pk;
+            }
+          }
+        }
+      } else {
+        // key: LayerNorm over columns 0..127 of this token's row, fp32 math
+        float x[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld_32cols(tbase + c * 32, r);
+          tmem_ld_wait(r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[c * 32 + i] = __uint_as_float(r[i]);
+        }
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) sum += x[i];
+        const float mean = sum * (1.0f / 128.0f);
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const float d = x[i] - mean;
+          ss = fmaf(d, d, ss);
+        }
+        const float rstd = rsqrtf(ss * (1.0f / 128.0f) + p.kw.eps);
+        uint32_t wr[32];
+        tmem_ld_32cols(tbase + 128, wr);
+        tmem_ld_wait(wr);
+        if (row < p.M) {
+          const int t = row;
+          const int pos = p.kw.positions[t];
+          // sequence of token t: the last b with q_seq_offsets[b] <= t
+          int lo = 0, hi = p.kw.B - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.kw.q_seq_offsets[mid] <= t) lo = mid;
+            else hi = mid - 1;
+          }
+          const int64_t base = p.kw.cache_offsets[lo];
+          const int64_t len = p.kw.cache_offsets[lo + 1] - base;
+          if (pos >= 0 && pos < len && base >= 0 && base + pos < p.kw.cache_rows) {
+            uint4* d4 = reinterpret_cast<uint4*>(p.kw.key_cache + static_cast<size_t>(base + pos) * kHeadDim);
+#pragma unroll
+            for (int v = 0; v < 16; ++v) {
+              float y[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const int d = 8 * v + i;
+                y[i] = fmaf((x[d] - mean) * rstd, s_gamma[d], s_beta[d]);
+              }
+              uint4 pk;
+              pk.x = pack_bf16x2(y[0], y[1]);
+              pk.y = pack_bf16x2(y[2], y[3]);
+              pk.z = pack_bf16x2(y[4], y[5]);
+              pk.w = pack_bf16x2(y[6], y[7]);
+              d4[v] = pk;
+            }
+          } else {
+            atomicOr(p.err, kErrBounds);
+          }
+          float4* w4 = reinterpret_cast<float4*>(p.kw.w_out + static_cast<size_t>(t) * kHeads);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            w4[v] = make_float4(__uint_as_float(wr[4 * v]), __uint_as_float(wr[4 * v + 1]),
+                                __uint_as_float(wr[4 * v + 2]), __uint_as_float(wr[4 * v + 3]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- key LayerNorm on its own
+__global__ void __launch_bounds__(256) key_norm_kernel(int64_t n, const float* __restrict__ raw,
+                                                       __nv_bfloat16* __restrict__ out, const float* __restrict__ gamma,
+                                                       const float* __restrict__ beta, float eps) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const float4 v = reinterpret_cast<const float4*>(raw + row * kHeadDim)[lane];
+  float s = v.x + v.y + v.z + v.w;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s * (1.0f / 128.0f);
+  const float d0 = v.x - mean, d1 = v.y - mean, d2 = v.z - mean, d3 = v.w - mean;
+  float ss = d0 * d0 + d1 * d1 + d2 * d2 + d3 * d3;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rstd = rsqrtf(ss * (1.0f / 128.0f) + eps);
+  const float4 g = reinterpret_cast<const float4*>(gamma)[lane];
+  const float4 b = reinterpret_cast<const float4*>(beta)[lane];
+  uint2 pk;
+  pk.x = pack_bf16x2(fmaf(d0 * rstd, g.x, b.x), fmaf(d1 * rstd, g.y, b.y));
+  pk.y = pack_bf16x2(fmaf(d2 * rstd, g.z, b.z), fmaf(d3 * rstd, g.w, b.w));
+  reinterpret_cast<uint2*>(out + row * kHeadDim)[lane] = pk;
+}
+
+// ---------------------------------------------------------------- weight re-layout at create
+__global__ void transpose_bf16_kernel(const __nv_bfloat16* __restrict__ src, int K, int N,
+                                      __nv_bfloat16* __restrict__ dst, int dst_row0) {
+  __shared__ __nv_bfloat16 tile[32][33];
+  const int k0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int k = k0 + i, nn = n0 + threadIdx.x;
+    if (k < K && nn < N) tile[i][threadIdx.x] = src[static_cast<size_t>(k) * N + nn];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    const int nn = n0 + i, k = k0 + threadIdx.x;
+    if (k < K && nn < N) dst[static_cast<size_t>(dst_row0 + nn) * K + k] = tile[threadIdx.x][i];
+  }
+}
+
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_proj(const CUtensorMap& tmA, const CUtensorMap& tmB, const ProjParams& p, int n_tiles,
+                        cudaStream_t s) {
+  using L = ProjSmem<BN, STAGES>;
+  auto kern = proj_gemm_kernel<BN, STAGES, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+  if (e != cudaSuccess) return e;
+  dim3 grid(n_tiles, (p.M + kBM - 1) / kBM);
+  kern<<<grid, 192, L::kTotal, s>>>(tmA, tmB, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N,
+                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s) {
+  ProjParams p{};
+  p.M = M;
+  p.K = K;
+  p.q_out = q_out;
+  p.ldq = N;
+  p.err = err;
+  p.timeout_ns = timeout_ns;
+  return launch_proj<256, 4, EPI_Q>(tmA, tmB, p, N / 256, s);
+}
+
+cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K, const ProjKwEpilogue& e,
+                           cudaStream_t s) {
+  ProjParams p{};
+  p.M = e.M;
+  p.K = K;
+  p.kw = e;
+  p.err = e.err;
+  p.timeout_ns = e.timeout_ns;
+  return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
+}
+
+cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,
+                            const float* beta, float eps, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 7) / 8;
+  key_norm_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(n, raw, out, gamma, beta, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, int K, int N, __nv_bfloat16* dst, int dst_row0,
+                                  cudaStream_t s) {
+  dim3 grid((N + 31) / 32, (K + 31) / 32);
+  transpose_bf16_kernel<<<grid, dim3(32, 8), 0, s>>>(src, K, N, dst, dst_row0);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -1,0 +1,175 @@
+/*
+ * dsa_indexer.h -- C ABI of the B200 (sm_100a) DSA lightning indexer.
+ *
+ * The operation (archdiff.com compare pages on Kimi K3.1 Pro, component table,
+ * 'Sparse / compressed attn' row, Kimi K3.1 Pro column): every MLA layer owns an
+ * indexer with 32 heads x 128 dims.  Per token t it forms
+ *     q_t = q_latent_t W_q           (1,536 -> 4,096 = 32 heads x 128),
+ *     k_t = LayerNorm(hidden_t W_k)  (7,168 -> 128, one key shared by all heads),
+ *     w_t = hidden_t W_w             (7,168 -> 32 per-head weights),
+ * scores every causal prior token s of its sequence with
+ *     I[t,s] = sum_h w_t[h] * ReLU(q_t[h] . k_s)
+ * and keeps the 2,048 highest-scoring tokens.  The key norm is a LayerNorm
+ * ('QK-Clip and normalized latents; LayerNorm on the indexer key' row), no
+ * rotary step is applied ('Partial RoPE / NoPE' row: index_rope_dim = 0), the
+ * weights are BF16 ('FP8 -> FP4 training' row) and the whole prefix is scored
+ * ('Long-context extension' row).
+ *
+ * Conventions for every entry point:
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory, 16-byte
+ *     aligned, densely packed row-major.  bf16 tensors are passed as void*.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous on that stream; the library never synchronises the host,
+ *     except dsa_indexer_create / _destroy / _device_error.
+ *   - Host-detectable argument errors return a status and launch nothing.
+ *     Problems only the device can see (a position outside its sequence's key
+ *     cache, malformed offsets, a pipeline wait that ran out) set bits in the
+ *     handle's device error word and leave the affected outputs in a defined
+ *     padded state; dsa_indexer_device_error() reports and clears them.
+ *   - A handle may be used from one stream at a time (its workspace is shared
+ *     by consecutive calls and ordered by that stream).
+ */
+#ifndef DSA_INDEXER_H
+#define DSA_INDEXER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_INDEXER_ABI_VERSION 1
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,    /* NULL/misaligned pointer, bad size, bad config */
+  DSA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement */
+  DSA_ERR_CUDA = 3,           /* a CUDA runtime/driver call or a launch failed */
+  DSA_ERR_OOM = 4,            /* device allocation failed at create */
+  DSA_ERR_WORKSPACE = 5,      /* T exceeds the handle's max_tokens */
+  DSA_ERR_DEVICE_TIMEOUT = 6, /* a bounded device-side wait ran out (kernel exited early) */
+  DSA_ERR_DEVICE_BOUNDS = 7   /* a position / offset was outside its sequence's cache rows */
+} dsa_status_t;
+
+/* flags of dsa_indexer_topk */
+#define DSA_TOPK_SORTED   1u  /* rows ordered by (score desc, position asc), padding last */
+#define DSA_TOPK_SPLIT    2u  /* force the split-key path (one query per work item, key chunks merged) */
+#define DSA_TOPK_NO_SPLIT 4u  /* never use the split-key path */
+
+typedef struct dsa_indexer* dsa_indexer_t;
+
+/* Create-time configuration.  Only n_heads = 32, head_dim = 128 and
+ * top_k = 2048 are implemented (other values: DSA_ERR_UNSUPPORTED);
+ * hidden_dim and q_latent_dim must be positive multiples of 64. */
+typedef struct {
+  int32_t hidden_dim;    /* 7168: width of the hidden state feeding W_k and W_w */
+  int32_t q_latent_dim;  /* 1536: width of the MLA query latent feeding W_q */
+  int32_t n_heads;       /* 32 */
+  int32_t head_dim;      /* 128 */
+  int32_t top_k;         /* 2048 */
+  float ln_eps;          /* LayerNorm epsilon of the key norm; 1e-6 by default */
+  int64_t max_tokens;    /* largest T passed to _topk; sizes the handle's workspace */
+} dsa_indexer_config_t;
+
+/* Fills *cfg with the Kimi K3.1 Pro indexer dimensions (above) and
+ * max_tokens = 131072. */
+void dsa_indexer_default_config(dsa_indexer_config_t* cfg);
+
+/* Creates a handle for one layer's indexer on the current CUDA device.
+ * Weight pointers are device bf16 tensors stored (in x out), row-major:
+ *   W_q [q_latent_dim, n_heads*head_dim]   (head h = columns h*128 .. h*128+127)
+ *   W_k [hidden_dim, head_dim], W_w [hidden_dim, n_heads],
+ *   ln_gamma [head_dim], ln_beta [head_dim].
+ * The weights are copied (re-laid out for the tensor cores) into memory the
+ * handle owns; the caller may free its copies on return.  Synchronous.
+ * Returns DSA_ERR_INVALID_ARG / _UNSUPPORTED / _OOM / _CUDA on failure, in
+ * which case *out is left NULL. */
+dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q, const void* W_k,
+                                const void* W_w, const void* ln_gamma, const void* ln_beta,
+                                dsa_indexer_t* out);
+
+/* Frees the handle and its device memory (synchronises the device first). */
+dsa_status_t dsa_indexer_destroy(dsa_indexer_t h);
+
+/* Projections of T tokens belonging to B sequences ('Sparse / compressed attn'
+ * row: query latent 1,536 -> 4,096, hidden -> one LayerNorm'd 128-dim key,
+ * hidden 7,168 -> 32 head weights).
+ *   hidden        bf16 [T, hidden_dim]
+ *   q_latent      bf16 [T, q_latent_dim]
+ *   positions     int32 [T], position of token t inside its sequence
+ *   q_seq_offsets int32 [B+1], tokens of sequence b are q_seq_offsets[b] .. [b+1]-1
+ *   key_cache     bf16 [cache_rows, head_dim]; k_t is written to row
+ *                 cache_offsets[b] + positions[t] (one 256-byte row per token)
+ *   cache_rows    number of rows the key_cache allocation holds
+ *   cache_offsets int64 [B+1], key-cache rows of sequence b are
+ *                 cache_offsets[b] .. cache_offsets[b+1]-1, with
+ *                 0 <= cache_offsets[b] <= cache_offsets[b+1] <= cache_rows
+ *   q_out         bf16 [T, n_heads*head_dim] = bf16(q_latent W_q), fp32 accumulate
+ *   w_out         fp32 [T, n_heads]          = hidden W_w, fp32 accumulate
+ * The key is k = bf16(gamma * (x - mean) / sqrt(var + eps) + beta) with
+ * x = hidden W_k kept in fp32 and the biased variance.  A token whose position
+ * lies outside [0, rows of its sequence) gets no key row and sets
+ * DSA_ERR_DEVICE_BOUNDS.  T = 0 is a no-op. */
+dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
+                                 const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                                 void* key_cache, int64_t cache_rows, const int64_t* cache_offsets, void* q_out,
+                                 float* w_out, void* stream);
+
+/* LayerNorm + bf16 cast of n pre-norm key rows (the key-norm step of the
+ * projection on its own, for callers that compute hidden W_k elsewhere or fill
+ * a cache from stored pre-norm keys).
+ *   raw_keys fp32 [n, head_dim] -> keys_out bf16 [n, head_dim]. */
+dsa_status_t dsa_indexer_key_norm(dsa_indexer_t h, int64_t n, const float* raw_keys, void* keys_out,
+                                  void* stream);
+
+/* Score + top-k of T query tokens ('Sparse / compressed attn' row: I = sum_h
+ * w_h ReLU(q_h . k), top 2,048 per query; 'Long-context extension' row: the
+ * whole causal prefix is scored).
+ *   q          bf16 [T, n_heads, head_dim]   (as written by _project)
+ *   w          fp32 [T, n_heads]
+ *   positions, q_seq_offsets, B, cache_rows, cache_offsets: as for _project
+ *   key_cache  bf16 [cache_rows, head_dim]
+ *   idx_out    int32 [T, top_k]
+ *   score_out  fp32 [T, top_k] or NULL
+ * Query t at position p of sequence b scores keys s = 0..p (inclusive) read
+ * from row cache_offsets[b] + s.  Indices are positions inside the sequence.
+ * If p + 1 <= top_k the row is exactly [0, 1, ..., p, -1, ...] (scores in
+ * the same order, -inf in the padding).  Otherwise the row holds the top_k
+ * positions of highest score, in unspecified order (DSA_TOPK_SORTED: score
+ * descending, position ascending); among exactly equal scores at the cut any
+ * subset may be kept.  The T x S score matrix is never written to memory.
+ * Flags: DSA_TOPK_SORTED, DSA_TOPK_SPLIT, DSA_TOPK_NO_SPLIT (default: the
+ * split-key path when T <= 256).  A query whose position is outside its
+ * sequence's cache rows gets an all-padding row and sets
+ * DSA_ERR_DEVICE_BOUNDS; malformed offsets set it too and leave the output
+ * rows unwritten.  Returns DSA_ERR_WORKSPACE if T or B exceeds max_tokens,
+ * and DSA_ERR_UNSUPPORTED for DSA_TOPK_SPLIT with T > 256. */
+dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const float* w,
+                              const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                              const void* key_cache, int64_t cache_rows, const int64_t* cache_offsets,
+                              int32_t* idx_out,
+                              float* score_out, uint32_t flags, void* stream);
+
+/* Synchronises the device, then returns DSA_OK or the first device-side error
+ * recorded since the last call (DSA_ERR_DEVICE_BOUNDS, DSA_ERR_DEVICE_TIMEOUT)
+ * and clears the error word. */
+dsa_status_t dsa_indexer_device_error(dsa_indexer_t h);
+
+/* Launches one kernel that waits on a barrier nothing will ever signal, with a
+ * device-side limit of timeout_ns nanoseconds, synchronises the stream and
+ * returns the status the kernel reported: DSA_ERR_DEVICE_TIMEOUT when the
+ * bounded wait works.  Used to test the failure path without hanging a GPU. */
+dsa_status_t dsa_indexer_selftest_wait_timeout(int64_t timeout_ns, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* dsa_indexer_status_string(dsa_status_t s);
+
+/* DSA_INDEXER_ABI_VERSION of the loaded library. */
+int32_t dsa_indexer_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_INDEXER_H */

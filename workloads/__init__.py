@@ -22,4 +22,5 @@ from .generate import (  # noqa: F401
     make_decode,
     heavy_hitter_rows,
     causal_pairs,
+    make_scoring_inputs,
 )

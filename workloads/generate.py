@@ -157,6 +157,17 @@ def heavy_hitter_rows(seed: int, cache_offsets: torch.Tensor, frac: float = 0.01
     return torch.cat(rows).to(torch.int64) if rows else torch.zeros(0, dtype=torch.int64)
 
 
+def make_scoring_inputs(seed: int, n_queries: int, n_keys: int, n_heads: int = 32, head_dim: int = 128,
+                        key_scale: float = 1.0):
+    """Direct inputs of the score + top-k step, for testing it on its own:
+    q bf16 N(0,1) [T, n_heads, head_dim], keys bf16 N(0, key_scale^2) [S, head_dim]
+    (the scale of LayerNorm outputs), w fp32 N(0,1) [T, n_heads]."""
+    q = _normal(_gen(seed, _S_QLAT, 1), (n_queries, n_heads, head_dim)).to(torch.bfloat16)
+    keys = _normal(_gen(seed, _S_RAWK, 1), (n_keys, head_dim), key_scale).to(torch.bfloat16)
+    w = _normal(_gen(seed, _S_WW, 1), (n_queries, n_heads))
+    return q, keys, w
+
+
 def causal_pairs(positions: torch.Tensor) -> int:
     """Number of (query, key) pairs a causal pass scores: sum over queries of pos + 1."""
     return int(positions.to(torch.int64).sum()) + int(positions.numel())
