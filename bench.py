@@ -178,8 +178,7 @@ def _prefill_step(st, ev=None):
 def _setup_decode(d, seed_offset, device):
     cfg = W.WORKLOADS["decode_64"]
     wts = W.make_weights(cfg["weight_seed"])
-    g = torch.Generator().manual_seed(1000 + seed_offset)
-    lengths = torch.randint(cfg["L_min"], cfg["L_max"] + 1, (cfg["batch"],), generator=g)
+    lengths = W.decode_lengths(cfg["act_seed"] + seed_offset, cfg["batch"], cfg["L_min"], cfg["L_max"])
     batch = W.make_decode(cfg["act_seed"] + seed_offset, lengths=torch.ones_like(lengths))  # new tokens only
     to = lambda t: t.to(device).contiguous()  # noqa: E731
     ix = d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta), max_tokens=256)
@@ -358,10 +357,11 @@ def gpu_arm(args, rank, world, local_rank, dist):
 
 # ------------------------------------------------------------------------------------------ CPU oracle arm
 
-def cpu_oracle_sample(name, n_rows=24, seed=0):
-    """The oracle as it stands on a bounded sample of the workload: keys of the
-    whole prefix plus q/w/top-k of n_rows query rows spread over the positions.
-    Returns (Gpairs/s, description)."""
+def cpu_oracle_sample(name, proj_tokens=256, n_rows=12, seed=0):
+    """The oracle as it stands, on bounded samples of the workload: its projection
+    of `proj_tokens` tokens (seconds per token) and its score + top-k of `n_rows`
+    query rows spread over the positions (seconds per causal pair), extrapolated
+    to the whole workload.  Returns (Gpairs/s, description, seconds spent)."""
     import numpy as np
 
     import oracle
@@ -369,42 +369,52 @@ def cpu_oracle_sample(name, n_rows=24, seed=0):
     wts = W.make_weights(cfg["weight_seed"])
     batch = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
     T = batch.hidden.shape[0]
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(T, size=min(n_rows, T), replace=False))
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    Wq, Wk, Ww, g, b = f(wts.W_q), f(wts.W_k), f(wts.W_w), f(wts.gamma), f(wts.beta)
+    hid = f(batch.hidden[:proj_tokens])
+    qlat = f(batch.q_latent[:proj_tokens])
     t0 = time.perf_counter()
-    max_pos = int(batch.positions[rows].max())
-    _, k, _ = oracle.project(f(batch.hidden[:max_pos + 1]), f(batch.q_latent[:max_pos + 1]), f(wts.W_q), f(wts.W_k),
-                             f(wts.W_w), f(wts.gamma), f(wts.beta))
-    q, _, w = oracle.project(f(batch.hidden[rows]), f(batch.q_latent[rows]), f(wts.W_q), f(wts.W_k), f(wts.W_w),
-                             f(wts.gamma), f(wts.beta))
+    oracle.project(hid, qlat, Wq, Wk, Ww, g, b)
+    t_proj = (time.perf_counter() - t0) / proj_tokens
+    # score + top-k rows: keys = the oracle's key norm of seeded pre-norm rows (the
+    # workload's key distribution), q / w of the sampled rows from the oracle projection
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(np.arange(T // 2, T), size=n_rows, replace=False))
+    raw = W.make_decode(cfg["act_seed"], lengths=[T]).raw_keys
+    keys = oracle.key_norm(raw.to(torch.float64).numpy(), g, b)
+    q, _, w = oracle.project(f(batch.hidden[rows]), f(batch.q_latent[rows]), Wq, Wk, Ww, g, b)
     qq = np.zeros((T, 32, 128))
     ww = np.zeros((T, 32))
     qq[rows] = q
     ww[rows] = w
-    oracle.topk(qq, ww, batch.positions.numpy(), batch.q_seq_offsets.numpy(), k, np.array([0, k.shape[0]]),
-                rows=rows)
-    dt = time.perf_counter() - t0
-    pairs = int((batch.positions[rows].to(torch.int64) + 1).sum())
-    return pairs / dt / 1e9, f"{len(rows)} query rows of {name} (keys of their whole prefix projected), {dt:.1f} s"
+    t0 = time.perf_counter()
+    oracle.topk(qq, ww, batch.positions.numpy(), batch.q_seq_offsets.numpy(), keys, np.array([0, T]), rows=rows)
+    t_topk = time.perf_counter() - t0
+    pairs_s = int((batch.positions[rows].to(torch.int64) + 1).sum())
+    total_pairs = W.causal_pairs(batch.positions)
+    t_full = T * t_proj + total_pairs * (t_topk / pairs_s)
+    desc = (f"{name}: projection of {proj_tokens} tokens ({t_proj * 1e3:.2f} ms/token) and score+top-k of "
+            f"{n_rows} query rows ({pairs_s} causal pairs, {t_topk:.2f} s), extrapolated to all {T} tokens "
+            f"/ {total_pairs} pairs ({t_full:.0f} s)")
+    return total_pairs / t_full / 1e9, desc, t_proj * proj_tokens + t_topk
 
 
 def reference_arm(args):
     vals = []
     desc = ""
-    for _ in range(args.warmup):
-        cpu_oracle_sample(args.workload, n_rows=4)
-    t0 = time.perf_counter()
+    for _ in range(min(args.warmup, 1)):
+        cpu_oracle_sample(args.workload, proj_tokens=32, n_rows=2)
+    wall = 0.0
     for i in range(args.steps):
-        v, desc = cpu_oracle_sample(args.workload, n_rows=8, seed=i)
+        v, desc, spent = cpu_oracle_sample(args.workload, seed=i)
         vals.append(v)
-    wall = time.perf_counter() - t0
+        wall += spent
     value = statistics.mean(vals)
     cores = _cpu_threads()
     return {
         "impl": "reference",
         "metric": METRIC,
-        "value": round(value, 6),
+        "value": float(f"{value:.6g}"),
         "unit": "Gpairs/s",
         "n_gpus": 1,
         "steps": args.steps,
@@ -417,9 +427,10 @@ def reference_arm(args):
         "data": "synthetic",
         "config": {"workload": args.workload, "batch": len(W.WORKLOADS[args.workload]["seq_lens"]),
                    "seq_len": W.WORKLOADS[args.workload]["seq_lens"][0], "top_k": 2048},
-        "cpu_baseline": {"value": round(value, 6), "unit": "Gpairs/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": float(f"{value:.6g}"), "unit": "Gpairs/s", "cores": cores, "kind": "oracle",
                          "sample": desc},
-        "e2e": {"value": round(value, 6), "unit": "Gpairs/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": float(f"{value:.6g}"), "unit": "Gpairs/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
     }
 
 
@@ -455,8 +466,8 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     line = gpu_arm(args, rank, world, local_rank, dist)
     if rank == 0 and not args.no_cpu_baseline:
-        v, desc = cpu_oracle_sample(args.workload, n_rows=24)
-        line["cpu_baseline"] = {"value": round(v, 6), "unit": "Gpairs/s", "cores": _cpu_threads(), "kind": "oracle",
+        v, desc, _ = cpu_oracle_sample(args.workload)
+        line["cpu_baseline"] = {"value": float(f"{v:.6g}"), "unit": "Gpairs/s", "cores": _cpu_threads(), "kind": "oracle",
                                 "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)

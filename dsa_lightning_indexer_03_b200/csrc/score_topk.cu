@@ -21,12 +21,14 @@
 //              (quadrant, lane) owns one key; per query it loads that query's 32
 //              head columns (tcgen05.ld 32x32b.x32), applies ReLU and the fp32
 //              head weights in registers, masks s > pos, and appends (score, s)
-//              to the query's candidate list if the score reaches the query's
-//              running threshold (warp ballot + one shared atomic per warp).
-//              A list that nears its capacity is compacted to its best 2,048
-//              (radix select in shared memory), which raises the threshold.
-//              At the end of the item each list is reduced to exactly the top
-//              2,048 and written out.
+//              to its own append area of the query's candidates if the score
+//              reaches the query's running threshold (warp ballot; the counts
+//              stay warp-uniform in registers, no atomics).  When an append area
+//              nears its capacity, the query's keep set and append areas are
+//              compacted into the other keep set holding the exact best 2,048
+//              (histogram selection in shared memory), which raises the
+//              threshold.  At the end of the item each query's candidates are
+//              reduced to exactly the top 2,048 and written out.
 
 #include "kernels.h"
 
@@ -61,108 +63,329 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------------------------------
-// Radix select over `n` order-preserving keys held in shared memory by a group of NT
-// threads (tid = 0..NT-1, named barrier `bar`).  Returns the k-th largest key K*
-// (1 <= k <= n); *n_above receives the number of keys strictly greater than K*.
-// Four passes of 8 bits, most significant first; each pass histograms the keys that
-// match the prefix found so far (warp-aggregated shared atomics).
+// Group-wide helpers for a group of NT threads (tid = 0..NT-1) that synchronise on the
+// named barrier `bar`.
+
+// Sum of v over the threads of the group with a larger tid.
 template <int NT>
-__device__ uint32_t radix_kth(const uint32_t* skeys, int n, int k, uint32_t* hist, int* sh, int tid, int bar,
-                              int* n_above) {
-  const int lane = tid & 31;
-  uint32_t prefix = 0, mask = 0;
-  int need = k;
-#pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += NT) hist[i] = 0;
-    named_bar_sync(bar, NT);
-    for (int base = 0; base < n; base += NT) {
-      const int e = base + tid;
-      const uint32_t key = (e < n) ? skeys[e] : 0u;
-      const bool act = (e < n) && ((key & mask) == prefix);
-      const uint32_t bin = act ? ((key >> shift) & 255u) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
-    }
-    named_bar_sync(bar, NT);
-    if (tid < 32) {
-      // lane l owns bins 255-8l .. 248-8l (from the top)
-      uint32_t c[8], tot = 0;
+__device__ __forceinline__ uint32_t group_suffix_excl(uint32_t v, int tid, uint32_t* scratch, int bar) {
+  const int lane = tid & 31, wid = tid >> 5;
+  uint32_t x = v;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        c[i] = hist[255 - 8 * lane - i];
-        tot += c[i];
-      }
-      uint32_t incl = tot;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-      }
-      const uint32_t excl = incl - tot;
-      if (excl < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= incl) {
-        uint32_t cum = excl;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (cum + c[i] >= static_cast<uint32_t>(need)) {
-            sh[0] = 255 - 8 * lane - i;
-            sh[1] = static_cast<int>(cum);
-            break;
-          }
-          cum += c[i];
-        }
-      }
-    }
-    named_bar_sync(bar, NT);
-    const uint32_t bin = static_cast<uint32_t>(sh[0]);
-    need -= sh[1];
-    prefix |= bin << shift;
-    mask |= 255u << shift;
-    named_bar_sync(bar, NT);
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
+    if (lane + off < 32) x += y;
   }
-  *n_above = k - need;
-  return prefix;
+  if (lane == 0) scratch[wid] = x;  // warp total
+  named_bar_sync(bar, NT);
+  uint32_t wa = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w)
+    if (w > wid) wa += scratch[w];
+  named_bar_sync(bar, NT);
+  return wa + x - v;
 }
 
-// Emits the top k of n candidate (key, idx) pairs: every key > kth and the first
-// (k - n_above) keys equal to kth.  sink(slot, key, e) is called once per kept
-// entry with a distinct slot in [0, k).  ctr[0..1] are zeroed shared counters.
-template <int NT, class Sink>
-__device__ void emit_topk(const uint32_t* skeys, int n, int k, uint32_t kth, int n_above, int* ctr, int tid,
-                          Sink sink) {
-  const int lane = tid & 31;
-  const int ties = k - n_above;
-  for (int base = 0; base < n; base += NT) {
-    const int e = base + tid;
-    const uint32_t key = (e < n) ? skeys[e] : 0u;
-    const bool gt = (e < n) && key > kth;
-    const bool eq = (e < n) && key == kth;
-    const uint32_t bg = __ballot_sync(0xffffffffu, gt);
-    const uint32_t be = __ballot_sync(0xffffffffu, eq);
-    int b0 = 0, b1 = 0;
-    if (lane == 0) {
-      if (bg) b0 = atomicAdd(&ctr[0], __popc(bg));
-      if (be) b1 = atomicAdd(&ctr[1], __popc(be));
+// Group minimum of lo and maximum of hi.
+template <int NT>
+__device__ __forceinline__ void group_minmax(uint32_t& lo, uint32_t& hi, int tid, uint32_t* scratch, int bar) {
+  const int lane = tid & 31, wid = tid >> 5;
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    scratch[wid] = lo;
+    scratch[NT / 32 + wid] = hi;
+  }
+  named_bar_sync(bar, NT);
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    lo = min(lo, scratch[w]);
+    hi = max(hi, scratch[NT / 32 + w]);
+  }
+  named_bar_sync(bar, NT);
+}
+
+// k-th largest of n order-preserving keys held in shared memory (1 <= k <= n), all of
+// them inside [lo, hi].  Each round histograms the keys of the current window into at
+// most kHistBins bins of width 2^shift, locates the bin that holds the k-th largest,
+// and narrows the window to that bin; a round of width-1 bins ends it (at most three
+// rounds for 32-bit keys).  *n_above receives the number of keys strictly greater
+// than the returned key.
+constexpr int kHistBins = 2048;
+
+template <int NT>
+__device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo, uint32_t hi, uint32_t* hist,
+                                uint32_t* scratch, int* sh, int tid, int bar, int* n_above) {
+  constexpr int kBPT = kHistBins / NT;  // bins owned by one thread when locating the k-th
+  uint32_t base = lo, span = hi - lo;
+  int need = k, above_total = 0;
+#pragma unroll 1
+  while (true) {
+    const int shift = (span >> 11) ? 32 - __clz(static_cast<int>(span >> 11)) : 0;
+    const int nb = static_cast<int>(span >> shift) + 1;
+    for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
+    named_bar_sync(bar, NT);
+#pragma unroll 4
+    for (int e = tid; e < n; e += NT) {
+      const uint32_t d = keys[e] - base;
+      if (d <= span) atomicAdd(&hist[d >> shift], 1u);
     }
-    b0 = __shfl_sync(0xffffffffu, b0, 0);
-    b1 = __shfl_sync(0xffffffffu, b1, 0);
-    if (gt) sink(b0 + __popc(bg & lanemask_lt()), key, e);
-    if (eq) {
-      const int r = b1 + __popc(be & lanemask_lt());
-      if (r < ties) sink(n_above + r, key, e);
+    named_bar_sync(bar, NT);
+    const int b0 = tid * kBPT;
+    uint32_t c[kBPT];
+    uint32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < kBPT; ++i) {
+      c[i] = hist[b0 + i];
+      s += c[i];
+    }
+    const uint32_t above_t = group_suffix_excl<NT>(s, tid, scratch, bar);
+    if (above_t < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= above_t + s) {
+      uint32_t cum = above_t;
+#pragma unroll
+      for (int i = kBPT - 1; i >= 0; --i) {
+        if (cum + c[i] >= static_cast<uint32_t>(need)) {
+          sh[0] = b0 + i;
+          sh[1] = static_cast<int>(cum);
+          break;
+        }
+        cum += c[i];
+      }
+    }
+    named_bar_sync(bar, NT);
+    const int bstar = sh[0];
+    const int above = sh[1];
+    named_bar_sync(bar, NT);
+    need -= above;
+    above_total += above;
+    if (shift == 0 || nb <= 0) {
+      *n_above = above_total;
+      return base + static_cast<uint32_t>(bstar);
+    }
+    base += static_cast<uint32_t>(bstar) << shift;
+    span = (1u << shift) - 1u;
+  }
+}
+
+// Candidate views: a fixed set of slots (a multiple of 4), some of them empty.
+// load4(s0, k, i) fetches slots s0..s0+3 with 16-byte loads where the four are all
+// occupied and returns the occupied-slot mask; empty slots read key 0, position -1.
+constexpr int kSlots = 2 * kTopK;          // keep set + append area of one query
+constexpr int kWarpApp = kAppCap / 4;      // append slots of one epilogue warp
+
+// The candidates of one query in the score kernel: the current keep set (slots
+// 0..2047) followed by the four warps' append areas (512 slots each).
+struct QueryCands {
+  const uint32_t* kk;
+  const int32_t* ki;
+  const uint32_t* ak;
+  const int32_t* ai;
+  int cnt_k;
+  int cnt_w0, cnt_w1, cnt_w2, cnt_w3;   // scalars: a runtime-indexed array would live in local memory
+
+  __device__ __forceinline__ int cnt_w(int w) const {
+    return w == 0 ? cnt_w0 : w == 1 ? cnt_w1 : w == 2 ? cnt_w2 : cnt_w3;
+  }
+
+  template <bool kKeys, bool kIdx>
+  __device__ __forceinline__ uint32_t load4(int s0, uint4& k, int4& i) const {
+    const uint32_t* kp;
+    const int32_t* ip;
+    int local, cnt;
+    if (s0 < kTopK) {
+      kp = kk;
+      ip = ki;
+      local = s0;
+      cnt = cnt_k;
+    } else {
+      const int w = (s0 - kTopK) / kWarpApp;
+      local = (s0 - kTopK) % kWarpApp;
+      kp = ak + w * kWarpApp;
+      ip = ai + w * kWarpApp;
+      cnt = cnt_w(w);
+    }
+    if (local + 3 < cnt) {
+      if (kKeys) k = *reinterpret_cast<const uint4*>(kp + local);
+      if (kIdx) i = *reinterpret_cast<const int4*>(ip + local);
+      return 0xFu;
+    }
+    uint32_t m = 0;
+    uint32_t kv[4] = {0u, 0u, 0u, 0u};
+    int iv[4] = {-1, -1, -1, -1};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (local + j < cnt) {
+        m |= 1u << j;
+        if (kKeys) kv[j] = kp[local + j];
+        if (kIdx) iv[j] = ip[local + j];
+      }
+    }
+    if (kKeys) k = make_uint4(kv[0], kv[1], kv[2], kv[3]);
+    if (kIdx) i = make_int4(iv[0], iv[1], iv[2], iv[3]);
+    return m;
+  }
+  __device__ __forceinline__ int valid_count() const { return cnt_k + cnt_w0 + cnt_w1 + cnt_w2 + cnt_w3; }
+};
+
+// A dense list of n slots (n a multiple of 4); slots with position < 0 are empty.
+struct FlatCands {
+  const uint32_t* k;
+  const int32_t* i;
+  template <bool kKeys, bool kIdx>
+  __device__ __forceinline__ uint32_t load4(int s0, uint4& kv, int4& iv) const {
+    if (kKeys) kv = *reinterpret_cast<const uint4*>(k + s0);
+    if (kIdx) {
+      iv = *reinterpret_cast<const int4*>(i + s0);
+      return (iv.x >= 0 ? 1u : 0u) | (iv.y >= 0 ? 2u : 0u) | (iv.z >= 0 ? 4u : 0u) | (iv.w >= 0 ? 8u : 0u);
+    }
+    return 0xFu;
+  }
+};
+
+__device__ __forceinline__ uint32_t u4_get(const uint4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+__device__ __forceinline__ int i4_get(const int4& v, int j) {
+  return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
+}
+
+// Copies the keys of n slots into shared memory (empty slots as 0) and returns the
+// range of the occupied ones.
+template <int NT, class View>
+__device__ __forceinline__ void stage_view(const View& v, int n, uint32_t* skeys, int tid, uint32_t* scratch,
+                                           int bar, uint32_t& lo, uint32_t& hi) {
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
+#pragma unroll 2
+  for (int g = tid; g < n / 4; g += NT) {
+    uint4 k;
+    int4 dummy;
+    const uint32_t m = v.template load4<true, false>(4 * g, k, dummy);
+    reinterpret_cast<uint4*>(skeys)[g] = k;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (m & (1u << j)) {
+        lo = min(lo, u4_get(k, j));
+        hi = max(hi, u4_get(k, j));
+      }
     }
   }
+  group_minmax<NT>(lo, hi, tid, scratch, bar);
+  if (lo > hi) lo = hi;  // no occupied slot
+}
+
+// Emits the top k of the occupied slots: every key > kth and the first (k - n_above)
+// keys equal to kth.  sink(slot, key, pos) is called once per kept entry with a
+// distinct slot in [0, k).  ctr[0..1] are shared counters zeroed beforehand.
+template <int NT, class View, class Sink>
+__device__ void emit_view(const View& v, const uint32_t* skeys, int n, int k, uint32_t kth, int n_above, int* ctr,
+                          int tid, Sink sink) {
+  const int lane = tid & 31;
+  const int ties = k - n_above;
+  const uint32_t lt = lanemask_lt();
+  for (int base = 0; base < n / 4; base += NT) {
+    const int g = base + tid;
+    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
+    int4 ii = make_int4(-1, -1, -1, -1);
+    uint32_t m = 0;
+    if (g < n / 4) {
+      uint4 dummy;
+      m = v.template load4<false, true>(4 * g, dummy, ii);
+      kk = reinterpret_cast<const uint4*>(skeys)[g];
+    }
+    uint32_t bg[4], be[4];
+    int tg = 0, te = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = u4_get(kk, j);
+      const bool valid = (m >> j) & 1u;
+      bg[j] = __ballot_sync(0xffffffffu, valid && key > kth);
+      be[j] = __ballot_sync(0xffffffffu, valid && key == kth);
+      tg += __popc(bg[j]);
+      te += __popc(be[j]);
+    }
+    if (tg | te) {
+      int b0 = 0, b1 = 0;
+      if (lane == 0) {
+        if (tg) b0 = atomicAdd(&ctr[0], tg);
+        if (te) b1 = atomicAdd(&ctr[1], te);
+      }
+      b0 = __shfl_sync(0xffffffffu, b0, 0);
+      b1 = __shfl_sync(0xffffffffu, b1, 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if ((bg[j] >> lane) & 1u) sink(b0 + __popc(bg[j] & lt), u4_get(kk, j), i4_get(ii, j));
+        if ((be[j] >> lane) & 1u) {
+          const int r = b1 + __popc(be[j] & lt);
+          if (r < ties) sink(n_above + r, u4_get(kk, j), i4_get(ii, j));
+        }
+        b0 += __popc(bg[j]);
+        b1 += __popc(be[j]);
+      }
+    }
+  }
+}
+
+// Calls sink(rank, key, pos) for every occupied slot, ranks 0..count-1 (order unspecified).
+template <int NT, class View, class Sink>
+__device__ void compact_view(const View& v, int n, int* ctr, int tid, Sink sink) {
+  const int lane = tid & 31;
+  const uint32_t lt = lanemask_lt();
+  for (int base = 0; base < n / 4; base += NT) {
+    const int g = base + tid;
+    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
+    int4 ii = make_int4(-1, -1, -1, -1);
+    uint32_t m = 0;
+    if (g < n / 4) m = v.template load4<true, true>(4 * g, kk, ii);
+    uint32_t b[4];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      b[j] = __ballot_sync(0xffffffffu, (m >> j) & 1u);
+      tot += __popc(b[j]);
+    }
+    if (tot) {
+      int b0 = 0;
+      if (lane == 0) b0 = atomicAdd(&ctr[0], tot);
+      b0 = __shfl_sync(0xffffffffu, b0, 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if ((b[j] >> lane) & 1u) sink(b0 + __popc(b[j] & lt), u4_get(kk, j), i4_get(ii, j));
+        b0 += __popc(b[j]);
+      }
+    }
+  }
+}
+
+// Selects the top kTopK occupied slots of a view into sink(slot, key, pos), slots
+// 0..kTopK-1 (the view holds at least kTopK occupied slots).  Returns K*.
+template <int NT, class View, class Sink>
+__device__ uint32_t select_topk(const View& v, int n, uint32_t* skeys, uint32_t* hist, uint32_t* scratch, int* sh,
+                                int* ctr, int tid, int bar, Sink sink) {
+  if (tid == 0) {
+    ctr[0] = 0;
+    ctr[1] = 0;
+  }
+  uint32_t lo, hi;
+  stage_view<NT>(v, n, skeys, tid, scratch, bar, lo, hi);
+  int above;
+  const uint32_t kth = kth_largest<NT>(skeys, n, kTopK, lo, hi, hist, scratch, sh, tid, bar, &above);
+  emit_view<NT>(v, skeys, n, kTopK, kth, above, ctr, tid, sink);
+  return kth;
 }
 
 // ------------------------------------------------------------------------------------------
 template <int QPW>
 struct WGState {
-  uint32_t skeys[kCandCap];   // staged candidate keys for a selection
-  uint32_t hist[256];
+  uint32_t skeys[kSlots];     // staged candidate keys of one selection
+  uint32_t hist[kHistBins];
   float w[QPW][kHeads];
-  int cnt[QPW];
-  uint32_t thr[QPW];
+  int cnt_w[QPW][4];          // per-warp append counts, published at barriers
+  int cnt_k[QPW];             // entries in the current keep set
+  int kcur[QPW];              // which keep set is current
+  uint32_t thr[QPW];          // smallest key still admitted
   int pos[QPW];
+  uint32_t scratch[32];
   int sh[4];
   int ctr[2];
 };
@@ -188,7 +411,23 @@ struct ScoreCfg {
   static constexpr int kSmemBytes = kMiscOff + 64 + 1024;
   static_assert(kTmemNeed <= 512, "TMEM holds 512 columns");
   static_assert(kQHalf % 1024 == 0, "Q halves must stay 1024-byte aligned");
+  static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 };
+
+// one query's score for this thread's key: sum_h w_h * max(v_h, 0), packed pairs
+__device__ __forceinline__ float head_weighted_relu(const uint32_t (&v)[32], const float* w) {
+  const float4* w4 = reinterpret_cast<const float4*>(w);
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int h4 = 0; h4 < 8; ++h4) {
+    const float4 ww = w4[h4];
+    const float2 r0 = make_float2(fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.f), fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.f));
+    const float2 r1 = make_float2(fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.f), fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.f));
+    a0 = ffma2(make_float2(ww.x, ww.y), r0, a0);
+    a1 = ffma2(make_float2(ww.z, ww.w), r1, a1);
+  }
+  return (a0.x + a0.y) + (a1.x + a1.y);
+}
 
 template <int QMAX, int STAGES, int ACC_BUFS, int NWG>
 __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThreads, 1)
@@ -338,13 +577,31 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
     // ===================================================== epilogue warpgroups
     const int ew = warp - 2;
     const int g = ew >> 2;                 // warpgroup
-    const int qd = warp & 3;               // TMEM lane quadrant of this warp
+    const int qd = warp & 3;               // TMEM lane quadrant of this warp (also its append area)
     const int gtid = threadIdx.x - 64 - g * 128;
     const int bar = 1 + g;
     const int r = qd * 32 + lane;          // key row of this thread inside a tile
+    const uint32_t lt = lanemask_lt();
     WGState<QPW>& st = *reinterpret_cast<WGState<QPW>*>(smem + C::kWGOff + g * C::kWGBytes);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+    const size_t slot_base = static_cast<size_t>(blockIdx.x) * QMAX + g * QPW;
     int acc_ctr = 0;
+
+    // the candidates of query jj of this group, with the published counts
+    auto cands = [&](int jj) {
+      const size_t q = (slot_base + jj) * kCandStride;
+      QueryCands v;
+      v.kk = p.cand_keys + q + st.kcur[jj] * kTopK;
+      v.ki = p.cand_idx + q + st.kcur[jj] * kTopK;
+      v.ak = p.cand_keys + q + 2 * kTopK;
+      v.ai = p.cand_idx + q + 2 * kTopK;
+      v.cnt_k = st.cnt_k[jj];
+      v.cnt_w0 = st.cnt_w[jj][0];
+      v.cnt_w1 = st.cnt_w[jj][1];
+      v.cnt_w2 = st.cnt_w[jj][2];
+      v.cnt_w3 = st.cnt_w[jj][3];
+      return v;
+    };
 
     for (int local = 0;; ++local) {
       const int slot = local & 1;
@@ -356,7 +613,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
       if (it >= 0) wi = p.items[it];
       if (gtid < QPW && it >= 0) {
         const int j = g * QPW + gtid;
-        st.cnt[gtid] = 0;
+        st.cnt_k[gtid] = 0;
+        st.kcur[gtid] = 0;
         st.thr[gtid] = 0u;
         st.pos[gtid] = (j < wi.nq) ? p.pos_eff[wi.t0 + j] : -2;
       }
@@ -370,6 +628,14 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
 
       const int nloc = min(QPW, wi.nq - g * QPW);
       const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
+      int pos_r[QPW], cnt_r[QPW];
+      uint32_t thr_r[QPW];
+#pragma unroll
+      for (int jj = 0; jj < QPW; ++jj) {
+        pos_r[jj] = st.pos[jj];
+        thr_r[jj] = 0u;
+        cnt_r[jj] = 0;
+      }
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
         const int ab = acc_ctr % ACC_BUFS;
@@ -377,135 +643,176 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
         tc_fence_after();
         bool need = false;
         const int s_pos = kt * kKeyTile + r;
+        const bool in_range = s_pos < wi.k_end;
+        const uint32_t tcol = tlane + ab * C::kAccCols + g * QPW * kHeads;
         if (ok) {
-#pragma unroll 1
-          for (int jj = 0; jj < nloc; ++jj) {
-            uint32_t v[32];
-            tmem_ld_32cols(tlane + ab * C::kAccCols + (g * QPW + jj) * kHeads, v);
-            tmem_ld_wait(v);
-            const float4* w4 = reinterpret_cast<const float4*>(st.w[jj]);
-            float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+          float score[QPW];
+          if (nloc == QPW) {
+            // queries in pairs: two 32-column loads in flight, then the pair's scores
+            constexpr int kPair = QPW >= 2 ? 2 : 1;
 #pragma unroll
-            for (int h4 = 0; h4 < 8; ++h4) {
-              const float4 ww = w4[h4];
-              a0 = fmaf(ww.x, fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.f), a0);
-              a1 = fmaf(ww.y, fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.f), a1);
-              a2 = fmaf(ww.z, fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.f), a2);
-              a3 = fmaf(ww.w, fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.f), a3);
+            for (int j0 = 0; j0 < QPW; j0 += kPair) {
+              uint32_t v[kPair][32];
+#pragma unroll
+              for (int jj = 0; jj < kPair; ++jj) tmem_ld_32cols(tcol + (j0 + jj) * kHeads, v[jj]);
+#pragma unroll
+              for (int jj = 0; jj < kPair; ++jj) tmem_ld_wait(v[jj]);
+              if (j0 + kPair == QPW) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
+              }
+#pragma unroll
+              for (int jj = 0; jj < kPair; ++jj) score[j0 + jj] = head_weighted_relu(v[jj], st.w[j0 + jj]);
             }
-            const float score = (a0 + a1) + (a2 + a3);
-            const uint32_t u = float_to_ordered(score);
-            const bool pass = (s_pos < wi.k_end) && (s_pos <= st.pos[jj]) && (u >= st.thr[jj]);
+          } else {
+#pragma unroll 1
+            for (int jj = 0; jj < nloc; ++jj) {
+              uint32_t v[32];
+              tmem_ld_32cols(tcol + jj * kHeads, v);
+              tmem_ld_wait(v);
+              score[jj] = head_weighted_relu(v, st.w[jj]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          }
+          // append (score, position) to this warp's area of each query; the counts stay
+          // warp-uniform in registers
+#pragma unroll
+          for (int jj = 0; jj < QPW; ++jj) {
+            if (jj >= nloc) break;
+            const uint32_t u = float_to_ordered(score[jj]);
+            const bool pass = in_range && (s_pos <= pos_r[jj]) && (u >= thr_r[jj]);
             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-            if (bal) {
-              int base = 0;
-              if (lane == 0) {
-                base = atomicAdd(&st.cnt[jj], __popc(bal));
-                if (base + __popc(bal) > kCandCap - kKeyTile) need = true;
-              }
-              base = __shfl_sync(0xffffffffu, base, 0);
-              if (pass) {
-                const size_t q = (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW + jj) * kCandStride;
-                const int o = base + __popc(bal & lanemask_lt());
-                p.cand_keys[q + o] = u;
-                p.cand_idx[q + o] = s_pos;
-              }
+            if (pass) {
+              const size_t q = (slot_base + jj) * kCandStride + 2 * kTopK + qd * kWarpApp + cnt_r[jj] +
+                               __popc(bal & lt);
+              p.cand_keys[q] = u;
+              p.cand_idx[q] = s_pos;
             }
+            cnt_r[jj] += __popc(bal);
+            need |= cnt_r[jj] > kWarpApp - 32;
           }
         } else {
           failed = true;
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0 && ok) mbar_arrive(&acc_empty[ab]);
         if (named_bar_or(bar, 128, need || failed)) {
           if (named_bar_or(bar, 128, failed)) { failed = true; break; }
-          int cnts[QPW];
+          if (lane == 0) {
 #pragma unroll
-          for (int jj = 0; jj < QPW; ++jj) cnts[jj] = st.cnt[jj];
+            for (int jj = 0; jj < QPW; ++jj) st.cnt_w[jj][qd] = cnt_r[jj];
+          }
+          named_bar_sync(bar, 128);
 #pragma unroll 1
+          for (int jj = 0; jj < nloc; ++jj) {
+            // st.*[jj] is read by every thread here and written only after the barriers below
+            const QueryCands v = cands(jj);
+            const int cmax = max(max(v.cnt_w0, v.cnt_w1), max(v.cnt_w2, v.cnt_w3));
+            if (cmax <= kWarpApp - 32) continue;
+            const size_t q = (slot_base + jj) * kCandStride;
+            const int kc = st.kcur[jj];
+            const int n_valid = v.valid_count();
+            if (n_valid <= kTopK) {
+              // fewer than kTopK so far: move the append areas into the keep set
+              uint32_t* kk = p.cand_keys + q + kc * kTopK;
+              int32_t* ki = p.cand_idx + q + kc * kTopK;
+              if (gtid == 0) st.ctr[0] = 0;
+              named_bar_sync(bar, 128);
+              QueryCands a = v;
+              a.cnt_k = 0;
+              compact_view<128>(a, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
+                kk[v.cnt_k + rank] = key;
+                ki[v.cnt_k + rank] = pos;
+              });
+              named_bar_sync(bar, 128);
+              if (gtid == 0) {
+                st.cnt_k[jj] = n_valid;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
+              }
+            } else {
+              uint32_t* kn = p.cand_keys + q + (kc ^ 1) * kTopK;
+              int32_t* in = p.cand_idx + q + (kc ^ 1) * kTopK;
+              const uint32_t kth = select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid,
+                                                    bar, [&](int s2, uint32_t key, int pos) {
+                                                      kn[s2] = key;
+                                                      in[s2] = pos;
+                                                    });
+              named_bar_sync(bar, 128);
+              if (gtid == 0) {
+                st.cnt_k[jj] = kTopK;
+                st.kcur[jj] = kc ^ 1;
+                st.thr[jj] = (kth == 0xFFFFFFFFu) ? kth : kth + 1u;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
+              }
+            }
+            named_bar_sync(bar, 128);
+          }
+#pragma unroll
           for (int jj = 0; jj < QPW; ++jj) {
-            if (jj >= nloc || cnts[jj] <= kCandCap - kKeyTile) continue;
-            // ---- compaction: keep the best kTopK candidates, raise the threshold
-            const size_t q = (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW + jj) * kCandStride;
-            uint32_t* ck = p.cand_keys + q;
-            int32_t* ci = p.cand_idx + q;
-            const int n = cnts[jj];
-            for (int e = gtid; e < n; e += 128) st.skeys[e] = ck[e];
-            if (gtid == 0) { st.ctr[0] = 0; st.ctr[1] = 0; }
-            named_bar_sync(bar, 128);
-            int above;
-            const uint32_t kth = radix_kth<128>(st.skeys, n, kTopK, st.hist, st.sh, gtid, bar, &above);
-            emit_topk<128>(st.skeys, n, kTopK, kth, above, st.ctr, gtid, [&](int slot2, uint32_t key, int e) {
-              ck[kCandCap + slot2] = key;
-              ci[kCandCap + slot2] = ci[e];
-            });
-            named_bar_sync(bar, 128);
-            for (int e = gtid; e < kTopK; e += 128) {
-              ck[e] = ck[kCandCap + e];
-              ci[e] = ci[kCandCap + e];
-            }
-            if (gtid == 0) {
-              st.cnt[jj] = kTopK;
-              st.thr[jj] = (kth == 0xFFFFFFFFu) ? kth : kth + 1u;
-            }
-            named_bar_sync(bar, 128);
+            thr_r[jj] = st.thr[jj];
+            cnt_r[jj] = st.cnt_w[jj][qd];
           }
         }
       }
       if (failed) break;
 
-      // ---- end of item: exact top-k of each query's list
+      // ---- end of item: exact top-k of each query's candidates
+      if (lane == 0) {
+#pragma unroll
+        for (int jj = 0; jj < QPW; ++jj) st.cnt_w[jj][qd] = cnt_r[jj];
+      }
+      named_bar_sync(bar, 128);
 #pragma unroll 1
       for (int jj = 0; jj < nloc; ++jj) {
         const int t = wi.t0 + g * QPW + jj;
-        const size_t q = (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW + jj) * kCandStride;
-        const uint32_t* ck = p.cand_keys + q;
-        const int32_t* ci = p.cand_idx + q;
-        const int n = st.cnt[jj];
+        const QueryCands v = cands(jj);
+        const int n_valid = v.valid_count();
         if (wi.chunk < 0) {
           int32_t* oi = p.idx_out + static_cast<size_t>(t) * kTopK;
           float* os = p.score_out ? p.score_out + static_cast<size_t>(t) * kTopK : nullptr;
-          const int prefix = st.pos[jj] + 1;   // keys this query scores (0 if invalid)
+          const int prefix = st.pos[jj] + 1;   // keys this query scores (<= 0 if invalid)
           if (prefix <= kTopK) {
-            for (int e = gtid; e < n; e += 128) {
-              const int s = ci[e];
-              oi[s] = s;
-              if (os) os[s] = ordered_to_float(ck[e]);
-            }
-            for (int s = max(prefix, 0) + gtid; s < kTopK; s += 128) {
-              oi[s] = -1;
-              if (os) os[s] = -INFINITY;
+            // every position 0..prefix-1 is a candidate: place each at its own index
+            if (gtid == 0) st.ctr[0] = 0;
+            named_bar_sync(bar, 128);
+            compact_view<128>(v, kSlots, st.ctr, gtid, [&](int, uint32_t key, int pos) {
+              oi[pos] = pos;
+              if (os) os[pos] = ordered_to_float(key);
+            });
+            for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += 128) {
+              oi[s2] = -1;
+              if (os) os[s2] = -INFINITY;
             }
           } else {
-            for (int e = gtid; e < n; e += 128) st.skeys[e] = ck[e];
-            if (gtid == 0) { st.ctr[0] = 0; st.ctr[1] = 0; }
-            named_bar_sync(bar, 128);
-            int above;
-            const uint32_t kth = radix_kth<128>(st.skeys, n, kTopK, st.hist, st.sh, gtid, bar, &above);
-            emit_topk<128>(st.skeys, n, kTopK, kth, above, st.ctr, gtid, [&](int slot2, uint32_t key, int e) {
-              oi[slot2] = ci[e];
-              if (os) os[slot2] = ordered_to_float(key);
-            });
+            select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid, bar,
+                             [&](int s2, uint32_t key, int pos) {
+                               oi[s2] = pos;
+                               if (os) os[s2] = ordered_to_float(key);
+                             });
           }
         } else {
           uint32_t* pk = p.part_keys + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
           int32_t* pi = p.part_idx + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
-          if (n <= kTopK) {
-            for (int e = gtid; e < kTopK; e += 128) {
-              pk[e] = (e < n) ? ck[e] : 0u;
-              pi[e] = (e < n) ? ci[e] : -1;
+          if (n_valid <= kTopK) {
+            if (gtid == 0) st.ctr[0] = 0;
+            named_bar_sync(bar, 128);
+            compact_view<128>(v, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
+              pk[rank] = key;
+              pi[rank] = pos;
+            });
+            for (int e = n_valid + gtid; e < kTopK; e += 128) {
+              pk[e] = 0u;
+              pi[e] = -1;
             }
           } else {
-            for (int e = gtid; e < n; e += 128) st.skeys[e] = ck[e];
-            if (gtid == 0) { st.ctr[0] = 0; st.ctr[1] = 0; }
-            named_bar_sync(bar, 128);
-            int above;
-            const uint32_t kth = radix_kth<128>(st.skeys, n, kTopK, st.hist, st.sh, gtid, bar, &above);
-            emit_topk<128>(st.skeys, n, kTopK, kth, above, st.ctr, gtid, [&](int slot2, uint32_t key, int e) {
-              pk[slot2] = key;
-              pi[slot2] = ci[e];
-            });
+            select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid, bar,
+                             [&](int s2, uint32_t key, int pos) {
+                               pk[s2] = key;
+                               pi[s2] = pos;
+                             });
           }
         }
         named_bar_sync(bar, 128);
@@ -530,25 +837,21 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
                                                               int32_t* __restrict__ idx_out,
                                                               float* __restrict__ score_out) {
   extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK]
-  __shared__ uint32_t hist[256];
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t scratch[32];
   __shared__ int sh[4];
   __shared__ int ctr[2];
   const int t = blockIdx.x;
   const int nch = tok_nchunks[t];
   if (nch < 2) return;
   const int n = nch * kTopK;
-  const uint32_t* pk = part_keys + static_cast<size_t>(t) * kMaxChunks * kTopK;
-  const int32_t* pi = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
-  for (int e = threadIdx.x * 4; e < n; e += kMergeThreads * 4)
-    *reinterpret_cast<uint4*>(mkeys + e) = *reinterpret_cast<const uint4*>(pk + e);
-  if (threadIdx.x == 0) { ctr[0] = 0; ctr[1] = 0; }
-  __syncthreads();
-  int above;
-  const uint32_t kth = radix_kth<kMergeThreads>(mkeys, n, kTopK, hist, sh, threadIdx.x, 1, &above);
+  FlatCands v;
+  v.k = part_keys + static_cast<size_t>(t) * kMaxChunks * kTopK;
+  v.i = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
   int32_t* oi = idx_out + static_cast<size_t>(t) * kTopK;
   float* os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
-  emit_topk<kMergeThreads>(mkeys, n, kTopK, kth, above, ctr, threadIdx.x, [&](int slot, uint32_t key, int e) {
-    oi[slot] = pi[e];
+  select_topk<kMergeThreads>(v, n, mkeys, hist, scratch, sh, ctr, threadIdx.x, 1, [&](int slot, uint32_t key, int pos) {
+    oi[slot] = pos;
     if (os) os[slot] = ordered_to_float(key);
   });
 }
@@ -564,6 +867,7 @@ struct PrepParams {
   const int32_t* q_seq_offsets;
   const int64_t* cache_offsets;
   int split;
+  int num_sms;
   TopkWorkspace ws;
 };
 
@@ -614,18 +918,25 @@ __device__ __forceinline__ int owner_of(const int* base, int n_owners, int i) {
   return lo;
 }
 
-__device__ __forceinline__ int chunk_len_for(int n) {
-  // shortest multiple of 128 that is >= kMinChunk and covers n in kMaxChunks chunks
-  int c = (n + kMaxChunks - 1) / kMaxChunks;
+// Key-chunk length of a split query with n keys: chunks of about `target` keys (a
+// multiple of 128), at most kMaxChunks of them, of equal length but for the last.
+__device__ __forceinline__ int chunk_len_for(int n, int target) {
+  int nch = (n + target - 1) / target;
+  nch = nch < 1 ? 1 : (nch > kMaxChunks ? kMaxChunks : nch);
+  int c = (n + nch - 1) / nch;
   c = (c + kKeyTile - 1) / kKeyTile * kKeyTile;
-  return c < kMinChunk ? kMinChunk : c;
+  return c < kKeyTile ? kKeyTile : c;
 }
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __shared__ int warp_sums[32];
   __shared__ int bad;
+  __shared__ unsigned long long total_keys;
   const TopkWorkspace& ws = p.ws;
-  if (threadIdx.x == 0) bad = 0;
+  if (threadIdx.x == 0) {
+    bad = 0;
+    total_keys = 0;
+  }
   __syncthreads();
   // 1. offsets
   for (int b = threadIdx.x; b <= p.B; b += kPrepThreads) {
@@ -661,15 +972,20 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     if (!ok) atomicOr(ws.err, kErrBounds);
     ws.pos_eff[t] = ok ? pos : -1;
     ws.tok_nchunks[t] = 0;
+    if (p.split && ok) atomicAdd(&total_keys, static_cast<unsigned long long>(pos) + 1ull);
   }
   __syncthreads();
+  // split path: chunks sized so that about two chunks per SM cover all the keys
+  long long tgt = (static_cast<long long>(total_keys) + 2ll * p.num_sms - 1) / (2ll * p.num_sms);
+  tgt = (tgt + kKeyTile - 1) / kKeyTile * kKeyTile;
+  const int target = static_cast<int>(tgt < kMinChunk ? kMinChunk : (tgt > (1 << 30) ? (1 << 30) : tgt));
   // 3. items per owner (sequence on the prefill path, query on the split path)
   const int n_owners = p.split ? p.T : p.B;
   for (int o = threadIdx.x; o < n_owners; o += kPrepThreads) {
     int c;
     if (p.split) {
       const int n = ws.pos_eff[o] + 1;
-      const int cl = chunk_len_for(n);
+      const int cl = chunk_len_for(n, target);
       c = n > cl ? (n + cl - 1) / cl : 1;
       ws.tok_nchunks[o] = c;
     } else {
@@ -696,7 +1012,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       const int t = o;
       const int n = ws.pos_eff[t] + 1;
       const int nch = ws.tok_nchunks[t];
-      const int cl = chunk_len_for(n);
+      const int cl = chunk_len_for(n, target);
       int lo = 0, hi = p.B - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -764,6 +1080,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   pp.q_seq_offsets = a.q_seq_offsets;
   pp.cache_offsets = a.cache_offsets;
   pp.split = a.split ? 1 : 0;
+  pp.num_sms = num_sms;
   pp.ws = ws;
   prep_kernel<<<1, kPrepThreads, 0, s>>>(pp);
   cudaError_t e = cudaGetLastError();

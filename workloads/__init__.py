@@ -20,6 +20,7 @@ from .generate import (  # noqa: F401
     make_weights,
     make_prefill,
     make_decode,
+    decode_lengths,
     heavy_hitter_rows,
     causal_pairs,
     make_scoring_inputs,

@@ -122,13 +122,18 @@ def make_prefill(seed: int, seq_lens, start_positions=None, cache_lens=None,
     return PrefillBatch(hidden, q_latent, positions, q_seq_offsets, cache_offsets)
 
 
+def decode_lengths(seed: int, batch: int = 64, L_min: int = 16384, L_max: int = 131072) -> torch.Tensor:
+    """Cache length of each decode sequence, uniform in [L_min, L_max]."""
+    return torch.randint(L_min, L_max + 1, (batch,), generator=_gen(seed, _S_LENS), dtype=torch.int64)
+
+
 def make_decode(seed: int, batch: int = 64, L_min: int = 16384, L_max: int = 131072,
                 hidden_dim: int = 7168, q_latent_dim: int = 1536, head_dim: int = 128,
                 lengths=None) -> DecodeBatch:
     """One new query token per sequence; sequence b holds L_b cached tokens
     (the new token is the last, at position L_b - 1)."""
     if lengths is None:
-        lengths = torch.randint(L_min, L_max + 1, (batch,), generator=_gen(seed, _S_LENS), dtype=torch.int64)
+        lengths = decode_lengths(seed, batch, L_min, L_max)
     else:
         lengths = torch.as_tensor(lengths, dtype=torch.int64)
         batch = int(lengths.numel())
