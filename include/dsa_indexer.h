@@ -151,6 +151,31 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
                               int32_t* idx_out,
                               float* score_out, uint32_t flags, void* stream);
 
+/* Allocation-free score + top-k (no counterpart on the pages; it exists for the
+ * library's users).  Some callers cannot let a library allocate device memory:
+ * a framework whose memory pool already holds the device's whole budget, or a
+ * latency-critical loop that must never pay for cudaMalloc / cudaFree and the
+ * device synchronisation they can imply.  This entry point needs no handle and
+ * calls no allocator: its scratch is a fixed array in the library's static
+ * device memory, 6,473,216 bytes (6.2 MiB), which every GPU that loads the library holds until the
+ * process exits.  The caller still passes every input and output, as for
+ * dsa_indexer_topk (same arguments without handle and flags; same output rules;
+ * the prefill path of dsa_indexer_topk with DSA_TOPK_NO_SPLIT).
+ * Limits: T <= 4096 and B <= 4096 (otherwise DSA_ERR_WORKSPACE); the kernels run
+ * on at most 16 SMs (the scratch holds 16 per-SM candidate areas), so this is
+ * slower than dsa_indexer_topk.  Device-side problems are not reported through
+ * a status word (there is no handle): affected rows are padded as documented
+ * for dsa_indexer_topk.
+ * The first call on a device looks up the scratch's device address with that
+ * device current.  All calls on a device share the one scratch array, which keeps
+ * the previous call's contents (the call clears what must start at zero): calls
+ * whose kernels can overlap on the GPU (e.g. on unordered streams) race and
+ * corrupt each other's results; order them on one stream. */
+dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const float* w, const int32_t* positions,
+                                      const int32_t* q_seq_offsets, int32_t B, const void* key_cache,
+                                      int64_t cache_rows, const int64_t* cache_offsets, int32_t* idx_out,
+                                      float* score_out, void* stream);
+
 /* Synchronises the device, then returns DSA_OK or the first device-side error
  * recorded since the last call (DSA_ERR_DEVICE_BOUNDS, DSA_ERR_DEVICE_TIMEOUT)
  * and clears the error word. */
