@@ -44,9 +44,10 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, int K, int N, __nv_b
 
 // ---------------------------------------------------------------- score + top-k
 // Candidate storage of one query: two keep sets of kTopK entries (the current
-// best list and the target of the next compaction) and an append area.
-constexpr int kAppCap = kTopK;                 // appended candidates before a compaction
-constexpr int kCandStride = 3 * kTopK;         // keep set 0 | keep set 1 | append area
+// best list and the target of the next compaction) and an append area split
+// evenly between the four warps of an epilogue warpgroup.
+constexpr int kAppCap = 2 * kTopK;             // appended candidates before a compaction
+constexpr int kCandStride = 2 * kTopK + kAppCap;  // keep set 0 | keep set 1 | append area
 constexpr int kMaxChunks = 16;                 // key chunks per query on the split-key path
 constexpr int kMinChunk = 4096;                // shortest key chunk on the split-key path
 constexpr int kSplitMaxTokens = 256;           // split-key path is offered up to this many queries

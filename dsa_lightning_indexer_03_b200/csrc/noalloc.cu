@@ -22,7 +22,7 @@ using namespace dsa;
 
 namespace {
 
-constexpr int kStaticCtas = 16;          // persistent CTAs (candidate areas) the scratch holds
+constexpr int kStaticCtas = 12;          // persistent CTAs (candidate areas) the scratch holds
 constexpr int kStaticMaxTokens = 4096;   // largest T (and B) this entry point accepts
 constexpr int kStaticMaxItems = kStaticMaxTokens + 16;
 

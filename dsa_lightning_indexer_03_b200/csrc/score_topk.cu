@@ -105,14 +105,16 @@ __device__ __forceinline__ void group_minmax(uint32_t& lo, uint32_t& hi, int tid
   named_bar_sync(bar, NT);
 }
 
-// k-th largest of n order-preserving keys held in shared memory (1 <= k <= n), all of
-// them inside [lo, hi].  Each round histograms the keys of the current window into at
-// most kHistBins bins of width 2^shift, locates the bin that holds the k-th largest,
-// and narrows the window to that bin; a round of width-1 bins ends it (at most three
-// rounds for 32-bit keys).  *n_above receives the number of keys strictly greater
-// than the returned key.
-constexpr int kHistBins = 2048;
+constexpr int kHistBins = 1024;   // histogram bins of one selection round
+constexpr int kRankList = 256;    // boundary-bin keys ranked directly
 
+// k-th largest of n order-preserving keys held in shared memory (1 <= k <= n), all of
+// them inside [lo, hi] (keys outside are ignored).  Each round histograms the keys of
+// the current window into at most kHistBins bins of width 2^shift, locates the bin that
+// holds the k-th largest, and narrows the window to that bin; a round of width-1 bins
+// ends it (at most four rounds for 32-bit keys).  *n_above receives the number of keys
+// strictly greater than the returned key.  Used where the value-binned round below
+// cannot isolate the boundary (crowded bins: ties, extreme ranges).
 template <int NT>
 __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo, uint32_t hi, uint32_t* hist,
                                 uint32_t* scratch, int* sh, int tid, int bar, int* n_above) {
@@ -121,11 +123,9 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
   int need = k, above_total = 0;
 #pragma unroll 1
   while (true) {
-    const int shift = (span >> 11) ? 32 - __clz(static_cast<int>(span >> 11)) : 0;
-    const int nb = static_cast<int>(span >> shift) + 1;
+    const int shift = (span >> 10) ? 32 - __clz(static_cast<int>(span >> 10)) : 0;
     for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
     named_bar_sync(bar, NT);
-#pragma unroll 4
     for (int e = tid; e < n; e += NT) {
       const uint32_t d = keys[e] - base;
       if (d <= span) atomicAdd(&hist[d >> shift], 1u);
@@ -158,7 +158,7 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
     named_bar_sync(bar, NT);
     need -= above;
     above_total += above;
-    if (shift == 0 || nb <= 0) {
+    if (shift == 0) {
       *n_above = above_total;
       return base + static_cast<uint32_t>(bstar);
     }
@@ -170,11 +170,11 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
 // Candidate views: a fixed set of slots (a multiple of 4), some of them empty.
 // load4(s0, k, i) fetches slots s0..s0+3 with 16-byte loads where the four are all
 // occupied and returns the occupied-slot mask; empty slots read key 0, position -1.
-constexpr int kSlots = 2 * kTopK;          // keep set + append area of one query
 constexpr int kWarpApp = kAppCap / 4;      // append slots of one epilogue warp
+constexpr int kSlots = kTopK + kAppCap;    // keep set + append area of one query
 
 // The candidates of one query in the score kernel: the current keep set (slots
-// 0..2047) followed by the four warps' append areas (512 slots each).
+// 0..kTopK-1) followed by the four warps' append areas (kWarpApp slots each).
 struct QueryCands {
   const uint32_t* kk;
   const int32_t* ki;
@@ -249,31 +249,6 @@ __device__ __forceinline__ int i4_get(const int4& v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 
-// Copies the keys of n slots into shared memory (empty slots as 0) and returns the
-// range of the occupied ones.
-template <int NT, class View>
-__device__ __forceinline__ void stage_view(const View& v, int n, uint32_t* skeys, int tid, uint32_t* scratch,
-                                           int bar, uint32_t& lo, uint32_t& hi) {
-  lo = 0xFFFFFFFFu;
-  hi = 0u;
-#pragma unroll 2
-  for (int g = tid; g < n / 4; g += NT) {
-    uint4 k;
-    int4 dummy;
-    const uint32_t m = v.template load4<true, false>(4 * g, k, dummy);
-    reinterpret_cast<uint4*>(skeys)[g] = k;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (m & (1u << j)) {
-        lo = min(lo, u4_get(k, j));
-        hi = max(hi, u4_get(k, j));
-      }
-    }
-  }
-  group_minmax<NT>(lo, hi, tid, scratch, bar);
-  if (lo > hi) lo = hi;  // no occupied slot
-}
-
 // Emits the top k of the occupied slots: every key > kth and the first (k - n_above)
 // keys equal to kth.  sink(slot, key, pos) is called once per kept entry with a
 // distinct slot in [0, k).  ctr[0..1] are shared counters zeroed beforehand.
@@ -283,15 +258,19 @@ __device__ void emit_view(const View& v, const uint32_t* skeys, int n, int k, ui
   const int lane = tid & 31;
   const int ties = k - n_above;
   const uint32_t lt = lanemask_lt();
+#pragma unroll 12
   for (int base = 0; base < n / 4; base += NT) {
     const int g = base + tid;
     uint4 kk = make_uint4(0u, 0u, 0u, 0u);
     int4 ii = make_int4(-1, -1, -1, -1);
     uint32_t m = 0;
     if (g < n / 4) {
-      uint4 dummy;
-      m = v.template load4<false, true>(4 * g, dummy, ii);
       kk = reinterpret_cast<const uint4*>(skeys)[g];
+      // only groups holding a kept key need their positions
+      if (kk.x >= kth || kk.y >= kth || kk.z >= kth || kk.w >= kth) {
+        uint4 dummy;
+        m = v.template load4<false, true>(4 * g, dummy, ii);
+      }
     }
     uint32_t bg[4], be[4];
     int tg = 0, te = 0;
@@ -331,6 +310,7 @@ template <int NT, class View, class Sink>
 __device__ void compact_view(const View& v, int n, int* ctr, int tid, Sink sink) {
   const int lane = tid & 31;
   const uint32_t lt = lanemask_lt();
+#pragma unroll 2
   for (int base = 0; base < n / 4; base += NT) {
     const int g = base + tid;
     uint4 kk = make_uint4(0u, 0u, 0u, 0u);
@@ -357,20 +337,159 @@ __device__ void compact_view(const View& v, int n, int* ctr, int tid, Sink sink)
   }
 }
 
-// Selects the top kTopK occupied slots of a view into sink(slot, key, pos), slots
-// 0..kTopK-1 (the view holds at least kTopK occupied slots).  Returns K*.
+// Histogram bin of a key for the selection's first round: bins of equal width in
+// score value between the smallest and largest candidate (a monotone map from the
+// ordered keys, so the bin holding the k-th largest can be found exactly).
+__device__ __forceinline__ int value_bin(uint32_t key, float lo_f, float scale) {
+  const float x = (ordered_to_float(key) - lo_f) * scale;
+  int b = __float2int_rz(x);
+  b = b < 0 ? 0 : (b > kHistBins - 1 ? kHistBins - 1 : b);
+  return x == x ? b : 0;
+}
+
+// Selects the top kTopK occupied slots of a view (which holds at least kTopK):
+// 1. stage the keys of the n slots into shared memory (empty slots as 0) and find
+//    the occupied keys' range;
+// 2. histogram the keys into kHistBins bins of equal width in score value and
+//    locate the bin that holds the kTopK-th largest;
+// 3. gather that bin's keys into `list` and find the exact kTopK-th largest K* there
+//    by counting ranks (a crowded bin falls back to kth_largest over all keys);
+// 4. emit every key > K* and the first kTopK - n_above keys equal to K* through
+//    sink(slot, key, pos).  Returns K*.
 template <int NT, class View, class Sink>
-__device__ uint32_t select_topk(const View& v, int n, uint32_t* skeys, uint32_t* hist, uint32_t* scratch, int* sh,
-                                int* ctr, int tid, int bar, Sink sink) {
+__device__ uint32_t select_topk(const View& v, int n, uint32_t* skeys, uint32_t* hist, uint32_t* list, int list_cap,
+                                uint32_t* scratch, int* sh, int* ctr, int tid, int bar, Sink sink) {
+  const int lane = tid & 31, wid = tid >> 5;
+  // 1. stage + range; the histogram is cleared and the counters zeroed in the same phase
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll 12
+  for (int g = tid; g < n / 4; g += NT) {
+    uint4 k;
+    int4 unused;
+    const uint32_t m = v.template load4<true, false>(4 * g, k, unused);
+    reinterpret_cast<uint4*>(skeys)[g] = k;
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if ((m >> j) & 1u) {
+        lo = min(lo, u4_get(k, j));
+        hi = max(hi, u4_get(k, j));
+      }
+  }
+  for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
   if (tid == 0) {
     ctr[0] = 0;
     ctr[1] = 0;
+    sh[5] = 0;
   }
-  uint32_t lo, hi;
-  stage_view<NT>(v, n, skeys, tid, scratch, bar, lo, hi);
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  if (lane == 0) {
+    scratch[wid] = lo;
+    scratch[NT / 32 + wid] = hi;
+  }
+  named_bar_sync(bar, NT);
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    lo = min(lo, scratch[w]);
+    hi = max(hi, scratch[NT / 32 + w]);
+  }
+  const float lo_f = ordered_to_float(lo), hi_f = ordered_to_float(hi);
+  float scale = (hi_f > lo_f) ? static_cast<float>(kHistBins) / (hi_f - lo_f) : 0.f;
+  if (!(scale < 3.0e38f)) scale = 0.f;
+
+  // 2. value-binned histogram of the occupied keys (empty slots hold key 0)
+#pragma unroll 4
+  for (int g = tid; g < n / 4; g += NT) {
+    const uint4 k = reinterpret_cast<const uint4*>(skeys)[g];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = u4_get(k, j);
+      if (key >= lo && key != 0u) atomicAdd(&hist[value_bin(key, lo_f, scale)], 1u);
+    }
+  }
+  named_bar_sync(bar, NT);
   int above;
-  const uint32_t kth = kth_largest<NT>(skeys, n, kTopK, lo, hi, hist, scratch, sh, tid, bar, &above);
-  emit_view<NT>(v, skeys, n, kTopK, kth, above, ctr, tid, sink);
+  int bstar;
+  {
+    constexpr int kBPT = kHistBins / NT;
+    const int b0 = tid * kBPT;
+    uint32_t c[kBPT];
+    uint32_t s = 0;
+#pragma unroll
+    for (int i = 0; i < kBPT; ++i) {
+      c[i] = hist[b0 + i];
+      s += c[i];
+    }
+    // suffix sum over threads: warp shuffles + one exchange of warp totals
+    uint32_t x = s;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
+      if (lane + off < 32) x += y;
+    }
+    if (lane == 0) scratch[2 * (NT / 32) + wid] = x;
+    named_bar_sync(bar, NT);
+    uint32_t above_t = x - s;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w)
+      if (w > wid) above_t += scratch[2 * (NT / 32) + w];
+    const uint32_t need = kTopK;
+    if (above_t < need && need <= above_t + s) {
+      uint32_t cum = above_t;
+#pragma unroll
+      for (int i = kBPT - 1; i >= 0; --i) {
+        if (cum + c[i] >= need) {
+          sh[0] = b0 + i;
+          sh[1] = static_cast<int>(cum);
+          break;
+        }
+        cum += c[i];
+      }
+    }
+    named_bar_sync(bar, NT);
+    bstar = sh[0];
+    above = sh[1];
+  }
+  // 3. gather the boundary bin and rank its keys
+#pragma unroll 4
+  for (int g = tid; g < n / 4; g += NT) {
+    const uint4 k = reinterpret_cast<const uint4*>(skeys)[g];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = u4_get(k, j);
+      if (key >= lo && key != 0u && value_bin(key, lo_f, scale) == bstar) {
+        const int o = atomicAdd(&sh[5], 1);
+        if (o < list_cap) list[o] = key;
+      }
+    }
+  }
+  named_bar_sync(bar, NT);
+  const int m = sh[5];
+  const int need2 = kTopK - above;
+  uint32_t kth;
+  int n_above;
+  if (m <= list_cap) {
+    for (int e = tid; e < m; e += NT) {
+      const uint32_t xk = list[e];
+      int greater = 0, equal = 0;
+      for (int j = 0; j < m; ++j) {
+        const uint32_t y = list[j];
+        greater += y > xk;
+        equal += y == xk;
+      }
+      if (greater < need2 && need2 <= greater + equal) {  // every finder writes the same values
+        sh[2] = static_cast<int>(xk);
+        sh[3] = greater;
+      }
+    }
+    named_bar_sync(bar, NT);
+    kth = static_cast<uint32_t>(sh[2]);
+    n_above = above + sh[3];
+  } else {
+    kth = kth_largest<NT>(skeys, n, kTopK, lo, hi, hist, scratch, sh, tid, bar, &n_above);
+  }
+  // 4. emit
+  emit_view<NT>(v, skeys, n, kTopK, kth, n_above, ctr, tid, sink);
   return kth;
 }
 
@@ -379,21 +498,33 @@ template <int QPW>
 struct WGState {
   uint32_t skeys[kSlots];     // staged candidate keys of one selection
   uint32_t hist[kHistBins];
+  uint32_t list[kRankList];   // keys of the boundary bin
   float w[QPW][kHeads];
   int cnt_w[QPW][4];          // per-warp append counts, published at barriers
   int cnt_k[QPW];             // entries in the current keep set
   int kcur[QPW];              // which keep set is current
   uint32_t thr[QPW];          // smallest key still admitted
   int pos[QPW];
-  uint32_t scratch[32];
-  int sh[4];
+  uint32_t scratch[64];
+  int sh[8];
   int ctr[2];
 };
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG>
+// Thread layout of the score kernel.  EW = epilogue warps per group: 4 (one warp per
+// TMEM lane quadrant, each warp handles every query of the group) or 8 (two warps per
+// quadrant, each handles half of the group's queries).  With EW = 8 the two control
+// warps sit in a warpgroup of their own (warps 0-3) so that registers can be moved
+// from it to the epilogue warpgroups (setmaxnreg).
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
 struct ScoreCfg {
-  static constexpr int kQPW = QMAX / NWG;
-  static constexpr int kThreads = 64 + NWG * 128;
+  static constexpr int kQPW = QMAX / NWG;             // queries of one epilogue group
+  static constexpr int kQPH = kQPW / (EW / 4);        // queries of one epilogue warp
+  static constexpr int kEpiWarp0 = EW == 8 ? 4 : 2;   // first epilogue warp
+  static constexpr int kGroupThreads = EW * 32;
+  static constexpr int kThreads = kEpiWarp0 * 32 + NWG * kGroupThreads;
+  static constexpr bool kRegSplit = EW == 8;
+  static constexpr int kCtrlRegs = 32;                // per thread of warps 0-3 after the split
+  static constexpr int kEpiRegs = 112;                // per epilogue thread after the split
   static constexpr int kAccCols = QMAX * kHeads;
   static constexpr int kTmemNeed = ACC_BUFS * kAccCols;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
@@ -412,6 +543,8 @@ struct ScoreCfg {
   static_assert(kTmemNeed <= 512, "TMEM holds 512 columns");
   static_assert(kQHalf % 1024 == 0, "Q halves must stay 1024-byte aligned");
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+  static_assert(kQPH >= 1 && kQPH * (EW / 4) == kQPW, "queries split evenly over a quadrant's warps");
+  static_assert(kCtrlRegs % 8 == 0 && kEpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 };
 
 // one query's score for this thread's key: sum_h w_h * max(v_h, 0), packed pairs
@@ -429,12 +562,14 @@ __device__ __forceinline__ float head_weighted_relu(const uint32_t (&v)[32], con
   return (a0.x + a0.y) + (a1.x + a1.y);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG>
-__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThreads, 1)
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
+__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       ScoreParams p) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>;
   constexpr int QPW = C::kQPW;
+  constexpr int QPH = C::kQPH;
+  constexpr int NTG = C::kGroupThreads;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::kQOff;
@@ -462,13 +597,13 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
     }
     for (int a = 0; a < ACC_BUFS; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], NWG * 4);
+      mbar_init(&acc_empty[a], NWG * EW);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sched_full[i], 1);
-      mbar_init(&sched_empty[i], 1 + NWG * 4);
+      mbar_init(&sched_empty[i], 1 + NWG * EW);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -487,6 +622,11 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
   const int n_items = *p.n_items;
   const WaitCtl wc{p.err, abort_flag, p.timeout_ns};
 
+  if (warp < C::kEpiWarp0) {
+    // ===================================================== control warps
+    if constexpr (C::kRegSplit) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kCtrlRegs));
+    }
   if (warp == 0) {
     // ===================================================== TMA producer
     if (lane == 0) {
@@ -573,18 +713,24 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
       umma_commit(mma_done);
       drain_wait(mma_done, 0);
     }
+  }
   } else {
-    // ===================================================== epilogue warpgroups
-    const int ew = warp - 2;
-    const int g = ew >> 2;                 // warpgroup
-    const int qd = warp & 3;               // TMEM lane quadrant of this warp (also its append area)
-    const int gtid = threadIdx.x - 64 - g * 128;
+    // ===================================================== epilogue groups
+    if constexpr (C::kRegSplit) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::kEpiRegs));
+    }
+    const int ew = warp - C::kEpiWarp0;
+    const int g = ew / EW;                   // epilogue group = a set of QPW queries of the item
+    const int hq = (ew % EW) / 4;            // which half of the group's queries this warp scores
+    const int qd = warp & 3;                 // TMEM lane quadrant of this warp (also its append area)
+    const int gtid = threadIdx.x - C::kEpiWarp0 * 32 - g * NTG;
     const int bar = 1 + g;
-    const int r = qd * 32 + lane;          // key row of this thread inside a tile
+    const int r = qd * 32 + lane;            // key row of this thread inside a tile
     const uint32_t lt = lanemask_lt();
     WGState<QPW>& st = *reinterpret_cast<WGState<QPW>*>(smem + C::kWGOff + g * C::kWGBytes);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const size_t slot_base = static_cast<size_t>(blockIdx.x) * QMAX + g * QPW;
+    const int j0 = hq * QPH;                 // first of this warp's queries inside the group
     int acc_ctr = 0;
 
     // the candidates of query jj of this group, with the published counts
@@ -617,25 +763,23 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
         st.kcur[gtid] = 0;
         st.thr[gtid] = 0u;
         st.pos[gtid] = (j < wi.nq) ? p.pos_eff[wi.t0 + j] : -2;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) st.cnt_w[gtid][w] = 0;
       }
       if (it >= 0) {
-        for (int i = gtid; i < QPW * kHeads; i += 128) {
+        for (int i = gtid; i < QPW * kHeads; i += NTG) {
           const int jj = i / kHeads, j = g * QPW + jj;
           st.w[jj][i % kHeads] = (j < wi.nq) ? p.w[static_cast<size_t>(wi.t0 + j) * kHeads + (i % kHeads)] : 0.f;
         }
       }
-      if (named_bar_or(bar, 128, it < 0)) break;   // every thread of the group leaves together
+      if (named_bar_or(bar, NTG, it < 0)) break;   // every thread of the group leaves together
 
-      const int nloc = min(QPW, wi.nq - g * QPW);
+      const int nloc = min(QPW, wi.nq - g * QPW);  // queries of the group present in this item
+      const int nmine = min(QPH, nloc - j0);        // ... and scored by this warp (may be <= 0)
       const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
-      int pos_r[QPW], cnt_r[QPW];
-      uint32_t thr_r[QPW];
+      int cnt_r[QPH];
 #pragma unroll
-      for (int jj = 0; jj < QPW; ++jj) {
-        pos_r[jj] = st.pos[jj];
-        thr_r[jj] = 0u;
-        cnt_r[jj] = 0;
-      }
+      for (int j = 0; j < QPH; ++j) cnt_r[j] = 0;
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
         const int ab = acc_ctr % ACC_BUFS;
@@ -644,116 +788,115 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
         bool need = false;
         const int s_pos = kt * kKeyTile + r;
         const bool in_range = s_pos < wi.k_end;
-        const uint32_t tcol = tlane + ab * C::kAccCols + g * QPW * kHeads;
+        const uint32_t tcol = tlane + ab * C::kAccCols + (g * QPW + j0) * kHeads;
         if (ok) {
-          float score[QPW];
-          if (nloc == QPW) {
-            // queries in pairs: two 32-column loads in flight, then the pair's scores
-            constexpr int kPair = QPW >= 2 ? 2 : 1;
+          float score[QPH];
+          if (nmine == QPH) {
+            // every column this warp needs, requested at once: one TMEM round trip per tile
+            uint32_t v[QPH][32];
 #pragma unroll
-            for (int j0 = 0; j0 < QPW; j0 += kPair) {
-              uint32_t v[kPair][32];
+            for (int j = 0; j < QPH; ++j) tmem_ld_32cols(tcol + j * kHeads, v[j]);
 #pragma unroll
-              for (int jj = 0; jj < kPair; ++jj) tmem_ld_32cols(tcol + (j0 + jj) * kHeads, v[jj]);
+            for (int j = 0; j < QPH; ++j) tmem_ld_wait(v[j]);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
 #pragma unroll
-              for (int jj = 0; jj < kPair; ++jj) tmem_ld_wait(v[jj]);
-              if (j0 + kPair == QPW) {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
-              }
-#pragma unroll
-              for (int jj = 0; jj < kPair; ++jj) score[j0 + jj] = head_weighted_relu(v[jj], st.w[j0 + jj]);
-            }
+            for (int j = 0; j < QPH; ++j) score[j] = head_weighted_relu(v[j], st.w[j0 + j]);
           } else {
-#pragma unroll 1
-            for (int jj = 0; jj < nloc; ++jj) {
-              uint32_t v[32];
-              tmem_ld_32cols(tcol + jj * kHeads, v);
-              tmem_ld_wait(v);
-              score[jj] = head_weighted_relu(v, st.w[jj]);
+            // a partial query tile: static indices keep score[] in registers
+#pragma unroll
+            for (int j = 0; j < QPH; ++j) {
+              if (j < nmine) {
+                uint32_t v[32];
+                tmem_ld_32cols(tcol + j * kHeads, v);
+                tmem_ld_wait(v);
+                score[j] = head_weighted_relu(v, st.w[j0 + j]);
+              }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
           }
-          // append (score, position) to this warp's area of each query; the counts stay
-          // warp-uniform in registers
+          // append (score, position) to this warp's area of each of its queries; the
+          // counts stay warp-uniform in registers
 #pragma unroll
-          for (int jj = 0; jj < QPW; ++jj) {
-            if (jj >= nloc) break;
-            const uint32_t u = float_to_ordered(score[jj]);
-            const bool pass = in_range && (s_pos <= pos_r[jj]) && (u >= thr_r[jj]);
+          for (int j = 0; j < QPH; ++j) {
+            if (j >= nmine) break;
+            const int jj = j0 + j;
+            const uint32_t u = float_to_ordered(score[j]);
+            const bool pass = in_range && (s_pos <= st.pos[jj]) && (u >= st.thr[jj]);
             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
             if (pass) {
-              const size_t q = (slot_base + jj) * kCandStride + 2 * kTopK + qd * kWarpApp + cnt_r[jj] +
+              const size_t q = (slot_base + jj) * kCandStride + 2 * kTopK + qd * kWarpApp + cnt_r[j] +
                                __popc(bal & lt);
               p.cand_keys[q] = u;
               p.cand_idx[q] = s_pos;
             }
-            cnt_r[jj] += __popc(bal);
-            need |= cnt_r[jj] > kWarpApp - 32;
+            cnt_r[j] += __popc(bal);
+            need |= cnt_r[j] > kWarpApp - 2 * 32;
           }
         } else {
           failed = true;
         }
-        if (named_bar_or(bar, 128, need || failed)) {
-          if (named_bar_or(bar, 128, failed)) { failed = true; break; }
-          if (lane == 0) {
+        // capacity check every other tile (an append area takes at most 32 entries per tile)
+        if (((kt - kt0) & 1) == 1 || kt + 1 == kt1) {   // the same tiles for every warp of the group
+          if (named_bar_or(bar, NTG, need || failed)) {
+            if (named_bar_or(bar, NTG, failed)) { failed = true; break; }
+            if (lane == 0) {
 #pragma unroll
-            for (int jj = 0; jj < QPW; ++jj) st.cnt_w[jj][qd] = cnt_r[jj];
-          }
-          named_bar_sync(bar, 128);
-#pragma unroll 1
-          for (int jj = 0; jj < nloc; ++jj) {
-            // st.*[jj] is read by every thread here and written only after the barriers below
-            const QueryCands v = cands(jj);
-            const int cmax = max(max(v.cnt_w0, v.cnt_w1), max(v.cnt_w2, v.cnt_w3));
-            if (cmax <= kWarpApp - 32) continue;
-            const size_t q = (slot_base + jj) * kCandStride;
-            const int kc = st.kcur[jj];
-            const int n_valid = v.valid_count();
-            if (n_valid <= kTopK) {
-              // fewer than kTopK so far: move the append areas into the keep set
-              uint32_t* kk = p.cand_keys + q + kc * kTopK;
-              int32_t* ki = p.cand_idx + q + kc * kTopK;
-              if (gtid == 0) st.ctr[0] = 0;
-              named_bar_sync(bar, 128);
-              QueryCands a = v;
-              a.cnt_k = 0;
-              compact_view<128>(a, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
-                kk[v.cnt_k + rank] = key;
-                ki[v.cnt_k + rank] = pos;
-              });
-              named_bar_sync(bar, 128);
-              if (gtid == 0) {
-                st.cnt_k[jj] = n_valid;
-#pragma unroll
-                for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
-              }
-            } else {
-              uint32_t* kn = p.cand_keys + q + (kc ^ 1) * kTopK;
-              int32_t* in = p.cand_idx + q + (kc ^ 1) * kTopK;
-              const uint32_t kth = select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid,
-                                                    bar, [&](int s2, uint32_t key, int pos) {
-                                                      kn[s2] = key;
-                                                      in[s2] = pos;
-                                                    });
-              named_bar_sync(bar, 128);
-              if (gtid == 0) {
-                st.cnt_k[jj] = kTopK;
-                st.kcur[jj] = kc ^ 1;
-                st.thr[jj] = (kth == 0xFFFFFFFFu) ? kth : kth + 1u;
-#pragma unroll
-                for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
-              }
+              for (int j = 0; j < QPH; ++j)
+                if (j < nmine) st.cnt_w[j0 + j][qd] = cnt_r[j];
             }
-            named_bar_sync(bar, 128);
-          }
+            named_bar_sync(bar, NTG);
+#pragma unroll 1
+            for (int jj = 0; jj < nloc; ++jj) {
+              // st.*[jj] is read by every thread here and written only after the barriers below
+              const QueryCands v = cands(jj);
+              const int cmax = max(max(v.cnt_w0, v.cnt_w1), max(v.cnt_w2, v.cnt_w3));
+              if (cmax <= kWarpApp - 2 * 32) continue;
+              const size_t q = (slot_base + jj) * kCandStride;
+              const int kc = st.kcur[jj];
+              const int n_valid = v.valid_count();
+              if (n_valid <= kTopK) {
+                // fewer than kTopK so far: move the append areas into the keep set
+                uint32_t* kk = p.cand_keys + q + kc * kTopK;
+                int32_t* ki = p.cand_idx + q + kc * kTopK;
+                if (gtid == 0) st.ctr[0] = 0;
+                named_bar_sync(bar, NTG);
+                QueryCands a = v;
+                a.cnt_k = 0;
+                compact_view<NTG>(a, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
+                  kk[v.cnt_k + rank] = key;
+                  ki[v.cnt_k + rank] = pos;
+                });
+                named_bar_sync(bar, NTG);
+                if (gtid == 0) {
+                  st.cnt_k[jj] = n_valid;
 #pragma unroll
-          for (int jj = 0; jj < QPW; ++jj) {
-            thr_r[jj] = st.thr[jj];
-            cnt_r[jj] = st.cnt_w[jj][qd];
+                  for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
+                }
+              } else {
+                uint32_t* kn = p.cand_keys + q + (kc ^ 1) * kTopK;
+                int32_t* in = p.cand_idx + q + (kc ^ 1) * kTopK;
+                const uint32_t kth = select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch,
+                                                      st.sh, st.ctr, gtid, bar, [&](int s2, uint32_t key, int pos) {
+                                                        kn[s2] = key;
+                                                        in[s2] = pos;
+                                                      });
+                named_bar_sync(bar, NTG);
+                if (gtid == 0) {
+                  st.cnt_k[jj] = kTopK;
+                  st.kcur[jj] = kc ^ 1;
+                  st.thr[jj] = (kth == 0xFFFFFFFFu) ? kth : kth + 1u;
+#pragma unroll
+                  for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
+                }
+              }
+              named_bar_sync(bar, NTG);
+            }
+#pragma unroll
+            for (int j = 0; j < QPH; ++j) cnt_r[j] = st.cnt_w[j0 + j][qd];
           }
         }
       }
@@ -762,9 +905,10 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
       // ---- end of item: exact top-k of each query's candidates
       if (lane == 0) {
 #pragma unroll
-        for (int jj = 0; jj < QPW; ++jj) st.cnt_w[jj][qd] = cnt_r[jj];
+        for (int j = 0; j < QPH; ++j)
+          if (j < nmine) st.cnt_w[j0 + j][qd] = cnt_r[j];
       }
-      named_bar_sync(bar, 128);
+      named_bar_sync(bar, NTG);
 #pragma unroll 1
       for (int jj = 0; jj < nloc; ++jj) {
         const int t = wi.t0 + g * QPW + jj;
@@ -777,17 +921,17 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
           if (prefix <= kTopK) {
             // every position 0..prefix-1 is a candidate: place each at its own index
             if (gtid == 0) st.ctr[0] = 0;
-            named_bar_sync(bar, 128);
-            compact_view<128>(v, kSlots, st.ctr, gtid, [&](int, uint32_t key, int pos) {
+            named_bar_sync(bar, NTG);
+            compact_view<NTG>(v, kSlots, st.ctr, gtid, [&](int, uint32_t key, int pos) {
               oi[pos] = pos;
               if (os) os[pos] = ordered_to_float(key);
             });
-            for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += 128) {
+            for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += NTG) {
               oi[s2] = -1;
               if (os) os[s2] = -INFINITY;
             }
           } else {
-            select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid, bar,
+            select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch, st.sh, st.ctr, gtid, bar,
                              [&](int s2, uint32_t key, int pos) {
                                oi[s2] = pos;
                                if (os) os[s2] = ordered_to_float(key);
@@ -798,24 +942,24 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>::kThread
           int32_t* pi = p.part_idx + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
           if (n_valid <= kTopK) {
             if (gtid == 0) st.ctr[0] = 0;
-            named_bar_sync(bar, 128);
-            compact_view<128>(v, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
+            named_bar_sync(bar, NTG);
+            compact_view<NTG>(v, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
               pk[rank] = key;
               pi[rank] = pos;
             });
-            for (int e = n_valid + gtid; e < kTopK; e += 128) {
+            for (int e = n_valid + gtid; e < kTopK; e += NTG) {
               pk[e] = 0u;
               pi[e] = -1;
             }
           } else {
-            select_topk<128>(v, kSlots, st.skeys, st.hist, st.scratch, st.sh, st.ctr, gtid, bar,
+            select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch, st.sh, st.ctr, gtid, bar,
                              [&](int s2, uint32_t key, int pos) {
                                pk[s2] = key;
                                pi[s2] = pos;
                              });
           }
         }
-        named_bar_sync(bar, 128);
+        named_bar_sync(bar, NTG);
       }
     }
   }
@@ -838,8 +982,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
                                                               float* __restrict__ score_out) {
   extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK]
   __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t scratch[32];
-  __shared__ int sh[4];
+  __shared__ uint32_t mlist[kRankList];
+  __shared__ uint32_t scratch[64];
+  __shared__ int sh[8];
   __shared__ int ctr[2];
   const int t = blockIdx.x;
   const int nch = tok_nchunks[t];
@@ -850,7 +995,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   v.i = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
   int32_t* oi = idx_out + static_cast<size_t>(t) * kTopK;
   float* os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
-  select_topk<kMergeThreads>(v, n, mkeys, hist, scratch, sh, ctr, threadIdx.x, 1, [&](int slot, uint32_t key, int pos) {
+  select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
+                             [&](int slot, uint32_t key, int pos) {
     oi[slot] = pos;
     if (os) os[slot] = ordered_to_float(key);
   });
@@ -1057,13 +1203,24 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
   *status = ok ? 0 : ((err & kErrTimeout) ? 2 : 1);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
 cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const ScoreParams& p, int grid,
                          cudaStream_t s) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG>;
-  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>;
+  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  if (C::kRegSplit) {
+    // setmaxnreg.inc waits until the block's launch allocation can cover the request:
+    // refuse to launch a split that does not fit it rather than wait forever
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    const long launch_regs = static_cast<long>(fa.numRegs) * C::kThreads;
+    const long split_regs = static_cast<long>(C::kCtrlRegs) * C::kEpiWarp0 * 32 +
+                            static_cast<long>(C::kEpiRegs) * NWG * C::kGroupThreads;
+    if (split_regs > launch_regs) return cudaErrorInvalidConfiguration;
+  }
   kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tmQ, tmK, p);
   return cudaGetLastError();
 }
@@ -1103,7 +1260,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
   if (a.split) {
-    e = launch_score<1, 5, 4, 1>(tmQ1, tmK, sp, grid, s);
+    e = launch_score<1, 5, 4, 1, 4>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
     const int msmem = kMaxChunks * kTopK * 4;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
@@ -1112,7 +1269,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
                                                     a.score_out);
     return cudaGetLastError();
   }
-  return launch_score<kPrefillQ, 3, 2, 2>(tmQ8, tmK, sp, grid, s);
+  return launch_score<kPrefillQ, 3, 2, 2, 8>(tmQ8, tmK, sp, grid, s);
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s) {
