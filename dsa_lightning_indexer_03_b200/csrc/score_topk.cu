@@ -187,41 +187,25 @@ struct QueryCands {
     return w == 0 ? cnt_w0 : w == 1 ? cnt_w1 : w == 2 ? cnt_w2 : cnt_w3;
   }
 
+  // Branch-free: the 16-byte loads are always issued (the storage is allocated to
+  // capacity, so reading past the occupied count is safe) and the slots beyond the
+  // count are masked, so that consecutive groups' loads can all be in flight at once.
   template <bool kKeys, bool kIdx>
   __device__ __forceinline__ uint32_t load4(int s0, uint4& k, int4& i) const {
-    const uint32_t* kp;
-    const int32_t* ip;
-    int local, cnt;
-    if (s0 < kTopK) {
-      kp = kk;
-      ip = ki;
-      local = s0;
-      cnt = cnt_k;
-    } else {
-      const int w = (s0 - kTopK) / kWarpApp;
-      local = (s0 - kTopK) % kWarpApp;
-      kp = ak + w * kWarpApp;
-      ip = ai + w * kWarpApp;
-      cnt = cnt_w(w);
+    const bool in_keep = s0 < kTopK;
+    const int a = s0 - kTopK;                 // offset inside the append areas (they are contiguous)
+    const int local = in_keep ? s0 : (a % kWarpApp);
+    const int cnt = in_keep ? cnt_k : cnt_w(a / kWarpApp);
+    const int avail = cnt - local;
+    const uint32_t m = avail >= 4 ? 0xFu : (avail <= 0 ? 0u : ((1u << avail) - 1u));
+    if (kKeys) {
+      const uint4 r = *reinterpret_cast<const uint4*>(in_keep ? kk + s0 : ak + a);
+      k = make_uint4((m & 1u) ? r.x : 0u, (m & 2u) ? r.y : 0u, (m & 4u) ? r.z : 0u, (m & 8u) ? r.w : 0u);
     }
-    if (local + 3 < cnt) {
-      if (kKeys) k = *reinterpret_cast<const uint4*>(kp + local);
-      if (kIdx) i = *reinterpret_cast<const int4*>(ip + local);
-      return 0xFu;
+    if (kIdx) {
+      const int4 r = *reinterpret_cast<const int4*>(in_keep ? ki + s0 : ai + a);
+      i = make_int4((m & 1u) ? r.x : -1, (m & 2u) ? r.y : -1, (m & 4u) ? r.z : -1, (m & 8u) ? r.w : -1);
     }
-    uint32_t m = 0;
-    uint32_t kv[4] = {0u, 0u, 0u, 0u};
-    int iv[4] = {-1, -1, -1, -1};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (local + j < cnt) {
-        m |= 1u << j;
-        if (kKeys) kv[j] = kp[local + j];
-        if (kIdx) iv[j] = ip[local + j];
-      }
-    }
-    if (kKeys) k = make_uint4(kv[0], kv[1], kv[2], kv[3]);
-    if (kIdx) i = make_int4(iv[0], iv[1], iv[2], iv[3]);
     return m;
   }
   __device__ __forceinline__ int valid_count() const { return cnt_k + cnt_w0 + cnt_w1 + cnt_w2 + cnt_w3; }
@@ -266,11 +250,8 @@ __device__ void emit_view(const View& v, const uint32_t* skeys, int n, int k, ui
     uint32_t m = 0;
     if (g < n / 4) {
       kk = reinterpret_cast<const uint4*>(skeys)[g];
-      // only groups holding a kept key need their positions
-      if (kk.x >= kth || kk.y >= kth || kk.z >= kth || kk.w >= kth) {
-        uint4 dummy;
-        m = v.template load4<false, true>(4 * g, dummy, ii);
-      }
+      uint4 dummy;
+      m = v.template load4<false, true>(4 * g, dummy, ii);
     }
     uint32_t bg[4], be[4];
     int tg = 0, te = 0;
@@ -631,6 +612,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     // ===================================================== TMA producer
     if (lane == 0) {
       int kstage = 0, qloads = 0;
+      const uint64_t pol_q = l2_policy_evict_first();   // each Q tile is read once
+      const uint64_t pol_k = l2_policy_evict_last();    // key tiles are read by every item of a sequence
       for (int local = 0;; ++local) {
         const int slot = local & 1;
         if (local >= 2 && !mbar_wait(&sched_empty[slot], ((local >> 1) - 1) & 1, wc)) break;
@@ -644,8 +627,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         if (kt1 <= kt0) continue;
         if (qloads > 0 && !mbar_wait(q_empty, (qloads - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(q_full, 2 * C::kQHalf);
-        tma_load_2d(sQ, &tmQ, q_full, 0, wi.t0 * kHeads);
-        tma_load_2d(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * kHeads);
+        tma_load_2d_hint(sQ, &tmQ, q_full, 0, wi.t0 * kHeads, pol_q);
+        tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * kHeads, pol_q);
         ++qloads;
         const int row0 = static_cast<int>(p.cache_offsets[wi.b]);
         bool ok = true;
@@ -657,8 +640,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
           }
           mbar_arrive_expect_tx(&full[s], C::kKStage);
           uint8_t* dst = sK + s * C::kKStage;
-          tma_load_2d(dst, &tmK, &full[s], 0, row0 + kt * kKeyTile);
-          tma_load_2d(dst + C::kKHalf, &tmK, &full[s], 64, row0 + kt * kKeyTile);
+          tma_load_2d_hint(dst, &tmK, &full[s], 0, row0 + kt * kKeyTile, pol_k);
+          tma_load_2d_hint(dst + C::kKHalf, &tmK, &full[s], 64, row0 + kt * kKeyTile, pol_k);
         }
         if (!ok) break;
       }
@@ -923,18 +906,18 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
             if (gtid == 0) st.ctr[0] = 0;
             named_bar_sync(bar, NTG);
             compact_view<NTG>(v, kSlots, st.ctr, gtid, [&](int, uint32_t key, int pos) {
-              oi[pos] = pos;
-              if (os) os[pos] = ordered_to_float(key);
+              __stcs(oi + pos, pos);
+              if (os) __stcs(os + pos, ordered_to_float(key));
             });
             for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += NTG) {
-              oi[s2] = -1;
-              if (os) os[s2] = -INFINITY;
+              __stcs(oi + s2, -1);
+              if (os) __stcs(os + s2, -INFINITY);
             }
           } else {
             select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch, st.sh, st.ctr, gtid, bar,
                              [&](int s2, uint32_t key, int pos) {
-                               oi[s2] = pos;
-                               if (os) os[s2] = ordered_to_float(key);
+                               __stcs(oi + s2, pos);
+                               if (os) __stcs(os + s2, ordered_to_float(key));
                              });
           }
         } else {
@@ -997,8 +980,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   float* os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
   select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
                              [&](int slot, uint32_t key, int pos) {
-    oi[slot] = pos;
-    if (os) os[slot] = ordered_to_float(key);
+    __stcs(oi + slot, pos);
+    if (os) __stcs(os + slot, ordered_to_float(key));
   });
 }
 
