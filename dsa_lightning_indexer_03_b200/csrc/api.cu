@@ -151,8 +151,7 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
   ok = ok && h->alloc(&ws.items, ws.max_items) && h->alloc(&ws.n_items, 4) && h->alloc(&ws.work_counter, 4) &&
        h->alloc(&ws.seq_base, size_t(T) + 2) && h->alloc(&ws.pos_eff, size_t(T)) &&
        h->alloc(&ws.tok_nchunks, size_t(T)) &&
-       h->alloc(&ws.cand_keys, size_t(ws.cand_slots) * kPrefillQ * kCandStride) &&
-       h->alloc(&ws.cand_idx, size_t(ws.cand_slots) * kPrefillQ * kCandStride) &&
+       h->alloc(&ws.cand, size_t(ws.cand_slots) * kPrefillQ * kCandStride) &&
        h->alloc(&ws.part_keys, size_t(ws.part_tokens) * kMaxChunks * kTopK) &&
        h->alloc(&ws.part_idx, size_t(ws.part_tokens) * kMaxChunks * kTopK) && h->alloc(&ws.err, 4);
   if (!ok) {

@@ -43,11 +43,11 @@ cudaError_t launch_transpose_bf16(const __nv_bfloat16* src, int K, int N, __nv_b
                                   cudaStream_t s);
 
 // ---------------------------------------------------------------- score + top-k
-// Candidate storage of one query: two keep sets of kTopK entries (the current
-// best list and the target of the next compaction) and an append area split
-// evenly between the four warps of an epilogue warpgroup.
-constexpr int kAppCap = 2 * kTopK;             // appended candidates before a compaction
-constexpr int kCandStride = 2 * kTopK + kAppCap;  // keep set 0 | keep set 1 | append area
+// Candidate storage of one query, in (ordered score key, position) pairs: two keep
+// sets of kTopK entries (the current best list and the target of the next
+// compaction) and one append area per epilogue warp of the query's lane quadrants.
+constexpr int kWarpApp = 2048;                         // append slots of one warp, per query
+constexpr int kCandStride = 2 * kTopK + 4 * kWarpApp;  // keep 0 | keep 1 | areas 0..3
 constexpr int kMaxChunks = 16;                 // key chunks per query on the split-key path
 constexpr int kMinChunk = 4096;                // shortest key chunk on the split-key path
 constexpr int kSplitMaxTokens = 256;           // split-key path is offered up to this many queries
@@ -71,8 +71,7 @@ struct TopkWorkspace {
   int* seq_base;     // [max(B, T) + 2]
   int* pos_eff;      // [T] validated positions, -1 for an invalid query
   int* tok_nchunks;  // [T] key chunks of each query on the split-key path
-  uint32_t* cand_keys;
-  int32_t* cand_idx;
+  uint2* cand;       // [cand_slots][kPrefillQ][kCandStride]
   int cand_slots;    // CTA slots (x kPrefillQ queries each)
   uint32_t* part_keys;
   int32_t* part_idx;

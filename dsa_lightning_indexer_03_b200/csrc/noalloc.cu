@@ -22,7 +22,7 @@ using namespace dsa;
 
 namespace {
 
-constexpr int kStaticCtas = 12;          // persistent CTAs (candidate areas) the scratch holds
+constexpr int kStaticCtas = 8;           // persistent CTAs (candidate areas) the scratch holds
 constexpr int kStaticMaxTokens = 4096;   // largest T (and B) this entry point accepts
 constexpr int kStaticMaxItems = kStaticMaxTokens + 16;
 
@@ -35,9 +35,8 @@ constexpr size_t kOffSeqBase = kOffItems + align256(size_t(kStaticMaxItems) * si
 constexpr size_t kOffPos = kOffSeqBase + align256(size_t(kStaticMaxTokens + 2) * 4);
 constexpr size_t kOffNch = kOffPos + align256(size_t(kStaticMaxTokens) * 4);
 constexpr size_t kCandEntries = size_t(kStaticCtas) * kPrefillQ * kCandStride;
-constexpr size_t kOffCandKeys = kOffNch + align256(size_t(kStaticMaxTokens) * 4);
-constexpr size_t kOffCandIdx = kOffCandKeys + align256(kCandEntries * 4);
-constexpr size_t kScratchBytes = kOffCandIdx + align256(kCandEntries * 4);
+constexpr size_t kOffCand = kOffNch + align256(size_t(kStaticMaxTokens) * 4);
+constexpr size_t kScratchBytes = kOffCand + align256(kCandEntries * sizeof(uint2));
 static_assert(kScratchBytes == 6473216, "the scratch size is stated in include/dsa_indexer.h");
 
 constexpr int kMaxDevices = 64;
@@ -131,8 +130,7 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const
   ws.seq_base = reinterpret_cast<int*>(base + kOffSeqBase);
   ws.pos_eff = reinterpret_cast<int*>(base + kOffPos);
   ws.tok_nchunks = reinterpret_cast<int*>(base + kOffNch);
-  ws.cand_keys = reinterpret_cast<uint32_t*>(base + kOffCandKeys);
-  ws.cand_idx = reinterpret_cast<int32_t*>(base + kOffCandIdx);
+  ws.cand = reinterpret_cast<uint2*>(base + kOffCand);
   ws.cand_slots = kStaticCtas;
   ws.part_keys = nullptr;
   ws.part_idx = nullptr;

@@ -17,18 +17,18 @@
 //              K-major) once, then 128-key tiles of the key cache into a ring.
 //   warp 1     MMA issuer: D[key, (query, head)] = K_tile (M=128) x Q^T (N=nq*32),
 //              K=128 as 8 tcgen05.mma of K=16, into one of ACC_BUFS TMEM buffers.
-//   warps 2..  epilogue warpgroups (4 warps = the 4 TMEM lane quadrants).  Thread
-//              (quadrant, lane) owns one key; per query it loads that query's 32
-//              head columns (tcgen05.ld 32x32b.x32), applies ReLU and the fp32
-//              head weights in registers, masks s > pos, and appends (score, s)
-//              to its own append area of the query's candidates if the score
-//              reaches the query's running threshold (warp ballot; the counts
-//              stay warp-uniform in registers, no atomics).  When an append area
-//              nears its capacity, the query's keep set and append areas are
-//              compacted into the other keep set holding the exact best 2,048
-//              (histogram selection in shared memory), which raises the
-//              threshold.  At the end of the item each query's candidates are
-//              reduced to exactly the top 2,048 and written out.
+//   epilogue   warpgroups of 4 warps (the 4 TMEM lane quadrants).  Thread (quadrant,
+//              lane) owns one key of the tile; per query it loads that query's 32 head
+//              columns (tcgen05.ld 32x32b.x32), applies ReLU and the fp32 head weights
+//              in registers, masks s > pos, and admits (key, s) when the key reaches the
+//              query's admission threshold: the pair goes to the warp's own append area
+//              (warp ballot, warp-uniform counts in registers, no atomics) and the key is
+//              counted in the query's first-level histogram in shared memory.  Every
+//              kCheckTiles tiles the threshold rises to the lowest bin that still holds
+//              the query's best 2,048 counted keys (a warp scan of the histogram), and a
+//              nearly full append area is compacted to the exact best 2,048.  At the end
+//              of the item each query's candidates are reduced to exactly the top 2,048
+//              in one pass (resolve_topk) and written out.
 
 #include "kernels.h"
 
@@ -46,8 +46,7 @@ struct ScoreParams {
   const int64_t* cache_offsets; // [B+1]
   int32_t* idx_out;             // [T, 2048]
   float* score_out;             // [T, 2048] or null
-  uint32_t* cand_keys;          // [slots][QMAX][kCandStride]
-  int32_t* cand_idx;
+  uint2* cand;                  // [slots][QMAX][kCandStride] (key, position) pairs
   uint32_t* part_keys;          // [T][kMaxChunks][kTopK]
   int32_t* part_idx;
   int* err;
@@ -106,18 +105,18 @@ __device__ __forceinline__ void group_minmax(uint32_t& lo, uint32_t& hi, int tid
 }
 
 constexpr int kHistBins = 1024;   // histogram bins of one selection round
-constexpr int kRankList = 256;    // boundary-bin keys ranked directly
+constexpr int kRankList = 256;    // boundary-bin keys ranked directly (merge path)
 
-// k-th largest of n order-preserving keys held in shared memory (1 <= k <= n), all of
-// them inside [lo, hi] (keys outside are ignored).  Each round histograms the keys of
-// the current window into at most kHistBins bins of width 2^shift, locates the bin that
-// holds the k-th largest, and narrows the window to that bin; a round of width-1 bins
-// ends it (at most four rounds for 32-bit keys).  *n_above receives the number of keys
-// strictly greater than the returned key.  Used where the value-binned round below
-// cannot isolate the boundary (crowded bins: ties, extreme ranges).
-template <int NT>
-__device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo, uint32_t hi, uint32_t* hist,
-                                uint32_t* scratch, int* sh, int tid, int bar, int* n_above) {
+// k-th largest of the order-preserving keys that a group of NT threads visits, among those
+// inside the window [lo, hi] (1 <= k <= their number; keys outside are ignored).
+// keys(f) calls f(key) for every key the calling thread owns; each key has one owner, and
+// keys may be called once per round.  Each round histograms the window into at most
+// kHistBins bins of width 2^shift, locates the bin that holds the k-th largest and narrows
+// the window to it; a round of width-1 bins ends it (at most three rounds for 32-bit keys).
+// *n_above receives the number of keys in the window strictly greater than the result.
+template <int NT, class Keys>
+__device__ uint32_t kth_window(const Keys& keys, int k, uint32_t lo, uint32_t hi, uint32_t* hist,
+                               uint32_t* scratch, int* sh, int tid, int bar, int* n_above) {
   constexpr int kBPT = kHistBins / NT;  // bins owned by one thread when locating the k-th
   uint32_t base = lo, span = hi - lo;
   int need = k, above_total = 0;
@@ -126,10 +125,10 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
     const int shift = (span >> 10) ? 32 - __clz(static_cast<int>(span >> 10)) : 0;
     for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
     named_bar_sync(bar, NT);
-    for (int e = tid; e < n; e += NT) {
-      const uint32_t d = keys[e] - base;
+    keys([&](uint32_t key) {
+      const uint32_t d = key - base;
       if (d <= span) atomicAdd(&hist[d >> shift], 1u);
-    }
+    });
     named_bar_sync(bar, NT);
     const int b0 = tid * kBPT;
     uint32_t c[kBPT];
@@ -167,49 +166,19 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
   }
 }
 
-// Candidate views: a fixed set of slots (a multiple of 4), some of them empty.
-// load4(s0, k, i) fetches slots s0..s0+3 with 16-byte loads where the four are all
-// occupied and returns the occupied-slot mask; empty slots read key 0, position -1.
-constexpr int kWarpApp = kAppCap / 4;      // append slots of one epilogue warp
-constexpr int kSlots = kTopK + kAppCap;    // keep set + append area of one query
+// kth_window over n keys held in shared memory.
+template <int NT>
+__device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo, uint32_t hi, uint32_t* hist,
+                                uint32_t* scratch, int* sh, int tid, int bar, int* n_above) {
+  auto visit = [&](auto f) {
+    for (int e = tid; e < n; e += NT) f(keys[e]);
+  };
+  return kth_window<NT>(visit, k, lo, hi, hist, scratch, sh, tid, bar, n_above);
+}
 
-// The candidates of one query in the score kernel: the current keep set (slots
-// 0..kTopK-1) followed by the four warps' append areas (kWarpApp slots each).
-struct QueryCands {
-  const uint32_t* kk;
-  const int32_t* ki;
-  const uint32_t* ak;
-  const int32_t* ai;
-  int cnt_k;
-  int cnt_w0, cnt_w1, cnt_w2, cnt_w3;   // scalars: a runtime-indexed array would live in local memory
+// ------------------------------------------------------------------------------------------
+// Selection over dense lists (the merge of the split-key path's partial lists).
 
-  __device__ __forceinline__ int cnt_w(int w) const {
-    return w == 0 ? cnt_w0 : w == 1 ? cnt_w1 : w == 2 ? cnt_w2 : cnt_w3;
-  }
-
-  // Branch-free: the 16-byte loads are always issued (the storage is allocated to
-  // capacity, so reading past the occupied count is safe) and the slots beyond the
-  // count are masked, so that consecutive groups' loads can all be in flight at once.
-  template <bool kKeys, bool kIdx>
-  __device__ __forceinline__ uint32_t load4(int s0, uint4& k, int4& i) const {
-    const bool in_keep = s0 < kTopK;
-    const int a = s0 - kTopK;                 // offset inside the append areas (they are contiguous)
-    const int local = in_keep ? s0 : (a % kWarpApp);
-    const int cnt = in_keep ? cnt_k : cnt_w(a / kWarpApp);
-    const int avail = cnt - local;
-    const uint32_t m = avail >= 4 ? 0xFu : (avail <= 0 ? 0u : ((1u << avail) - 1u));
-    if (kKeys) {
-      const uint4 r = *reinterpret_cast<const uint4*>(in_keep ? kk + s0 : ak + a);
-      k = make_uint4((m & 1u) ? r.x : 0u, (m & 2u) ? r.y : 0u, (m & 4u) ? r.z : 0u, (m & 8u) ? r.w : 0u);
-    }
-    if (kIdx) {
-      const int4 r = *reinterpret_cast<const int4*>(in_keep ? ki + s0 : ai + a);
-      i = make_int4((m & 1u) ? r.x : -1, (m & 2u) ? r.y : -1, (m & 4u) ? r.z : -1, (m & 8u) ? r.w : -1);
-    }
-    return m;
-  }
-  __device__ __forceinline__ int valid_count() const { return cnt_k + cnt_w0 + cnt_w1 + cnt_w2 + cnt_w3; }
-};
 
 // A dense list of n slots (n a multiple of 4); slots with position < 0 are empty.
 struct FlatCands {
@@ -281,38 +250,6 @@ __device__ void emit_view(const View& v, const uint32_t* skeys, int n, int k, ui
         }
         b0 += __popc(bg[j]);
         b1 += __popc(be[j]);
-      }
-    }
-  }
-}
-
-// Calls sink(rank, key, pos) for every occupied slot, ranks 0..count-1 (order unspecified).
-template <int NT, class View, class Sink>
-__device__ void compact_view(const View& v, int n, int* ctr, int tid, Sink sink) {
-  const int lane = tid & 31;
-  const uint32_t lt = lanemask_lt();
-#pragma unroll 2
-  for (int base = 0; base < n / 4; base += NT) {
-    const int g = base + tid;
-    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
-    int4 ii = make_int4(-1, -1, -1, -1);
-    uint32_t m = 0;
-    if (g < n / 4) m = v.template load4<true, true>(4 * g, kk, ii);
-    uint32_t b[4];
-    int tot = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      b[j] = __ballot_sync(0xffffffffu, (m >> j) & 1u);
-      tot += __popc(b[j]);
-    }
-    if (tot) {
-      int b0 = 0;
-      if (lane == 0) b0 = atomicAdd(&ctr[0], tot);
-      b0 = __shfl_sync(0xffffffffu, b0, 0);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if ((b[j] >> lane) & 1u) sink(b0 + __popc(b[j] & lt), u4_get(kk, j), i4_get(ii, j));
-        b0 += __popc(b[j]);
       }
     }
   }
@@ -475,20 +412,354 @@ __device__ uint32_t select_topk(const View& v, int n, uint32_t* skeys, uint32_t*
 }
 
 // ------------------------------------------------------------------------------------------
+// Candidates of the score kernel.  A query's candidates are (ordered key, position) pairs:
+// its current keep set and the append areas of the four epilogue warps that own its key
+// rows.  Beside them, in shared memory, the query keeps the count of its candidates in
+// each of kBins1 first-level bins (bin = the key's top 11 bits: sign, exponent and two
+// mantissa bits of the score), two 16-bit counts per word.  The counts drive both the
+// admission threshold while scores stream in and the exact selection at the end.
+constexpr int kBinShift = 21;                  // first-level bin = key >> kBinShift
+constexpr int kBins1 = 1 << (32 - kBinShift);  // 2,048 bins
+constexpr int kSubShift = kBinShift - 11;      // second-level bin = next 11 bits
+constexpr int kListCap = 1024;                 // boundary-bin candidates gathered in shared memory
+constexpr int kCheckTiles = 4;                 // key tiles between threshold updates / capacity checks
+constexpr int kCheckMargin = kCheckTiles * 32; // appends one warp can make per query in that time
+constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
+
+__device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
+  atomicAdd(&h[bin >> 1], (bin & 1u) ? 0x10000u : 1u);
+}
+
+// Entry e (0..7) of a round: entries 2i and 2i+1 sit in x[i].
+__device__ __forceinline__ uint2 round_entry(const uint4 (&x)[4], int e) {
+  return (e & 1) ? make_uint2(x[e >> 1].z, x[e >> 1].w) : make_uint2(x[e >> 1].x, x[e >> 1].y);
+}
+
+struct CandView {
+  const uint2* keep;   // the current keep set
+  const uint2* area;   // warp w's append area starts at area + w * kWarpApp
+  int nk, n0, n1, n2, n3;
+  __device__ __forceinline__ int total() const { return nk + n0 + n1 + n2 + n3; }
+
+  // Calls f(x, lim) once per round.  A round gives each thread up to eight candidates,
+  // read in pairs with 16-byte loads: x[i] holds entries 2i and 2i+1, lim[i] how many of
+  // the two are valid.  Every thread of the group makes the same calls, so f may use
+  // warp-collective operations.
+  template <int NT, class F>
+  __device__ __forceinline__ void for_rounds(int tid, F&& f) const {
+    const int u0 = (nk + 1) >> 1;
+    const int u1 = u0 + ((n0 + 1) >> 1);
+    const int u2 = u1 + ((n1 + 1) >> 1);
+    const int u3 = u2 + ((n2 + 1) >> 1);
+    const int u4 = u3 + ((n3 + 1) >> 1);
+#pragma unroll 1
+    for (int base = 0; base < u4; base += 4 * NT) {
+      uint4 x[4];
+      int lim[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int u = base + i * NT + tid;
+        const uint2* p;
+        int off, cnt;
+        if (u < u0) { p = keep; off = u; cnt = nk; }
+        else if (u < u1) { p = area; off = u - u0; cnt = n0; }
+        else if (u < u2) { p = area + kWarpApp; off = u - u1; cnt = n1; }
+        else if (u < u3) { p = area + 2 * kWarpApp; off = u - u2; cnt = n2; }
+        else { p = area + 3 * kWarpApp; off = u - u3; cnt = n3; }
+        lim[i] = u < u4 ? min(2, cnt - 2 * off) : 0;
+        x[i] = lim[i] > 0 ? *reinterpret_cast<const uint4*>(p + 2 * off) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      f(x, lim);
+    }
+  }
+};
+
+// Calls f(rank, entry) for every candidate, ranks 0..total-1 (order unspecified);
+// *ctr is a shared counter zeroed beforehand.
+template <int NT, class F>
+__device__ __forceinline__ void collect(const CandView& v, int* ctr, int tid, F&& f) {
+  const int lane = tid & 31;
+  const uint32_t lt = lanemask_lt();
+  v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+    uint32_t b[8];
+    int tot = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      b[e] = __ballot_sync(0xffffffffu, lim[e >> 1] > (e & 1));
+      tot += __popc(b[e]);
+    }
+    if (tot) {
+      int o = 0;
+      if (lane == 0) o = atomicAdd(ctr, tot);
+      o = __shfl_sync(0xffffffffu, o, 0);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if ((b[e] >> lane) & 1u) f(o + __popc(b[e] & lt), round_entry(x, e));
+        o += __popc(b[e]);
+      }
+    }
+  });
+}
+
+// Bin b of kBins1 bins, counted two per word in hw, that holds the need-th largest counted
+// key: count(bins > b) < need <= count(bins >= b) (need <= the total count).  Returns b and
+// sets *above = count(bins > b); sh[0..1] carry the result.  With `clear` each thread
+// zeroes the words it read.
+template <int NT>
+__device__ int locate_packed(uint32_t* hw, uint32_t need, bool clear, uint32_t* scratch, int* sh, int tid, int bar,
+                             uint32_t* above) {
+  constexpr int kWPT = (kBins1 / 2) / NT;  // words per thread
+  const int w0 = tid * kWPT;
+  uint32_t c[2 * kWPT];
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < kWPT; ++i) {
+    const uint32_t word = hw[w0 + i];
+    c[2 * i] = word & 0xFFFFu;
+    c[2 * i + 1] = word >> 16;
+    s += c[2 * i] + c[2 * i + 1];
+  }
+  if (clear) {
+#pragma unroll
+    for (int i = 0; i < kWPT; ++i) hw[w0 + i] = 0u;
+  }
+  const uint32_t above_t = group_suffix_excl<NT>(s, tid, scratch, bar);
+  if (above_t < need && need <= above_t + s) {
+    uint32_t cum = above_t;
+#pragma unroll
+    for (int i = 2 * kWPT - 1; i >= 0; --i) {
+      if (cum + c[i] >= need) {
+        sh[0] = 2 * w0 + i;
+        sh[1] = static_cast<int>(cum);
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  named_bar_sync(bar, NT);
+  const int b = sh[0];
+  *above = static_cast<uint32_t>(sh[1]);
+  return b;
+}
+
+// One warp: the highest bin b with count(bins >= b) >= need in a packed kBins1-bin
+// histogram, or 0 if the histogram holds fewer than need keys.  Lane l first sums bins
+// 64l..64l+63 (the total of all counts stays below 2^16, so the two halves of a word sum
+// can be added without carries), then the lanes scan the 64 bins of the crossing.  Counts
+// may be growing meanwhile: the result is then a lower bound of the exact one.
+__device__ __forceinline__ int scan_bins_warp(const uint32_t* hw, uint32_t need, int lane) {
+  const uint4* q = reinterpret_cast<const uint4*>(hw) + lane * 8;
+  uint32_t s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 x = q[(i + lane) & 7];   // rotated: the lanes of one load cover every bank
+    s += x.x + x.y + x.z + x.w;
+  }
+  const uint32_t cnt = (s & 0xFFFFu) + (s >> 16);
+  uint32_t x = cnt;   // inclusive suffix over lanes >= lane
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
+    if (lane + off < 32) x += y;
+  }
+  const uint32_t m = __ballot_sync(0xffffffffu, x >= need);
+  if (!m) return 0;
+  const int ls = 31 - __clz(m);
+  const uint32_t run = __shfl_sync(0xffffffffu, x - cnt, ls);   // count above lane ls's bins
+  const uint32_t word = hw[ls * 32 + lane];
+  const uint32_t lo = word & 0xFFFFu;
+  uint32_t z = lo + (word >> 16);
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, z, off);
+    if (lane + off < 32) z += y;
+  }
+  const uint32_t cum_even = run + z;        // count(bins >= 64 ls + 2 lane)
+  const uint32_t cum_odd = cum_even - lo;   // count(bins >= 64 ls + 2 lane + 1)
+  const uint32_t m2 = __ballot_sync(0xffffffffu, cum_even >= need);
+  const int l = 31 - __clz(m2);             // m2 holds lane 0 at least
+  const uint32_t co = __shfl_sync(0xffffffffu, cum_odd, l);
+  return 64 * ls + 2 * l + (co >= need ? 1 : 0);
+}
+
+struct ResolveSmem {
+  uint32_t* rh;      // kBins1 / 2 words: second-level counts, then kth_window's bins
+  uint2* list;       // kListCap boundary-bin candidates
+  uint32_t* small;   // kSmallRank keys of the boundary sub-bin
+  uint32_t* scratch;
+  int* sh;
+  int* ctr;          // four shared counters
+};
+
+// Exact top kTopK of a query's candidates (at least kTopK of them), given h1, the packed
+// first-level counts of exactly those candidates:
+// 1. locate the bin b1 that holds the kTopK-th largest key; `above` keys lie above it;
+// 2. one pass over the candidates: keys above b1 go to slots [0, above); keys in b1 are
+//    gathered into the list and counted by their next 11 bits;
+// 3. locate the boundary's second-level bin b2 and find the exact kTopK-th largest key K*
+//    inside it: one warp ranks a small sub-bin, else a histogram round runs over the list
+//    (or over the candidates again when the list overflowed);
+// 4. emit the keys of b1 greater than K* and the first kTopK - n_above keys equal to K*.
+// sink(slot, key, pos) is called once for each slot 0..kTopK-1.  With clear_h1 the words
+// of h1 are zeroed before the first sink call.  Returns K*.
+template <int NT, class Sink>
+__device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1, const ResolveSmem& rs, int tid,
+                                 int bar, Sink&& sink) {
+  const int lane = tid & 31;
+  const uint32_t lt = lanemask_lt();
+  for (int i = tid; i < kBins1 / 2; i += NT) rs.rh[i] = 0u;
+  if (tid == 0) {
+    rs.ctr[0] = 0;
+    rs.ctr[1] = 0;
+    rs.ctr[2] = 0;
+    rs.ctr[3] = 0;
+  }
+  // 1. (its barriers also publish the zeroed scratch)
+  uint32_t above;
+  const int b1 = locate_packed<NT>(h1, kTopK, clear_h1, rs.scratch, rs.sh, tid, bar, &above);
+  const uint32_t ub1 = static_cast<uint32_t>(b1);
+  // 2.
+  v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+    uint32_t bu[8], ba[8];
+    int tu = 0, ta = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t b = round_entry(x, e).x >> kBinShift;
+      const bool ok = lim[e >> 1] > (e & 1);
+      bu[e] = __ballot_sync(0xffffffffu, ok && b > ub1);
+      ba[e] = __ballot_sync(0xffffffffu, ok && b == ub1);
+      tu += __popc(bu[e]);
+      ta += __popc(ba[e]);
+    }
+    if (tu | ta) {
+      int ou = 0, oa = 0;
+      if (lane == 0) {
+        if (tu) ou = atomicAdd(&rs.ctr[0], tu);
+        if (ta) oa = atomicAdd(&rs.ctr[1], ta);
+      }
+      ou = __shfl_sync(0xffffffffu, ou, 0);
+      oa = __shfl_sync(0xffffffffu, oa, 0);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint2 c = round_entry(x, e);
+        if ((bu[e] >> lane) & 1u) {
+          const int o = ou + __popc(bu[e] & lt);
+          if (o < kTopK) sink(o, c.x, c.y);
+        }
+        if ((ba[e] >> lane) & 1u) {
+          const int o = oa + __popc(ba[e] & lt);
+          if (o < kListCap) rs.list[o] = c;
+          count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
+        }
+        ou += __popc(bu[e]);
+        oa += __popc(ba[e]);
+      }
+    }
+  });
+  named_bar_sync(bar, NT);
+  const int m = rs.ctr[1];
+  // 3.
+  const uint32_t need2 = kTopK - above;
+  uint32_t above2;
+  const int b2 = locate_packed<NT>(rs.rh, need2, false, rs.scratch, rs.sh + 2, tid, bar, &above2);
+  const uint32_t lo = (ub1 << kBinShift) | (static_cast<uint32_t>(b2) << kSubShift);
+  const uint32_t hi = lo + ((1u << kSubShift) - 1u);
+  const int need3 = static_cast<int>(need2 - above2);
+  const int m2 = static_cast<int>((rs.rh[b2 >> 1] >> ((b2 & 1) * 16)) & 0xFFFFu);
+  const bool in_list = m <= kListCap;
+  int n3;
+  uint32_t kth;
+  if (in_list && m2 <= kSmallRank) {
+    // gather the sub-bin's keys; one warp ranks them
+    for (int e = tid; e < m; e += NT) {
+      const uint32_t key = rs.list[e].x;
+      if (key - lo <= hi - lo) {
+        const int o = atomicAdd(&rs.ctr[3], 1);
+        if (o < kSmallRank) rs.small[o] = key;
+      }
+    }
+    named_bar_sync(bar, NT);
+    if (tid < 32) {
+      const uint32_t mine = lane < m2 ? rs.small[lane] : 0u;
+      int gt = 0, eq = 0;
+      for (int j = 0; j < m2; ++j) {
+        const uint32_t y = __shfl_sync(0xffffffffu, mine, j);
+        gt += y > mine;
+        eq += y == mine;
+      }
+      if (lane < m2 && gt < need3 && need3 <= gt + eq) {   // every finder writes the same values
+        rs.sh[4] = static_cast<int>(mine);
+        rs.sh[5] = gt;
+      }
+    }
+    named_bar_sync(bar, NT);
+    kth = static_cast<uint32_t>(rs.sh[4]);
+    n3 = rs.sh[5];
+  } else if (in_list) {
+    auto keys = [&](auto f) {
+      for (int e = tid; e < m; e += NT) f(rs.list[e].x);
+    };
+    kth = kth_window<NT>(keys, need3, lo, hi, rs.rh, rs.scratch, rs.sh, tid, bar, &n3);
+  } else {
+    auto keys = [&](auto f) {
+      v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (lim[e >> 1] > (e & 1)) f(round_entry(x, e).x);
+      });
+    };
+    kth = kth_window<NT>(keys, need3, lo, hi, rs.rh, rs.scratch, rs.sh, tid, bar, &n3);
+  }
+  const int n_above = static_cast<int>(above + above2) + n3;
+  const int ties = kTopK - n_above;
+  // 4. slots below n_above continue rs.ctr[0] (== above after step 2); ties count in ctr[2]
+  auto fin = [&](uint2 c, bool ok) {
+    const bool in = ok && (c.x >> kBinShift) == ub1;
+    const bool gt = in && c.x > kth, eq = in && c.x == kth;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    if (bg | be) {
+      int og = 0, oe = 0;
+      if (lane == 0) {
+        if (bg) og = atomicAdd(&rs.ctr[0], __popc(bg));
+        if (be) oe = atomicAdd(&rs.ctr[2], __popc(be));
+      }
+      og = __shfl_sync(0xffffffffu, og, 0) + __popc(bg & lt);
+      oe = __shfl_sync(0xffffffffu, oe, 0) + __popc(be & lt);
+      if (gt && og < kTopK) sink(og, c.x, c.y);
+      if (eq && oe < ties && n_above + oe >= 0) sink(n_above + oe, c.x, c.y);
+    }
+  };
+  if (in_list) {
+    for (int base = 0; base < m; base += NT) {
+      const int e = base + tid;
+      const bool ok = e < m;
+      fin(ok ? rs.list[e] : make_uint2(0u, 0u), ok);
+    }
+  } else {
+    v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) fin(round_entry(x, e), lim[e >> 1] > (e & 1));
+    });
+  }
+  return kth;
+}
+
+// ------------------------------------------------------------------------------------------
 template <int QPW>
 struct WGState {
-  uint32_t skeys[kSlots];     // staged candidate keys of one selection
-  uint32_t hist[kHistBins];
-  uint32_t list[kRankList];   // keys of the boundary bin
+  uint32_t hist[QPW][kBins1 / 2];  // per query: first-level counts of its candidates (packed)
+  uint32_t rhist[kBins1 / 2];      // resolution scratch
+  uint2 list[kListCap];            // boundary-bin candidates of one resolution
+  uint32_t small[kSmallRank];      // keys of the boundary sub-bin
   float w[QPW][kHeads];
-  int cnt_w[QPW][4];          // per-warp append counts, published at barriers
-  int cnt_k[QPW];             // entries in the current keep set
-  int kcur[QPW];              // which keep set is current
-  uint32_t thr[QPW];          // smallest key still admitted
+  int cnt_w[QPW][4];               // per-warp append counts, published at check points
+  int cnt_k[QPW];                  // entries in the current keep set
+  int kcur[QPW];                   // which keep set is current
+  uint32_t thr[QPW];               // exact admission threshold left by a compaction
   int pos[QPW];
   uint32_t scratch[64];
   int sh[8];
-  int ctr[2];
+  int ctr[4];
 };
 
 // Thread layout of the score kernel.  EW = epilogue warps per group: 4 (one warp per
@@ -704,7 +975,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     }
     const int ew = warp - C::kEpiWarp0;
     const int g = ew / EW;                   // epilogue group = a set of QPW queries of the item
-    const int hq = (ew % EW) / 4;            // which half of the group's queries this warp scores
+    const int hq = (ew % EW) / 4;            // which part of the group's queries this warp scores
     const int qd = warp & 3;                 // TMEM lane quadrant of this warp (also its append area)
     const int gtid = threadIdx.x - C::kEpiWarp0 * 32 - g * NTG;
     const int bar = 1 + g;
@@ -712,25 +983,29 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     const uint32_t lt = lanemask_lt();
     WGState<QPW>& st = *reinterpret_cast<WGState<QPW>*>(smem + C::kWGOff + g * C::kWGBytes);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-    const size_t slot_base = static_cast<size_t>(blockIdx.x) * QMAX + g * QPW;
     const int j0 = hq * QPH;                 // first of this warp's queries inside the group
+    // candidates of query jj of this group start at qcand + jj * kCandStride
+    uint2* const qcand = p.cand + (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW) * kCandStride;
+    uint2* const my_area = qcand + static_cast<size_t>(j0) * kCandStride + 2 * kTopK + qd * kWarpApp;
+    const ResolveSmem rs{st.rhist, st.list, st.small, st.scratch, st.sh, st.ctr};
     int acc_ctr = 0;
 
     // the candidates of query jj of this group, with the published counts
     auto cands = [&](int jj) {
-      const size_t q = (slot_base + jj) * kCandStride;
-      QueryCands v;
-      v.kk = p.cand_keys + q + st.kcur[jj] * kTopK;
-      v.ki = p.cand_idx + q + st.kcur[jj] * kTopK;
-      v.ak = p.cand_keys + q + 2 * kTopK;
-      v.ai = p.cand_idx + q + 2 * kTopK;
-      v.cnt_k = st.cnt_k[jj];
-      v.cnt_w0 = st.cnt_w[jj][0];
-      v.cnt_w1 = st.cnt_w[jj][1];
-      v.cnt_w2 = st.cnt_w[jj][2];
-      v.cnt_w3 = st.cnt_w[jj][3];
+      const uint2* q = qcand + static_cast<size_t>(jj) * kCandStride;
+      CandView v;
+      v.keep = q + st.kcur[jj] * kTopK;
+      v.area = q + 2 * kTopK;
+      v.nk = st.cnt_k[jj];
+      v.n0 = st.cnt_w[jj][0];
+      v.n1 = st.cnt_w[jj][1];
+      v.n2 = st.cnt_w[jj][2];
+      v.n3 = st.cnt_w[jj][3];
       return v;
     };
+
+    // the histograms start empty (ordered before any count by the item barrier)
+    for (int i = gtid; i < QPW * (kBins1 / 2); i += NTG) (&st.hist[0][0])[i] = 0u;
 
     for (int local = 0;; ++local) {
       const int slot = local & 1;
@@ -760,17 +1035,22 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
       const int nloc = min(QPW, wi.nq - g * QPW);  // queries of the group present in this item
       const int nmine = min(QPH, nloc - j0);        // ... and scored by this warp (may be <= 0)
       const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
-      int cnt_r[QPH];
+      // an item of at most kWarpApp / 32 tiles cannot fill an append area: no capacity checks
+      const bool long_item = (kt1 - kt0) * 32 > kWarpApp;
+      int cnt_r[QPH], pos_r[QPH];
+      uint32_t thr_r[QPH];
 #pragma unroll
-      for (int j = 0; j < QPH; ++j) cnt_r[j] = 0;
+      for (int j = 0; j < QPH; ++j) {
+        cnt_r[j] = 0;
+        thr_r[j] = 0u;
+        pos_r[j] = (j < nmine) ? min(st.pos[j0 + j], wi.k_end - 1) : -2;   // last key position scored
+      }
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
         const int ab = acc_ctr % ACC_BUFS;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (acc_ctr / ACC_BUFS) & 1, wc));
         tc_fence_after();
-        bool need = false;
         const int s_pos = kt * kKeyTile + r;
-        const bool in_range = s_pos < wi.k_end;
         const uint32_t tcol = tlane + ab * C::kAccCols + (g * QPW + j0) * kHeads;
         if (ok) {
           float score[QPH];
@@ -801,58 +1081,54 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[ab]);
           }
-          // append (score, position) to this warp's area of each of its queries; the
-          // counts stay warp-uniform in registers
+          // admit (key, position) into this warp's area of each of its queries and count it;
+          // the append counts stay warp-uniform in registers
 #pragma unroll
           for (int j = 0; j < QPH; ++j) {
             if (j >= nmine) break;
-            const int jj = j0 + j;
             const uint32_t u = float_to_ordered(score[j]);
-            const bool pass = in_range && (s_pos <= st.pos[jj]) && (u >= st.thr[jj]);
+            const bool pass = (s_pos <= pos_r[j]) && (u >= thr_r[j]);
             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
             if (pass) {
-              const size_t q = (slot_base + jj) * kCandStride + 2 * kTopK + qd * kWarpApp + cnt_r[j] +
-                               __popc(bal & lt);
-              p.cand_keys[q] = u;
-              p.cand_idx[q] = s_pos;
+              my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)] =
+                  make_uint2(u, static_cast<uint32_t>(s_pos));
+              count_key(st.hist[j0 + j], u >> kBinShift);
             }
             cnt_r[j] += __popc(bal);
-            need |= cnt_r[j] > kWarpApp - 2 * 32;
           }
         } else {
           failed = true;
         }
-        // capacity check every other tile (an append area takes at most 32 entries per tile)
-        if (((kt - kt0) & 1) == 1 || kt + 1 == kt1) {   // the same tiles for every warp of the group
-          if (named_bar_or(bar, NTG, need || failed)) {
-            if (named_bar_or(bar, NTG, failed)) { failed = true; break; }
-            if (lane == 0) {
+        // check point every kCheckTiles tiles (the same tiles for every warp of the group)
+        if ((kt - kt0) % kCheckTiles == kCheckTiles - 1 && kt + 1 < kt1) {
+          bool need = false;
+          if (long_item) {
 #pragma unroll
-              for (int j = 0; j < QPH; ++j)
-                if (j < nmine) st.cnt_w[j0 + j][qd] = cnt_r[j];
+            for (int j = 0; j < QPH; ++j) {
+              if (j < nmine) {
+                need |= cnt_r[j] > kWarpApp - kCheckMargin;
+                if (lane == 0) st.cnt_w[j0 + j][qd] = cnt_r[j];
+              }
             }
-            named_bar_sync(bar, NTG);
+          }
+          if (long_item && named_bar_or(bar, NTG, need || failed)) {
+            if (named_bar_or(bar, NTG, failed)) { failed = true; break; }
 #pragma unroll 1
             for (int jj = 0; jj < nloc; ++jj) {
               // st.*[jj] is read by every thread here and written only after the barriers below
-              const QueryCands v = cands(jj);
-              const int cmax = max(max(v.cnt_w0, v.cnt_w1), max(v.cnt_w2, v.cnt_w3));
-              if (cmax <= kWarpApp - 2 * 32) continue;
-              const size_t q = (slot_base + jj) * kCandStride;
+              const CandView v = cands(jj);
+              if (max(max(v.n0, v.n1), max(v.n2, v.n3)) <= kWarpApp - kCheckMargin) continue;
+              uint2* const q = qcand + static_cast<size_t>(jj) * kCandStride;
               const int kc = st.kcur[jj];
-              const int n_valid = v.valid_count();
+              const int n_valid = v.total();
               if (n_valid <= kTopK) {
-                // fewer than kTopK so far: move the append areas into the keep set
-                uint32_t* kk = p.cand_keys + q + kc * kTopK;
-                int32_t* ki = p.cand_idx + q + kc * kTopK;
+                // fewer than kTopK so far: move the append areas behind the keep set
+                uint2* const kk = q + kc * kTopK + v.nk;
                 if (gtid == 0) st.ctr[0] = 0;
                 named_bar_sync(bar, NTG);
-                QueryCands a = v;
-                a.cnt_k = 0;
-                compact_view<NTG>(a, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
-                  kk[v.cnt_k + rank] = key;
-                  ki[v.cnt_k + rank] = pos;
-                });
+                CandView a = v;
+                a.nk = 0;
+                collect<NTG>(a, st.ctr, gtid, [&](int rank, uint2 x) { kk[rank] = x; });
                 named_bar_sync(bar, NTG);
                 if (gtid == 0) {
                   st.cnt_k[jj] = n_valid;
@@ -860,13 +1136,13 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
                   for (int w = 0; w < 4; ++w) st.cnt_w[jj][w] = 0;
                 }
               } else {
-                uint32_t* kn = p.cand_keys + q + (kc ^ 1) * kTopK;
-                int32_t* in = p.cand_idx + q + (kc ^ 1) * kTopK;
-                const uint32_t kth = select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch,
-                                                      st.sh, st.ctr, gtid, bar, [&](int s2, uint32_t key, int pos) {
-                                                        kn[s2] = key;
-                                                        in[s2] = pos;
-                                                      });
+                // keep exactly the best kTopK (in the other keep set) and count them afresh
+                uint2* const kn = q + (kc ^ 1) * kTopK;
+                uint32_t* const h = st.hist[jj];
+                const uint32_t kth = resolve_topk<NTG>(v, h, true, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+                  kn[s2] = make_uint2(key, pos);
+                  count_key(h, key >> kBinShift);
+                });
                 named_bar_sync(bar, NTG);
                 if (gtid == 0) {
                   st.cnt_k[jj] = kTopK;
@@ -879,46 +1155,61 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
               named_bar_sync(bar, NTG);
             }
 #pragma unroll
-            for (int j = 0; j < QPH; ++j) cnt_r[j] = st.cnt_w[j0 + j][qd];
+            for (int j = 0; j < QPH; ++j) {
+              if (j < nmine) {
+                cnt_r[j] = st.cnt_w[j0 + j][qd];
+                thr_r[j] = max(thr_r[j], st.thr[j0 + j]);
+              }
+            }
+          }
+          // raise each query's admission threshold to the lowest bin of its best kTopK (the
+          // counts need no barrier: a count read early only lowers the bin found)
+#pragma unroll
+          for (int j = 0; j < QPH; ++j) {
+            if (j < nmine) {
+              const int b = scan_bins_warp(st.hist[j0 + j], kTopK, lane);
+              thr_r[j] = max(thr_r[j], static_cast<uint32_t>(b) << kBinShift);
+            }
           }
         }
       }
-      if (failed) break;
-
       // ---- end of item: exact top-k of each query's candidates
       if (lane == 0) {
 #pragma unroll
         for (int j = 0; j < QPH; ++j)
           if (j < nmine) st.cnt_w[j0 + j][qd] = cnt_r[j];
       }
-      named_bar_sync(bar, NTG);
+      if (named_bar_or(bar, NTG, failed)) break;   // a failed wait ends every warp of the group
 #pragma unroll 1
       for (int jj = 0; jj < nloc; ++jj) {
         const int t = wi.t0 + g * QPW + jj;
-        const QueryCands v = cands(jj);
-        const int n_valid = v.valid_count();
+        const CandView v = cands(jj);
+        const int n_valid = v.total();
         if (wi.chunk < 0) {
           int32_t* oi = p.idx_out + static_cast<size_t>(t) * kTopK;
           float* os = p.score_out ? p.score_out + static_cast<size_t>(t) * kTopK : nullptr;
           const int prefix = st.pos[jj] + 1;   // keys this query scores (<= 0 if invalid)
           if (prefix <= kTopK) {
             // every position 0..prefix-1 is a candidate: place each at its own index
-            if (gtid == 0) st.ctr[0] = 0;
-            named_bar_sync(bar, NTG);
-            compact_view<NTG>(v, kSlots, st.ctr, gtid, [&](int, uint32_t key, int pos) {
-              __stcs(oi + pos, pos);
-              if (os) __stcs(os + pos, ordered_to_float(key));
+            v.for_rounds<NTG>(gtid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const uint2 c = round_entry(x, e);
+                if (lim[e >> 1] > (e & 1) && c.y < static_cast<uint32_t>(kTopK)) {
+                  __stcs(oi + c.y, static_cast<int>(c.y));
+                  if (os) __stcs(os + c.y, ordered_to_float(c.x));
+                }
+              }
             });
             for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += NTG) {
               __stcs(oi + s2, -1);
               if (os) __stcs(os + s2, -INFINITY);
             }
           } else {
-            select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch, st.sh, st.ctr, gtid, bar,
-                             [&](int s2, uint32_t key, int pos) {
-                               __stcs(oi + s2, pos);
-                               if (os) __stcs(os + s2, ordered_to_float(key));
-                             });
+            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+              __stcs(oi + s2, static_cast<int>(pos));
+              if (os) __stcs(os + s2, ordered_to_float(key));
+            });
           }
         } else {
           uint32_t* pk = p.part_keys + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
@@ -926,24 +1217,25 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
           if (n_valid <= kTopK) {
             if (gtid == 0) st.ctr[0] = 0;
             named_bar_sync(bar, NTG);
-            compact_view<NTG>(v, kSlots, st.ctr, gtid, [&](int rank, uint32_t key, int pos) {
-              pk[rank] = key;
-              pi[rank] = pos;
+            collect<NTG>(v, st.ctr, gtid, [&](int rank, uint2 x) {
+              pk[rank] = x.x;
+              pi[rank] = static_cast<int>(x.y);
             });
             for (int e = n_valid + gtid; e < kTopK; e += NTG) {
               pk[e] = 0u;
               pi[e] = -1;
             }
           } else {
-            select_topk<NTG>(v, kSlots, st.skeys, st.hist, st.list, kRankList, st.scratch, st.sh, st.ctr, gtid, bar,
-                             [&](int s2, uint32_t key, int pos) {
-                               pk[s2] = key;
-                               pi[s2] = pos;
-                             });
+            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+              pk[s2] = key;
+              pi[s2] = static_cast<int>(pos);
+            });
           }
         }
         named_bar_sync(bar, NTG);
       }
+      // empty histograms for the next item
+      for (int i = gtid; i < QPW * (kBins1 / 2); i += NTG) (&st.hist[0][0])[i] = 0u;
     }
   }
   tc_fence_before();
@@ -953,6 +1245,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     tmem_dealloc(tmem, C::kTmemCols);
   }
 }
+
 
 // ------------------------------------------------------------------------------------------
 // merge of the split-key path: top-k over the kMaxChunks partial lists of one query
@@ -1235,8 +1528,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.cache_offsets = a.cache_offsets;
   sp.idx_out = a.idx_out;
   sp.score_out = a.score_out;
-  sp.cand_keys = ws.cand_keys;
-  sp.cand_idx = ws.cand_idx;
+  sp.cand = ws.cand;
   sp.part_keys = ws.part_keys;
   sp.part_idx = ws.part_idx;
   sp.err = ws.err;

@@ -162,7 +162,7 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
  * dsa_indexer_topk (same arguments without handle and flags; same output rules;
  * the prefill path of dsa_indexer_topk with DSA_TOPK_NO_SPLIT).
  * Limits: T <= 4096 and B <= 4096 (otherwise DSA_ERR_WORKSPACE); the kernels run
- * on at most 12 SMs (the scratch holds 12 per-SM candidate areas), so this is
+ * on at most 8 SMs (the scratch holds 8 per-SM candidate areas), so this is
  * slower than dsa_indexer_topk.  Device-side problems are not reported through
  * a status word (there is no handle): affected rows are padded as documented
  * for dsa_indexer_topk.
