@@ -430,8 +430,10 @@ __device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
   atomicAdd(&h[bin >> 1], (bin & 1u) ? 0x10000u : 1u);
 }
 
-// Entry e (0..7) of a round: entries 2i and 2i+1 sit in x[i].
-__device__ __forceinline__ uint2 round_entry(const uint4 (&x)[4], int e) {
+constexpr int kRoundU = 4;   // 16-byte loads (two candidates each) per thread and round
+
+// Entry e (0..2 kRoundU - 1) of a round: entries 2i and 2i+1 sit in x[i].
+__device__ __forceinline__ uint2 round_entry(const uint4 (&x)[kRoundU], int e) {
   return (e & 1) ? make_uint2(x[e >> 1].z, x[e >> 1].w) : make_uint2(x[e >> 1].x, x[e >> 1].y);
 }
 
@@ -441,10 +443,10 @@ struct CandView {
   int nk, n0, n1, n2, n3;
   __device__ __forceinline__ int total() const { return nk + n0 + n1 + n2 + n3; }
 
-  // Calls f(x, lim) once per round.  A round gives each thread up to eight candidates,
-  // read in pairs with 16-byte loads: x[i] holds entries 2i and 2i+1, lim[i] how many of
-  // the two are valid.  Every thread of the group makes the same calls, so f may use
-  // warp-collective operations.
+  // Calls f(x, lim) once per round.  A round gives each thread up to 2 kRoundU candidates,
+  // all requested before any is used, read in pairs with 16-byte loads: x[i] holds entries
+  // 2i and 2i+1, lim[i] how many of the two are valid.  Every thread of the group makes
+  // the same calls, so f may use warp-collective operations.
   template <int NT, class F>
   __device__ __forceinline__ void for_rounds(int tid, F&& f) const {
     const int u0 = (nk + 1) >> 1;
@@ -453,11 +455,11 @@ struct CandView {
     const int u3 = u2 + ((n2 + 1) >> 1);
     const int u4 = u3 + ((n3 + 1) >> 1);
 #pragma unroll 1
-    for (int base = 0; base < u4; base += 4 * NT) {
-      uint4 x[4];
-      int lim[4];
+    for (int base = 0; base < u4; base += kRoundU * NT) {
+      uint4 x[kRoundU];
+      int lim[kRoundU];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kRoundU; ++i) {
         const int u = base + i * NT + tid;
         const uint2* p;
         int off, cnt;
@@ -480,23 +482,24 @@ template <int NT, class F>
 __device__ __forceinline__ void collect(const CandView& v, int* ctr, int tid, F&& f) {
   const int lane = tid & 31;
   const uint32_t lt = lanemask_lt();
-  v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
-    uint32_t b[8];
-    int tot = 0;
+  v.for_rounds<NT>(tid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
+    int c = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      b[e] = __ballot_sync(0xffffffffu, lim[e >> 1] > (e & 1));
-      tot += __popc(b[e]);
+    for (int i = 0; i < kRoundU; ++i) c += lim[i] > 0 ? lim[i] : 0;
+    int sc = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, sc, off);
+      if (lane >= off) sc += y;
     }
+    const int tot = __shfl_sync(0xffffffffu, sc, 31);
     if (tot) {
       int o = 0;
       if (lane == 0) o = atomicAdd(ctr, tot);
-      o = __shfl_sync(0xffffffffu, o, 0);
+      o = __shfl_sync(0xffffffffu, o, 0) + sc - c;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if ((b[e] >> lane) & 1u) f(o + __popc(b[e] & lt), round_entry(x, e));
-        o += __popc(b[e]);
-      }
+      for (int e = 0; e < 2 * kRoundU; ++e)
+        if (lim[e >> 1] > (e & 1)) f(o++, round_entry(x, e));
     }
   });
 }
@@ -619,40 +622,49 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
   const int b1 = locate_packed<NT>(h1, kTopK, clear_h1, rs.scratch, rs.sh, tid, bar, &above);
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   // 2.
-  v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
-    uint32_t bu[8], ba[8];
-    int tu = 0, ta = 0;
+  v.for_rounds<NT>(tid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
+    // each thread counts its own entries of each class; a warp scan of the counts and one
+    // shared counter per class give every entry its slot
+    int cu = 0, ca = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < 2 * kRoundU; ++e) {
       const uint32_t b = round_entry(x, e).x >> kBinShift;
       const bool ok = lim[e >> 1] > (e & 1);
-      bu[e] = __ballot_sync(0xffffffffu, ok && b > ub1);
-      ba[e] = __ballot_sync(0xffffffffu, ok && b == ub1);
-      tu += __popc(bu[e]);
-      ta += __popc(ba[e]);
+      cu += (ok && b > ub1) ? 1 : 0;
+      ca += (ok && b == ub1) ? 1 : 0;
     }
+    int su = cu, sa = ca;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int yu = __shfl_up_sync(0xffffffffu, su, off), ya = __shfl_up_sync(0xffffffffu, sa, off);
+      if (lane >= off) {
+        su += yu;
+        sa += ya;
+      }
+    }
+    const int tu = __shfl_sync(0xffffffffu, su, 31), ta = __shfl_sync(0xffffffffu, sa, 31);
     if (tu | ta) {
       int ou = 0, oa = 0;
       if (lane == 0) {
         if (tu) ou = atomicAdd(&rs.ctr[0], tu);
         if (ta) oa = atomicAdd(&rs.ctr[1], ta);
       }
-      ou = __shfl_sync(0xffffffffu, ou, 0);
-      oa = __shfl_sync(0xffffffffu, oa, 0);
+      ou = __shfl_sync(0xffffffffu, ou, 0) + su - cu;
+      oa = __shfl_sync(0xffffffffu, oa, 0) + sa - ca;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < 2 * kRoundU; ++e) {
         const uint2 c = round_entry(x, e);
-        if ((bu[e] >> lane) & 1u) {
-          const int o = ou + __popc(bu[e] & lt);
-          if (o < kTopK) sink(o, c.x, c.y);
+        const uint32_t b = c.x >> kBinShift;
+        if (lim[e >> 1] > (e & 1)) {
+          if (b > ub1) {
+            if (ou < kTopK) sink(ou, c.x, c.y);
+            ++ou;
+          } else if (b == ub1) {
+            if (oa < kListCap) rs.list[oa] = c;
+            count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
+            ++oa;
+          }
         }
-        if ((ba[e] >> lane) & 1u) {
-          const int o = oa + __popc(ba[e] & lt);
-          if (o < kListCap) rs.list[o] = c;
-          count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
-        }
-        ou += __popc(bu[e]);
-        oa += __popc(ba[e]);
       }
     }
   });
@@ -702,9 +714,9 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
     kth = kth_window<NT>(keys, need3, lo, hi, rs.rh, rs.scratch, rs.sh, tid, bar, &n3);
   } else {
     auto keys = [&](auto f) {
-      v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+      v.for_rounds<NT>(tid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < 2 * kRoundU; ++e)
           if (lim[e >> 1] > (e & 1)) f(round_entry(x, e).x);
       });
     };
@@ -736,9 +748,9 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
       fin(ok ? rs.list[e] : make_uint2(0u, 0u), ok);
     }
   } else {
-    v.for_rounds<NT>(tid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+    v.for_rounds<NT>(tid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) fin(round_entry(x, e), lim[e >> 1] > (e & 1));
+      for (int e = 0; e < 2 * kRoundU; ++e) fin(round_entry(x, e), lim[e >> 1] > (e & 1));
     });
   }
   return kth;
@@ -756,6 +768,7 @@ struct WGState {
   int cnt_k[QPW];                  // entries in the current keep set
   int kcur[QPW];                   // which keep set is current
   uint32_t thr[QPW];               // exact admission threshold left by a compaction
+  uint32_t thr_bin[QPW];           // admission threshold found by the query's scanning warp
   int pos[QPW];
   uint32_t scratch[64];
   int sh[8];
@@ -799,19 +812,27 @@ struct ScoreCfg {
   static_assert(kCtrlRegs % 8 == 0 && kEpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
 };
 
-// one query's score for this thread's key: sum_h w_h * max(v_h, 0), packed pairs
-__device__ __forceinline__ float head_weighted_relu(const uint32_t (&v)[32], const float* w) {
-  const float4* w4 = reinterpret_cast<const float4*>(w);
-  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
+// The four threads t, t^1, t^2, t^3 hold partial sums over disjoint head sets for the same
+// 2 x 2 rows (lane half h = 0/1, row t/4 or t/4 + 8) of each of QPH queries.  Two butterfly
+// steps, each sending half of the remaining values to the partner, leave every thread
+// with the full sums of one row for each query: the row of lane half (t & 1), offset
+// 8 ((t >> 1) & 1).
+template <int QPH>
+__device__ __forceinline__ void sum_over_quad(const float (&part)[4 * QPH], float (&s)[QPH], int lane) {
+  const bool b0 = lane & 1, b1 = (lane >> 1) & 1;
+  float q[2 * QPH];
 #pragma unroll
-  for (int h4 = 0; h4 < 8; ++h4) {
-    const float4 ww = w4[h4];
-    const float2 r0 = make_float2(fmaxf(__uint_as_float(v[4 * h4 + 0]), 0.f), fmaxf(__uint_as_float(v[4 * h4 + 1]), 0.f));
-    const float2 r1 = make_float2(fmaxf(__uint_as_float(v[4 * h4 + 2]), 0.f), fmaxf(__uint_as_float(v[4 * h4 + 3]), 0.f));
-    a0 = ffma2(make_float2(ww.x, ww.y), r0, a0);
-    a1 = ffma2(make_float2(ww.z, ww.w), r1, a1);
+  for (int i = 0; i < 2 * QPH; ++i) {
+    const float send = b0 ? part[i] : part[2 * QPH + i];
+    const float keep = b0 ? part[2 * QPH + i] : part[i];
+    q[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
   }
-  return (a0.x + a0.y) + (a1.x + a1.y);
+#pragma unroll
+  for (int i = 0; i < QPH; ++i) {
+    const float send = b1 ? q[i] : q[QPH + i];
+    const float keep = b1 ? q[QPH + i] : q[i];
+    s[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  }
 }
 
 template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
@@ -950,16 +971,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
             break;
           }
           tc_fence_after();
-          const uint32_t d = tmem + ab * C::kAccCols;
-          const uint32_t ka = smem_u32(sK + s * C::kKStage);
-#pragma unroll
-          for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(d, umma_desc_sw128(ka + kb * C::kKHalf + kk * 32),
-                        umma_desc_sw128(qa + kb * C::kQHalf + kk * 32), idesc, (kb | kk) != 0);
-          umma_commit(&empty[s]);
-          umma_commit(&acc_full[ab]);
+          umma_tile_k128<C::kKHalf, C::kQHalf>(tmem + ab * C::kAccCols, smem_u32(sK + s * C::kKStage), qa, idesc,
+                                              &empty[s], &acc_full[ab]);
         }
         umma_commit(q_empty);
         if (!ok) break;
@@ -979,7 +992,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     const int qd = warp & 3;                 // TMEM lane quadrant of this warp (also its append area)
     const int gtid = threadIdx.x - C::kEpiWarp0 * 32 - g * NTG;
     const int bar = 1 + g;
-    const int r = qd * 32 + lane;            // key row of this thread inside a tile
+    // key row of this thread inside a tile (the row whose scores it holds after sum_over_quad)
+    const int r = qd * 32 + (lane >> 2) + 8 * ((lane >> 1) & 1) + 16 * (lane & 1);
     const uint32_t lt = lanemask_lt();
     WGState<QPW>& st = *reinterpret_cast<WGState<QPW>*>(smem + C::kWGOff + g * C::kWGBytes);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
@@ -988,6 +1002,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     uint2* const qcand = p.cand + (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW) * kCandStride;
     uint2* const my_area = qcand + static_cast<size_t>(j0) * kCandStride + 2 * kTopK + qd * kWarpApp;
     const ResolveSmem rs{st.rhist, st.list, st.small, st.scratch, st.sh, st.ctr};
+    const uint64_t pol_cand = l2_policy_evict_last();   // candidates are read back at the item's end
     int acc_ctr = 0;
 
     // the candidates of query jj of this group, with the published counts
@@ -1020,6 +1035,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         st.cnt_k[gtid] = 0;
         st.kcur[gtid] = 0;
         st.thr[gtid] = 0u;
+        st.thr_bin[gtid] = 0u;
         st.pos[gtid] = (j < wi.nq) ? p.pos_eff[wi.t0 + j] : -2;
 #pragma unroll
         for (int w = 0; w < 4; ++w) st.cnt_w[gtid][w] = 0;
@@ -1045,6 +1061,13 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         thr_r[j] = 0u;
         pos_r[j] = (j < nmine) ? min(st.pos[j0 + j], wi.k_end - 1) : -2;   // last key position scored
       }
+      // this thread's head weights: heads 8 blk + 2 (lane % 4) + {0, 1} of each of its queries
+      float2 w2[QPH][4];
+#pragma unroll
+      for (int j = 0; j < QPH; ++j)
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk)
+          w2[j][blk] = *reinterpret_cast<const float2*>(&st.w[j0 + j][8 * blk + 2 * (lane & 3)]);
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
         const int ab = acc_ctr % ACC_BUFS;
@@ -1053,34 +1076,38 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         const int s_pos = kt * kKeyTile + r;
         const uint32_t tcol = tlane + ab * C::kAccCols + (g * QPW + j0) * kHeads;
         if (ok) {
-          float score[QPH];
-          if (nmine == QPH) {
-            // every column this warp needs, requested at once: one TMEM round trip per tile
-            uint32_t v[QPH][32];
-#pragma unroll
-            for (int j = 0; j < QPH; ++j) tmem_ld_32cols(tcol + j * kHeads, v[j]);
-#pragma unroll
-            for (int j = 0; j < QPH; ++j) tmem_ld_wait(v[j]);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
-#pragma unroll
-            for (int j = 0; j < QPH; ++j) score[j] = head_weighted_relu(v[j], st.w[j0 + j]);
+          // this warp's columns of the tile, as 16x256b blocks: one TMEM round trip per tile
+          uint32_t v[2 * QPH][16];   // [lane half h][query j] at h * QPH + j
+          constexpr uint32_t kHalf16 = 16u << 16;   // lane offset of the quadrant's upper half
+          if constexpr (QPH == 2) {
+            tmem_ld4_16x256b_x4_wait(tcol, tcol + kHeads, tcol + kHalf16, tcol + kHalf16 + kHeads, v);
           } else {
-            // a partial query tile: static indices keep score[] in registers
+            static_assert(QPH == 1, "one or two queries per epilogue warp");
+            tmem_ld2_16x256b_x4_wait(tcol, tcol + kHalf16, v);
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
+          // partial sums over this thread's 8 heads, for its two rows of each lane half
+          float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
-              if (j < nmine) {
-                uint32_t v[32];
-                tmem_ld_32cols(tcol + j * kHeads, v);
-                tmem_ld_wait(v);
-                score[j] = head_weighted_relu(v, st.w[j0 + j]);
+              const uint32_t(&x)[16] = v[h * QPH + j];
+              float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int blk = 0; blk < 4; ++blk) {
+                a = ffma2(w2[j][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
+                                                  fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
+                b = ffma2(w2[j][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
+                                                  fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
               }
+              part[(2 * h) * QPH + j] = a.x + a.y;
+              part[(2 * h + 1) * QPH + j] = b.x + b.y;
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          }
+          float score[QPH];
+          sum_over_quad<QPH>(part, score, lane);
           // admit (key, position) into this warp's area of each of its queries and count it;
           // the append counts stay warp-uniform in registers
 #pragma unroll
@@ -1090,8 +1117,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
             const bool pass = (s_pos <= pos_r[j]) && (u >= thr_r[j]);
             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
             if (pass) {
-              my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)] =
-                  make_uint2(u, static_cast<uint32_t>(s_pos));
+              st_global_u2_hint(&my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)],
+                                make_uint2(u, static_cast<uint32_t>(s_pos)), pol_cand);
               count_key(st.hist[j0 + j], u >> kBinShift);
             }
             cnt_r[j] += __popc(bal);
@@ -1162,13 +1189,23 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
               }
             }
           }
-          // raise each query's admission threshold to the lowest bin of its best kTopK (the
-          // counts need no barrier: a count read early only lowers the bin found)
+          // raise each query's admission threshold to the lowest bin of its best kTopK.  Query
+          // jl of the group is scanned by the warp of lane quadrant jl % 4 among those that score
+          // it, which publishes the bin; the others pick it up here, possibly one check point
+          // late.  Neither needs a barrier: a count read early only lowers the bin found, and
+          // the published thresholds only rise.
 #pragma unroll
           for (int j = 0; j < QPH; ++j) {
             if (j < nmine) {
-              const int b = scan_bins_warp(st.hist[j0 + j], kTopK, lane);
-              thr_r[j] = max(thr_r[j], static_cast<uint32_t>(b) << kBinShift);
+              const int jl = j0 + j;
+              if ((jl & 3) == qd) {
+                const uint32_t t = static_cast<uint32_t>(scan_bins_warp(st.hist[jl], kTopK, lane)) << kBinShift;
+                thr_r[j] = max(thr_r[j], t);
+                __syncwarp();
+                if (lane == 0) st.thr_bin[jl] = max(st.thr_bin[jl], t);
+              } else {
+                thr_r[j] = max(thr_r[j], st.thr_bin[jl]);
+              }
             }
           }
         }
@@ -1191,9 +1228,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
           const int prefix = st.pos[jj] + 1;   // keys this query scores (<= 0 if invalid)
           if (prefix <= kTopK) {
             // every position 0..prefix-1 is a candidate: place each at its own index
-            v.for_rounds<NTG>(gtid, [&](const uint4 (&x)[4], const int (&lim)[4]) {
+            v.for_rounds<NTG>(gtid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
+              for (int e = 0; e < 2 * kRoundU; ++e) {
                 const uint2 c = round_entry(x, e);
                 if (lim[e >> 1] > (e & 1) && c.y < static_cast<uint32_t>(kTopK)) {
                   __stcs(oi + c.y, static_cast<int>(c.y));
