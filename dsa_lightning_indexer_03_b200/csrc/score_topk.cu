@@ -432,8 +432,9 @@ __device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
 
 constexpr int kRoundU = 4;   // 16-byte loads (two candidates each) per thread and round
 
-// Entry e (0..2 kRoundU - 1) of a round: entries 2i and 2i+1 sit in x[i].
-__device__ __forceinline__ uint2 round_entry(const uint4 (&x)[kRoundU], int e) {
+// Entry e (0..2 U - 1) of a round: entries 2i and 2i+1 sit in x[i].
+template <int U>
+__device__ __forceinline__ uint2 round_entry(const uint4 (&x)[U], int e) {
   return (e & 1) ? make_uint2(x[e >> 1].z, x[e >> 1].w) : make_uint2(x[e >> 1].x, x[e >> 1].y);
 }
 
@@ -447,7 +448,7 @@ struct CandView {
   // all requested before any is used, read in pairs with 16-byte loads: x[i] holds entries
   // 2i and 2i+1, lim[i] how many of the two are valid.  Every thread of the group makes
   // the same calls, so f may use warp-collective operations.
-  template <int NT, class F>
+  template <int NT, int U = kRoundU, class F>
   __device__ __forceinline__ void for_rounds(int tid, F&& f) const {
     const int u0 = (nk + 1) >> 1;
     const int u1 = u0 + ((n0 + 1) >> 1);
@@ -455,11 +456,11 @@ struct CandView {
     const int u3 = u2 + ((n2 + 1) >> 1);
     const int u4 = u3 + ((n3 + 1) >> 1);
 #pragma unroll 1
-    for (int base = 0; base < u4; base += kRoundU * NT) {
-      uint4 x[kRoundU];
-      int lim[kRoundU];
+    for (int base = 0; base < u4; base += U * NT) {
+      uint4 x[U];
+      int lim[U];
 #pragma unroll
-      for (int i = 0; i < kRoundU; ++i) {
+      for (int i = 0; i < U; ++i) {
         const int u = base + i * NT + tid;
         const uint2* p;
         int off, cnt;
@@ -526,6 +527,10 @@ __device__ int locate_packed(uint32_t* hw, uint32_t need, bool clear, uint32_t* 
 #pragma unroll
     for (int i = 0; i < kWPT; ++i) hw[w0 + i] = 0u;
   }
+  if (tid == 0) {   // defaults in case no bin qualifies (the barrier below orders them first)
+    sh[0] = 0;
+    sh[1] = 0;
+  }
   const uint32_t above_t = group_suffix_excl<NT>(s, tid, scratch, bar);
   if (above_t < need && need <= above_t + s) {
     uint32_t cum = above_t;
@@ -540,8 +545,8 @@ __device__ int locate_packed(uint32_t* hw, uint32_t need, bool clear, uint32_t* 
     }
   }
   named_bar_sync(bar, NT);
-  const int b = sh[0];
-  *above = static_cast<uint32_t>(sh[1]);
+  const int b = min(max(sh[0], 0), kBins1 - 1);
+  *above = static_cast<uint32_t>(max(sh[1], 0));
   return b;
 }
 
@@ -622,12 +627,13 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
   const int b1 = locate_packed<NT>(h1, kTopK, clear_h1, rs.scratch, rs.sh, tid, bar, &above);
   const uint32_t ub1 = static_cast<uint32_t>(b1);
   // 2.
-  v.for_rounds<NT>(tid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
+  constexpr int kPassU = kRoundU;
+  v.for_rounds<NT, kPassU>(tid, [&](const uint4 (&x)[kPassU], const int (&lim)[kPassU]) {
     // each thread counts its own entries of each class; a warp scan of the counts and one
     // shared counter per class give every entry its slot
     int cu = 0, ca = 0;
 #pragma unroll
-    for (int e = 0; e < 2 * kRoundU; ++e) {
+    for (int e = 0; e < 2 * kPassU; ++e) {
       const uint32_t b = round_entry(x, e).x >> kBinShift;
       const bool ok = lim[e >> 1] > (e & 1);
       cu += (ok && b > ub1) ? 1 : 0;
@@ -652,19 +658,18 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
       ou = __shfl_sync(0xffffffffu, ou, 0) + su - cu;
       oa = __shfl_sync(0xffffffffu, oa, 0) + sa - ca;
 #pragma unroll
-      for (int e = 0; e < 2 * kRoundU; ++e) {
+      for (int e = 0; e < 2 * kPassU; ++e) {
         const uint2 c = round_entry(x, e);
         const uint32_t b = c.x >> kBinShift;
-        if (lim[e >> 1] > (e & 1)) {
-          if (b > ub1) {
-            if (ou < kTopK) sink(ou, c.x, c.y);
-            ++ou;
-          } else if (b == ub1) {
-            if (oa < kListCap) rs.list[oa] = c;
-            count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
-            ++oa;
-          }
+        const bool ok = lim[e >> 1] > (e & 1);
+        const bool up = ok && b > ub1, at = ok && b == ub1;
+        if (up && ou < kTopK) sink(ou, c.x, c.y);
+        if (at) {
+          if (oa < kListCap) rs.list[oa] = c;
+          count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
         }
+        ou += up ? 1 : 0;
+        oa += at ? 1 : 0;
       }
     }
   });
@@ -683,6 +688,10 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
   uint32_t kth;
   if (in_list && m2 <= kSmallRank) {
     // gather the sub-bin's keys; one warp ranks them
+    if (tid == 0) {   // defaults in case no key qualifies (ordered first by the barrier below)
+      rs.sh[4] = static_cast<int>(lo);
+      rs.sh[5] = 0;
+    }
     for (int e = tid; e < m; e += NT) {
       const uint32_t key = rs.list[e].x;
       if (key - lo <= hi - lo) {
@@ -706,7 +715,7 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
     }
     named_bar_sync(bar, NT);
     kth = static_cast<uint32_t>(rs.sh[4]);
-    n3 = rs.sh[5];
+    n3 = min(max(rs.sh[5], 0), kTopK);
   } else if (in_list) {
     auto keys = [&](auto f) {
       for (int e = tid; e < m; e += NT) f(rs.list[e].x);
@@ -722,7 +731,7 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
     };
     kth = kth_window<NT>(keys, need3, lo, hi, rs.rh, rs.scratch, rs.sh, tid, bar, &n3);
   }
-  const int n_above = static_cast<int>(above + above2) + n3;
+  const int n_above = min(static_cast<int>(min(above + above2, static_cast<uint32_t>(kTopK))) + n3, kTopK);
   const int ties = kTopK - n_above;
   // 4. slots below n_above continue rs.ctr[0] (== above after step 2); ties count in ctr[2]
   auto fin = [&](uint2 c, bool ok) {

@@ -15,6 +15,7 @@ from .indexer_oracle import (  # noqa: F401
     layer_norm,
     key_norm,
     project,
+    project_keys,
     index_scores,
     select_topk,
     sequence_of,

@@ -124,6 +124,11 @@ def key_norm(raw_keys, gamma, beta, eps: float = LN_EPS) -> np.ndarray:
     return bf16_round(layer_norm(raw_keys, gamma, beta, eps))
 
 
+def project_keys(hidden, W_k, gamma, beta, eps: float = LN_EPS) -> np.ndarray:
+    """The key path of `project` alone: k = bf16(LayerNorm(hidden @ W_k)) in float64."""
+    return key_norm(np.asarray(hidden, np.float64) @ np.asarray(W_k, np.float64), gamma, beta, eps)
+
+
 def project(hidden, q_latent, W_q, W_k, W_w, gamma, beta, eps: float = LN_EPS,
             n_heads: int = 32, head_dim: int = 128):
     """Indexer projections of T tokens.
@@ -141,7 +146,7 @@ def project(hidden, q_latent, W_q, W_k, W_w, gamma, beta, eps: float = LN_EPS,
             raise ValueError(f"{name} has shape {np.shape(arr)}, expected {shapes[name]}")
     T = hidden.shape[0]
     q = bf16_round(q_latent @ np.asarray(W_q, np.float64)).reshape(T, n_heads, head_dim)
-    k = bf16_round(layer_norm(hidden @ np.asarray(W_k, np.float64), gamma, beta, eps))
+    k = project_keys(hidden, W_k, gamma, beta, eps)
     w = (hidden @ np.asarray(W_w, np.float64)).astype(np.float32).astype(np.float64)
     return q, k, w
 
