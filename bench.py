@@ -18,6 +18,7 @@ scaling, no collective on the data path); times are the max over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
@@ -70,10 +71,25 @@ def _profile_traffic(kernel_key: str):
     return None
 
 
-class ClockSampler:
-    """nvidia-smi clock/throttle samples every 200 ms while running."""
+def max_over_ranks(x, dist, device):
+    """Max of a per-rank scalar over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units of all ranks per second, given the slowest rank's time for its units."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running; summary() keeps the
+    samples taken between mark_start() and mark_end()."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -81,6 +97,14 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.path = None
+        self.t0 = None
+        self.t1 = None
+
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
 
     def __enter__(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
@@ -105,24 +129,27 @@ class ClockSampler:
     def summary(self):
         if not self.path or not os.path.exists(self.path):
             return None
-        sm, mx, reasons = [], 0.0, set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = max(mx, float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(f[2]), float(f[3]),
+                             {n for n, v in zip(names, f[6:10]) if v.lower().startswith("active")}))
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
         os.unlink(self.path)
-        if not sm:
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        pad = datetime.timedelta(milliseconds=100)
+        inside = [r for r in rows if self.t0 is not None and self.t1 is not None and self.t0 - pad <= r[0] <= self.t1 + pad]
+        use = inside or rows
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(set().union(*(r[3] for r in use))), "samples": len(use),
+                "in_timed_region": bool(inside)}
 
 
 def _flush_l2(buf):
@@ -265,12 +292,8 @@ def gpu_arm(args, rank, world, local_rank, dist):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def mx(x):
+        return max_over_ranks(x, dist, device)
 
     # ---------------- prefill (headline)
     st = _setup_prefill(d, args.workload, rank, device)
@@ -278,17 +301,19 @@ def gpu_arm(args, rank, world, local_rank, dist):
     _time_steps(fn, args.warmup, flush)
     barrier()
     with ClockSampler(device.index) as clk:
+        clk.mark_start()
         step_ms, topk_ms = _time_steps(fn, args.steps, flush)
+        clk.mark_end()
     barrier()
     clocks = clk.summary()
-    ms = max_over_ranks(statistics.mean(step_ms))
-    topk_avg = max_over_ranks(statistics.mean(topk_ms))
+    ms = mx(statistics.mean(step_ms))
+    topk_avg = mx(statistics.mean(topk_ms))
     pairs = st["pairs"]
-    value = pairs * world / (ms * 1e-3) / 1e9
+    value = whole_job_rate(pairs, world, ms) / 1e9
     achieved_tflops = pairs * FLOP_PER_PAIR / (topk_avg * 1e-3) / 1e12
     traffic = _profile_traffic(f"score_topk:{args.workload}")
     e2e_ms, bi, bo = _e2e_prefill(st, max(2, min(args.steps, 5)))
-    e2e_ms = max_over_ranks(e2e_ms)
+    e2e_ms = mx(e2e_ms)
     st["ix"].device_error()
 
     # ---------------- decode (second half of the metric)
@@ -313,8 +338,8 @@ def gpu_arm(args, rank, world, local_rank, dist):
         barrier()
         dstep, dtopk = _time_steps(dfn, args.steps, flush)
         barrier()
-        dms = max_over_ranks(statistics.mean(dtopk))
-        dstep_ms = max_over_ranks(statistics.mean(dstep))
+        dms = mx(statistics.mean(dtopk))
+        dstep_ms = mx(statistics.mean(dstep))
         gbs = ds["bytes"] / (dms * 1e-3) / 1e9
         dec = {"workload": "decode_64", "metric": "decode GB/s", "value": round(gbs * world, 2), "unit": "GB/s",
                "ms_score_topk": round(dms, 4), "ms_per_step": round(dstep_ms, 4),
@@ -345,7 +370,7 @@ def gpu_arm(args, rank, world, local_rank, dist):
                      "unit": "TFLOP/s", "frac": round(achieved_tflops / peaks["bf16_tflops"], 4),
                      "traffic": traffic, "kernel": "score_topk (dsa_indexer_topk: prep + score)",
                      "ms_per_launch": round(topk_avg, 4), "peak_source": peaks["source"] + " burst bf16"},
-        "e2e": {"value": round(pairs * world / (e2e_ms * 1e-3) / 1e9, 3), "unit": "Gpairs/s",
+        "e2e": {"value": round(whole_job_rate(pairs, world, e2e_ms) / 1e9, 3), "unit": "Gpairs/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
         "clocks": clocks,
         "gpu_launches": args.steps * 4,
@@ -439,7 +464,7 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill_8k", choices=["prefill_3k", "prefill_8k", "prefill_2x32k_heavy"])
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])

@@ -629,47 +629,37 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
   // 2.
   constexpr int kPassU = kRoundU;
   v.for_rounds<NT, kPassU>(tid, [&](const uint4 (&x)[kPassU], const int (&lim)[kPassU]) {
-    // each thread counts its own entries of each class; a warp scan of the counts and one
-    // shared counter per class give every entry its slot
-    int cu = 0, ca = 0;
+    // above-b1 entries: one ballot per entry position and one shared counter update per warp
+    // and round, so that each store instruction writes warp-contiguous slots; the few entries
+    // of the boundary bin take a slot each from their own counter
+    uint32_t bu[2 * kPassU];
+    int tu = 0, ca = 0;
 #pragma unroll
     for (int e = 0; e < 2 * kPassU; ++e) {
       const uint32_t b = round_entry(x, e).x >> kBinShift;
       const bool ok = lim[e >> 1] > (e & 1);
-      cu += (ok && b > ub1) ? 1 : 0;
+      bu[e] = __ballot_sync(0xffffffffu, ok && b > ub1);
+      tu += __popc(bu[e]);
       ca += (ok && b == ub1) ? 1 : 0;
     }
-    int su = cu, sa = ca;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int yu = __shfl_up_sync(0xffffffffu, su, off), ya = __shfl_up_sync(0xffffffffu, sa, off);
-      if (lane >= off) {
-        su += yu;
-        sa += ya;
-      }
+    int ou = 0;
+    if (tu) {
+      if (lane == 0) ou = atomicAdd(&rs.ctr[0], tu);
+      ou = __shfl_sync(0xffffffffu, ou, 0);
     }
-    const int tu = __shfl_sync(0xffffffffu, su, 31), ta = __shfl_sync(0xffffffffu, sa, 31);
-    if (tu | ta) {
-      int ou = 0, oa = 0;
-      if (lane == 0) {
-        if (tu) ou = atomicAdd(&rs.ctr[0], tu);
-        if (ta) oa = atomicAdd(&rs.ctr[1], ta);
-      }
-      ou = __shfl_sync(0xffffffffu, ou, 0) + su - cu;
-      oa = __shfl_sync(0xffffffffu, oa, 0) + sa - ca;
+    int oa = ca ? atomicAdd(&rs.ctr[1], ca) : 0;
 #pragma unroll
-      for (int e = 0; e < 2 * kPassU; ++e) {
-        const uint2 c = round_entry(x, e);
-        const uint32_t b = c.x >> kBinShift;
-        const bool ok = lim[e >> 1] > (e & 1);
-        const bool up = ok && b > ub1, at = ok && b == ub1;
-        if (up && ou < kTopK) sink(ou, c.x, c.y);
-        if (at) {
-          if (oa < kListCap) rs.list[oa] = c;
-          count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
-        }
-        ou += up ? 1 : 0;
-        oa += at ? 1 : 0;
+    for (int e = 0; e < 2 * kPassU; ++e) {
+      const uint2 c = round_entry(x, e);
+      if ((bu[e] >> lane) & 1u) {
+        const int o = ou + __popc(bu[e] & lt);
+        if (o < kTopK) sink(o, c.x, c.y);
+      }
+      ou += __popc(bu[e]);
+      if (lim[e >> 1] > (e & 1) && (c.x >> kBinShift) == ub1) {
+        if (oa < kListCap) rs.list[oa] = c;
+        count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
+        ++oa;
       }
     }
   });
