@@ -891,6 +891,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above overlaps the prep kernel; its work list is read only after it completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int n_items = *p.n_items;
   const WaitCtl wc{p.err, abort_flag, p.timeout_ns};
 
@@ -1386,11 +1388,32 @@ __device__ __forceinline__ int chunk_len_for(int n, int target) {
   return c < kKeyTile ? kKeyTile : c;
 }
 
+// Sequence of query token t: the last b with q_seq_offsets[b] <= t.
+__device__ __forceinline__ int sequence_of_token(const int32_t* qoff, int B, int t) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (qoff[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+constexpr int kPrepCopy = 4096;   // offset arrays up to this length are searched in shared memory
+
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __shared__ int warp_sums[32];
   __shared__ int bad;
   __shared__ unsigned long long total_keys;
+  __shared__ int s_qoff[kPrepCopy + 1];   // copy of q_seq_offsets when B < kPrepCopy
+  __shared__ int s_base[kPrepCopy + 1];   // copy of the items' owner bases when n_owners < kPrepCopy
   const TopkWorkspace& ws = p.ws;
+  // the score kernel may start its prologue now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const bool qoff_in_smem = p.B < kPrepCopy;
+  if (qoff_in_smem)
+    for (int b = threadIdx.x; b <= p.B; b += kPrepThreads) s_qoff[b] = p.q_seq_offsets[b];
+  const int32_t* qoff = qoff_in_smem ? s_qoff : p.q_seq_offsets;
   if (threadIdx.x == 0) {
     bad = 0;
     total_keys = 0;
@@ -1418,12 +1441,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   }
   // 2. validated positions
   for (int t = threadIdx.x; t < p.T; t += kPrepThreads) {
-    int lo = 0, hi = p.B - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (p.q_seq_offsets[mid] <= t) lo = mid;
-      else hi = mid - 1;
-    }
+    const int lo = sequence_of_token(qoff, p.B, t);
     const int64_t len = p.cache_offsets[lo + 1] - p.cache_offsets[lo];
     const int pos = p.positions[t];
     const bool ok = pos >= 0 && pos < len;
@@ -1433,12 +1451,15 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     if (p.split && ok) atomicAdd(&total_keys, static_cast<unsigned long long>(pos) + 1ull);
   }
   __syncthreads();
-  // split path: chunks sized so that about two chunks per SM cover all the keys
-  long long tgt = (static_cast<long long>(total_keys) + 2ll * p.num_sms - 1) / (2ll * p.num_sms);
+  // split path: chunks sized so that about four chunks per SM cover all the keys (more,
+  // shorter chunks balance the SMs better than fewer, longer ones; the merge reads at most
+  // kMaxChunks partial lists per query)
+  long long tgt = (static_cast<long long>(total_keys) + 4ll * p.num_sms - 1) / (4ll * p.num_sms);
   tgt = (tgt + kKeyTile - 1) / kKeyTile * kKeyTile;
   const int target = static_cast<int>(tgt < kMinChunk ? kMinChunk : (tgt > (1 << 30) ? (1 << 30) : tgt));
   // 3. items per owner (sequence on the prefill path, query on the split path)
   const int n_owners = p.split ? p.T : p.B;
+  int* const base = (n_owners < kPrepCopy) ? s_base : ws.seq_base;   // per-owner item counts, then bases
   for (int o = threadIdx.x; o < n_owners; o += kPrepThreads) {
     int c;
     if (p.split) {
@@ -1447,23 +1468,23 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       c = n > cl ? (n + cl - 1) / cl : 1;
       ws.tok_nchunks[o] = c;
     } else {
-      const int nq = p.q_seq_offsets[o + 1] - p.q_seq_offsets[o];
+      const int nq = qoff[o + 1] - qoff[o];
       c = (nq + kPrefillQ - 1) / kPrefillQ;
     }
-    ws.seq_base[o] = c;
+    base[o] = c;
   }
   __syncthreads();
-  const int total = block_exclusive_scan(ws.seq_base, n_owners, warp_sums);
+  const int total = block_exclusive_scan(base, n_owners, warp_sums);
   if (threadIdx.x == 0) {
-    ws.seq_base[n_owners] = total;
+    base[n_owners] = total;
     *ws.n_items = total;
     *ws.work_counter = 0;
   }
   __syncthreads();
   // 4. items, written in reverse order of (owner, tile) so the longest prefixes come first
   for (int i = threadIdx.x; i < total; i += kPrepThreads) {
-    const int o = owner_of(ws.seq_base, n_owners, i);
-    const int local = i - ws.seq_base[o];
+    const int o = owner_of(base, n_owners, i);
+    const int local = i - base[o];
     WorkItem wi;
     wi.pad0 = wi.pad1 = 0;
     if (p.split) {
@@ -1471,22 +1492,16 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       const int n = ws.pos_eff[t] + 1;
       const int nch = ws.tok_nchunks[t];
       const int cl = chunk_len_for(n, target);
-      int lo = 0, hi = p.B - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.q_seq_offsets[mid] <= t) lo = mid;
-        else hi = mid - 1;
-      }
       wi.t0 = t;
       wi.nq = 1;
-      wi.b = lo;
+      wi.b = sequence_of_token(qoff, p.B, t);
       wi.k_begin = (nch > 1) ? local * cl : 0;
       wi.k_end = (nch > 1) ? min(n, (local + 1) * cl) : n;
       wi.chunk = (nch > 1) ? local : -1;
     } else {
       const int b = o;
-      const int t0 = p.q_seq_offsets[b] + local * kPrefillQ;
-      const int nq = min(kPrefillQ, p.q_seq_offsets[b + 1] - t0);
+      const int t0 = qoff[b] + local * kPrefillQ;
+      const int nq = min(kPrefillQ, qoff[b + 1] - t0);
       int kend = 0;
       for (int j = 0; j < nq; ++j) kend = max(kend, ws.pos_eff[t0 + j] + 1);
       wi.t0 = t0;
@@ -1533,8 +1548,19 @@ cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const S
                             static_cast<long>(C::kEpiRegs) * NWG * C::kGroupThreads;
     if (split_regs > launch_regs) return cudaErrorInvalidConfiguration;
   }
-  kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tmQ, tmK, p);
-  return cudaGetLastError();
+  // launched as a programmatic dependent of the prep kernel (which lets it start at once):
+  // the prologue overlaps the prep kernel and griddepcontrol.wait orders the rest after it
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmQ, tmK, p);
 }
 
 }  // namespace
