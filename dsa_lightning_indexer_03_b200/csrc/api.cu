@@ -75,6 +75,10 @@ struct dsa_indexer {
   CUtensorMap tm_WqT, tm_WkwT;
   TopkWorkspace ws{};
   std::vector<void*> allocs;
+  // dsa_indexer_project runs the k|w GEMM (HBM-bound) on `side` next to the q GEMM
+  // (tensor-bound) on the caller's stream, forked and joined with the two events
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
 
   template <class T>
   bool alloc(T** p, size_t count) {
@@ -85,6 +89,9 @@ struct dsa_indexer {
     return true;
   }
   ~dsa_indexer() {
+    if (ev_fork) cudaEventDestroy(ev_fork);
+    if (ev_join) cudaEventDestroy(ev_join);
+    if (side) cudaStreamDestroy(side);
     for (void* p : allocs) cudaFree(p);
   }
 };
@@ -157,6 +164,12 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
   if (!ok) {
     delete h;
     return DSA_ERR_OOM;
+  }
+  if (cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    delete h;
+    return DSA_ERR_CUDA;
   }
   cudaStream_t s = nullptr;
   cudaError_t e = cudaMemset(ws.err, 0, sizeof(int));
@@ -233,10 +246,17 @@ dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden,
   e.eps = c.ln_eps;
   e.err = h->ws.err;
   e.timeout_ns = timeout_ns();
-  if (launch_proj_kw(tmX, h->tm_WkwT, c.hidden_dim, e, s) != cudaSuccess) return DSA_ERR_CUDA;
-  if (launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
-                    static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s) != cudaSuccess)
+  // k|w on the handle's side stream, q on the caller's; both ordered after the caller's
+  // earlier work, and the caller's later work after both
+  if (cudaEventRecord(h->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(h->side, h->ev_fork, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
+  const cudaError_t ekw = launch_proj_kw(tmX, h->tm_WkwT, c.hidden_dim, e, h->side);
+  const cudaError_t eq = launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
+                                       static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s);
+  // join even if a launch failed, so that the side stream never runs ahead unordered
+  if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess || cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (ekw != cudaSuccess || eq != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }
 

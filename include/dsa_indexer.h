@@ -26,8 +26,10 @@
  *     cache, malformed offsets, a pipeline wait that ran out) set bits in the
  *     handle's device error word and leave the affected outputs in a defined
  *     padded state; dsa_indexer_device_error() reports and clears them.
- *   - A handle may be used from one stream at a time (its workspace is shared
- *     by consecutive calls and ordered by that stream).
+ *   - A handle may be used from one stream and one host thread at a time (its
+ *     workspace is shared by consecutive calls and ordered by that stream, and
+ *     dsa_indexer_project forks part of its work onto a stream the handle owns
+ *     and joins it back with two events the handle owns).
  */
 #ifndef DSA_INDEXER_H
 #define DSA_INDEXER_H
