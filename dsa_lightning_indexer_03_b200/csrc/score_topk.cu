@@ -778,10 +778,14 @@ struct WGState {
 // TMEM lane quadrant, each warp handles every query of the group) or 8 (two warps per
 // quadrant, each handles half of the group's queries).  With EW = 8 the two control
 // warps sit in a warpgroup of their own (warps 0-3) so that registers can be moved
-// from it to the epilogue warpgroups (setmaxnreg).
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
+// from it to the epilogue warpgroups (setmaxnreg).  NWG groups either split each item's
+// queries (ALT = false) or, with ALT, take whole items in turn (group g takes the items
+// the CTA receives at positions g, g + 2, ...): one group's end-of-item selection then
+// overlaps the other group's tiles.
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
 struct ScoreCfg {
-  static constexpr int kQPW = QMAX / NWG;             // queries of one epilogue group
+  static constexpr int kQPW = ALT ? QMAX : QMAX / NWG;  // queries of one epilogue group
+  static constexpr int kConsumers = ALT ? EW : NWG * EW; // warps that consume each tile
   static constexpr int kQPH = kQPW / (EW / 4);        // queries of one epilogue warp
   static constexpr int kEpiWarp0 = EW == 8 ? 4 : 2;   // first epilogue warp
   static constexpr int kGroupThreads = EW * 32;
@@ -790,7 +794,8 @@ struct ScoreCfg {
   static constexpr int kCtrlRegs = 32;                // per thread of warps 0-3 after the split
   static constexpr int kEpiRegs = 112;                // per epilogue thread after the split
   static constexpr int kAccCols = QMAX * kHeads;
-  static constexpr int kTmemNeed = ACC_BUFS * kAccCols;
+  static constexpr int kTotalBufs = ALT ? NWG * ACC_BUFS : ACC_BUFS;  // with ALT each group has its own
+  static constexpr int kTmemNeed = kTotalBufs * kAccCols;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kQHalf = QMAX * kHeads * 128;  // bytes of one 64-column half of the Q tile
@@ -801,7 +806,7 @@ struct ScoreCfg {
   static constexpr int kWGOff = kKOff + STAGES * kKStage;
   static constexpr int kWGBytes = (static_cast<int>(sizeof(WGState<kQPW>)) + 15) / 16 * 16;
   static constexpr int kBarOff = kWGOff + NWG * kWGBytes;
-  static constexpr int kNumBars = 2 * STAGES + 2 * ACC_BUFS + 2 + 4 + 1;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kTotalBufs + 2 + 4 + 1;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr int kSmemBytes = kMiscOff + 64 + 1024;
   static_assert(kTmemNeed <= 512, "TMEM holds 512 columns");
@@ -809,6 +814,7 @@ struct ScoreCfg {
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   static_assert(kQPH >= 1 && kQPH * (EW / 4) == kQPW, "queries split evenly over a quadrant's warps");
   static_assert(kCtrlRegs % 8 == 0 && kEpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
+  static_assert(!ALT || NWG == 2, "alternating items need two epilogue groups");
 };
 
 // The four threads t, t^1, t^2, t^3 hold partial sums over disjoint head sets for the same
@@ -834,11 +840,11 @@ __device__ __forceinline__ void sum_over_quad(const float (&part)[4 * QPH], floa
   }
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
-__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kThreads, 1)
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
+__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>::kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       ScoreParams p) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
   constexpr int QPW = C::kQPW;
   constexpr int QPH = C::kQPH;
   constexpr int NTG = C::kGroupThreads;
@@ -850,8 +856,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
   uint64_t* full = bars;
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
-  uint64_t* acc_empty = acc_full + ACC_BUFS;
-  uint64_t* q_full = acc_empty + ACC_BUFS;
+  uint64_t* acc_empty = acc_full + C::kTotalBufs;
+  uint64_t* q_full = acc_empty + C::kTotalBufs;
   uint64_t* q_empty = q_full + 1;
   uint64_t* sched_full = q_empty + 1;
   uint64_t* sched_empty = sched_full + 2;
@@ -867,15 +873,15 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < ACC_BUFS; ++a) {
+    for (int a = 0; a < C::kTotalBufs; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], NWG * EW);
+      mbar_init(&acc_empty[a], C::kConsumers);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sched_full[i], 1);
-      mbar_init(&sched_empty[i], 1 + NWG * EW);
+      mbar_init(&sched_empty[i], 1 + C::kConsumers);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -914,7 +920,16 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         if (it >= n_items) it = -1;
         sched_item[slot] = it;
         mbar_arrive(&sched_full[slot]);
-        if (it < 0) break;
+        if (it < 0) {
+          if constexpr (ALT) {
+            // the other group waits on the next slot: end it as well
+            const int l2 = local + 1, s2 = l2 & 1;
+            if (l2 >= 2 && !mbar_wait(&sched_empty[s2], ((l2 >> 1) - 1) & 1, wc)) break;
+            sched_item[s2] = -1;
+            mbar_arrive(&sched_full[s2]);
+          }
+          break;
+        }
         const WorkItem wi = p.items[it];
         const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
         if (kt1 <= kt0) continue;
@@ -947,7 +962,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
   } else if (warp == 1) {
     // ===================================================== MMA issuer
     if (lane == 0) {
-      int kstage = 0, acc_ctr = 0, qloads = 0;
+      int kstage = 0, qloads = 0;
+      int acc0 = 0, acc1 = 0;   // tiles given to group 0 / group 1 (one shared ring without ALT)
       const uint32_t qa = smem_u32(sQ);
       for (int local = 0;; ++local) {
         const int slot = local & 1;
@@ -962,10 +978,14 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
         ++qloads;
         tc_fence_after();
         const uint32_t idesc = umma_idesc_bf16(kKeyTile, wi.nq * kHeads);
+        const bool second = ALT && (local & 1);   // with ALT, the CTA's odd items go to group 1
         bool ok = true;
-        for (int kt = kt0; kt < kt1; ++kt, ++kstage, ++acc_ctr) {
+        for (int kt = kt0; kt < kt1; ++kt, ++kstage) {
           const int s = kstage % STAGES;
-          const int ab = acc_ctr % ACC_BUFS;
+          const int acc_ctr = second ? acc1 : acc0;
+          const int ab = (second ? ACC_BUFS : 0) + acc_ctr % ACC_BUFS;
+          if (second) ++acc1;
+          else ++acc0;
           if (!mbar_wait(&full[s], (kstage / STAGES) & 1, wc)) { ok = false; break; }
           if (acc_ctr >= ACC_BUFS && !mbar_wait(&acc_empty[ab], ((acc_ctr / ACC_BUFS) - 1) & 1, wc)) {
             ok = false;
@@ -1000,7 +1020,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const int j0 = hq * QPH;                 // first of this warp's queries inside the group
     // candidates of query jj of this group start at qcand + jj * kCandStride
-    uint2* const qcand = p.cand + (static_cast<size_t>(blockIdx.x) * QMAX + g * QPW) * kCandStride;
+    const int qbase = ALT ? 0 : g * QPW;    // first query of the item this group scores
+    uint2* const qcand =
+        p.cand + (static_cast<size_t>(blockIdx.x) * (ALT ? QMAX * NWG : QMAX) + g * QPW) * kCandStride;
     uint2* const my_area = qcand + static_cast<size_t>(j0) * kCandStride + 2 * kTopK + qd * kWarpApp;
     const ResolveSmem rs{st.rhist, st.list, st.small, st.scratch, st.sh, st.ctr};
     const uint64_t pol_cand = l2_policy_evict_last();   // candidates are read back at the item's end
@@ -1023,7 +1045,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
     // the histograms start empty (ordered before any count by the item barrier)
     for (int i = gtid; i < QPW * (kBins1 / 2); i += NTG) (&st.hist[0][0])[i] = 0u;
 
-    for (int local = 0;; ++local) {
+    for (int n = 0;; ++n) {
+      const int local = ALT ? 2 * n + g : n;
       const int slot = local & 1;
       const bool got = __all_sync(0xffffffffu, mbar_wait(&sched_full[slot], (local >> 1) & 1, wc));
       const int it = got ? sched_item[slot] : -1;
@@ -1032,7 +1055,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
       WorkItem wi;
       if (it >= 0) wi = p.items[it];
       if (gtid < QPW && it >= 0) {
-        const int j = g * QPW + gtid;
+        const int j = qbase + gtid;
         st.cnt_k[gtid] = 0;
         st.kcur[gtid] = 0;
         st.thr[gtid] = 0u;
@@ -1043,13 +1066,13 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
       }
       if (it >= 0) {
         for (int i = gtid; i < QPW * kHeads; i += NTG) {
-          const int jj = i / kHeads, j = g * QPW + jj;
+          const int jj = i / kHeads, j = qbase + jj;
           st.w[jj][i % kHeads] = (j < wi.nq) ? p.w[static_cast<size_t>(wi.t0 + j) * kHeads + (i % kHeads)] : 0.f;
         }
       }
       if (named_bar_or(bar, NTG, it < 0)) break;   // every thread of the group leaves together
 
-      const int nloc = min(QPW, wi.nq - g * QPW);  // queries of the group present in this item
+      const int nloc = min(QPW, wi.nq - qbase);    // queries of the group present in this item
       const int nmine = min(QPH, nloc - j0);        // ... and scored by this warp (may be <= 0)
       const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
       // an item of at most kWarpApp / 32 tiles cannot fill an append area: no capacity checks
@@ -1071,11 +1094,11 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
           w2[j][blk] = *reinterpret_cast<const float2*>(&st.w[j0 + j][8 * blk + 2 * (lane & 3)]);
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
-        const int ab = acc_ctr % ACC_BUFS;
+        const int ab = (ALT ? g * ACC_BUFS : 0) + acc_ctr % ACC_BUFS;   // this group's ring
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (acc_ctr / ACC_BUFS) & 1, wc));
         tc_fence_after();
         const int s_pos = kt * kKeyTile + r;
-        const uint32_t tcol = tlane + ab * C::kAccCols + (g * QPW + j0) * kHeads;
+        const uint32_t tcol = tlane + ab * C::kAccCols + (qbase + j0) * kHeads;
         if (ok) {
           // this warp's columns of the tile, as 16x256b blocks: one TMEM round trip per tile
           uint32_t v[2 * QPH][16];   // [lane half h][query j] at h * QPH + j
@@ -1220,7 +1243,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>::kTh
       if (named_bar_or(bar, NTG, failed)) break;   // a failed wait ends every warp of the group
 #pragma unroll 1
       for (int jj = 0; jj < nloc; ++jj) {
-        const int t = wi.t0 + g * QPW + jj;
+        const int t = wi.t0 + qbase + jj;
         const CandView v = cands(jj);
         const int n_valid = v.total();
         if (wi.chunk < 0) {
@@ -1530,11 +1553,11 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
   *status = ok ? 0 : ((err & kErrTimeout) ? 2 : 1);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
 cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const ScoreParams& p, int grid,
                          cudaStream_t s) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW>;
-  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
+  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (C::kRegSplit) {
@@ -1597,7 +1620,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
   if (a.split) {
-    e = launch_score<1, 5, 4, 1, 4>(tmQ1, tmK, sp, grid, s);
+    e = launch_score<1, 5, 4, 2, 4, true>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
     const int msmem = kMaxChunks * kTopK * 4;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
@@ -1606,7 +1629,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
                                                     a.score_out);
     return cudaGetLastError();
   }
-  return launch_score<kPrefillQ, 3, 2, 2, 8>(tmQ8, tmK, sp, grid, s);
+  return launch_score<kPrefillQ, 3, 2, 2, 8, false>(tmQ8, tmK, sp, grid, s);
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s) {
