@@ -309,32 +309,9 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 
-// 16 TMEM lanes x 32 columns as four 8-column blocks (tcgen05.ld 16x256b, x4).  Thread t
+// tcgen05.ld 16x256b, x4: 16 TMEM lanes x 32 columns as four 8-column blocks.  Thread t
 // receives, for block b, r[4b], r[4b+1] = (lane base + t/4, columns 8b + 2(t%4) + {0,1})
 // and r[4b+2], r[4b+3] = the same columns of lane base + t/4 + 8.
-__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
-}
-
-// tcgen05.wait::ld, with two 16-register load targets tied to it so that no use of them
-// moves above the wait.
-__device__ __forceinline__ void tmem_ld_wait16x2(uint32_t (&a)[16], uint32_t (&b)[16]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
-        "+r"(a[8]), "+r"(a[9]), "+r"(a[10]), "+r"(a[11]), "+r"(a[12]), "+r"(a[13]), "+r"(a[14]), "+r"(a[15]),
-        "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7]),
-        "+r"(b[8]), "+r"(b[9]), "+r"(b[10]), "+r"(b[11]), "+r"(b[12]), "+r"(b[13]), "+r"(b[14]), "+r"(b[15])
-      :
-      : "memory");
-}
-
 // Four 16x256b.x4 loads (lane bases a0..a3) and the wait for them in one statement: the 64
 // results are defined only after tcgen05.wait::ld.
 __device__ __forceinline__ void tmem_ld4_16x256b_x4_wait(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -85,25 +85,6 @@ __device__ __forceinline__ uint32_t group_suffix_excl(uint32_t v, int tid, uint3
   return wa + x - v;
 }
 
-// Group minimum of lo and maximum of hi.
-template <int NT>
-__device__ __forceinline__ void group_minmax(uint32_t& lo, uint32_t& hi, int tid, uint32_t* scratch, int bar) {
-  const int lane = tid & 31, wid = tid >> 5;
-  lo = __reduce_min_sync(0xffffffffu, lo);
-  hi = __reduce_max_sync(0xffffffffu, hi);
-  if (lane == 0) {
-    scratch[wid] = lo;
-    scratch[NT / 32 + wid] = hi;
-  }
-  named_bar_sync(bar, NT);
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    lo = min(lo, scratch[w]);
-    hi = max(hi, scratch[NT / 32 + w]);
-  }
-  named_bar_sync(bar, NT);
-}
-
 constexpr int kHistBins = 1024;   // histogram bins of one selection round
 constexpr int kRankList = 256;    // boundary-bin keys ranked directly (merge path)
 
