@@ -17,18 +17,20 @@
 //              K-major) once, then 128-key tiles of the key cache into a ring.
 //   warp 1     MMA issuer: D[key, (query, head)] = K_tile (M=128) x Q^T (N=nq*32),
 //              K=128 as 8 tcgen05.mma of K=16, into one of ACC_BUFS TMEM buffers.
-//   epilogue   warpgroups of 4 warps (the 4 TMEM lane quadrants).  Thread (quadrant,
-//              lane) owns one key of the tile; per query it loads that query's 32 head
-//              columns (tcgen05.ld 32x32b.x32), applies ReLU and the fp32 head weights
-//              in registers, masks s > pos, and admits (key, s) when the key reaches the
-//              query's admission threshold: the pair goes to the warp's own append area
-//              (warp ballot, warp-uniform counts in registers, no atomics) and the key is
-//              counted in the query's first-level histogram in shared memory.  Every
-//              kCheckTiles tiles the threshold rises to the lowest bin that still holds
-//              the query's best 2,048 counted keys (a warp scan of the histogram), and a
-//              nearly full append area is compacted to the exact best 2,048.  At the end
-//              of the item each query's candidates are reduced to exactly the top 2,048
-//              in one pass (resolve_topk) and written out.
+//   epilogue   warpgroups of 4 warps (the 4 TMEM lane quadrants); a warp covers its
+//              quadrant's 32 keys for one or two queries.  It reads its columns with
+//              tcgen05.ld 16x256b, in which each thread holds a fixed set of 8 heads, so
+//              the fp32 head weights stay in registers; ReLU and the weights give partial
+//              sums that two shuffle steps across 4 threads turn into one score per thread
+//              and query.  A key is masked if s > pos, and (key, s) is admitted when the
+//              key reaches the query's admission threshold: the pair goes to the warp's own
+//              append area (warp ballot, warp-uniform counts in registers, no atomics) and
+//              the key is counted in the query's first-level histogram in shared memory.
+//              Every kCheckTiles tiles the threshold rises to the lowest bin that still
+//              holds the query's best 2,048 counted keys (a warp scan of the histogram);
+//              in long items a nearly full append area is compacted to the exact best
+//              2,048.  At the end of the item each query's candidates are reduced to
+//              exactly the top 2,048 in one pass (resolve_topk) and written out.
 
 #include "kernels.h"
 
@@ -403,8 +405,9 @@ constexpr int kBinShift = 21;                  // first-level bin = key >> kBinS
 constexpr int kBins1 = 1 << (32 - kBinShift);  // 2,048 bins
 constexpr int kSubShift = kBinShift - 11;      // second-level bin = next 11 bits
 constexpr int kListCap = 1024;                 // boundary-bin candidates gathered in shared memory
-constexpr int kCheckTiles = 4;                 // key tiles between threshold updates / capacity checks
-constexpr int kCheckMargin = kCheckTiles * 32; // appends one warp can make per query in that time
+constexpr int kCheckTiles = 8;                 // key tiles between threshold updates
+constexpr int kCapTiles = 16;                  // key tiles between capacity checks (long items)
+constexpr int kCheckMargin = kCapTiles * 32;   // appends one warp can make per query in that time
 constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
 
 __device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
@@ -1131,10 +1134,12 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
         } else {
           failed = true;
         }
-        // check point every kCheckTiles tiles (the same tiles for every warp of the group)
+        // check point every kCheckTiles tiles (the same tiles for every warp of the group); a
+        // long item also checks the append areas' capacity at every kCapTiles-th tile
         if ((kt - kt0) % kCheckTiles == kCheckTiles - 1 && kt + 1 < kt1) {
           bool need = false;
-          if (long_item) {
+          const bool cap_check = long_item && (kt - kt0) % kCapTiles == kCapTiles - 1;
+          if (cap_check) {
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
               if (j < nmine) {
@@ -1143,7 +1148,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
               }
             }
           }
-          if (long_item && named_bar_or(bar, NTG, need || failed)) {
+          if (cap_check && named_bar_or(bar, NTG, need || failed)) {
             if (named_bar_or(bar, NTG, failed)) { failed = true; break; }
 #pragma unroll 1
             for (int jj = 0; jj < nloc; ++jj) {
