@@ -41,3 +41,19 @@ def test_clock_summary_falls_back_to_all_samples():
     c.t0, c.t1 = t0, t0 + datetime.timedelta(milliseconds=5)
     s = c.summary()
     assert s["samples"] == 1 and not s["in_timed_region"] and s["sm_mhz"] == 1700
+
+
+def test_profile_traffic_reads_the_record_of_the_current_source():
+    from dsa_lightning_indexer_03_b200 import build as B
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    want = {}
+    for line in open(path):
+        line = line.strip()
+        if line and not line.startswith("#"):
+            key, _, rest = line.rpartition(":")
+            n, h = rest.split()[:2]
+            want[key.strip()] = (float(n), h)
+    for key, (n, h) in want.items():
+        got = bench._profile_traffic(key)
+        assert got == (n if h == B.source_hash() else None), key
+    assert bench._profile_traffic("score_topk:no_such_workload") is None
