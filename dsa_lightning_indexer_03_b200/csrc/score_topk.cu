@@ -405,7 +405,7 @@ constexpr int kBinShift = 21;                  // first-level bin = key >> kBinS
 constexpr int kBins1 = 1 << (32 - kBinShift);  // 2,048 bins
 constexpr int kSubShift = kBinShift - 11;      // second-level bin = next 11 bits
 constexpr int kListCap = 1024;                 // boundary-bin candidates gathered in shared memory
-constexpr int kCheckTiles = 8;                 // key tiles between threshold updates
+constexpr int kCheckTiles = 16;                // key tiles between threshold updates
 constexpr int kCapTiles = 16;                  // key tiles between capacity checks (long items)
 constexpr int kCheckMargin = kCapTiles * 32;   // appends one warp can make per query in that time
 constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
