@@ -905,6 +905,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
         sched_item[slot] = it;
         mbar_arrive(&sched_full[slot]);
         if (it < 0) {
+          // no work left for this CTA: a programmatic dependent (the merge of the split-key
+          // path) may be scheduled once every CTA got here; it still waits for this grid's end
+          asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
           if constexpr (ALT) {
             // the other group waits on the next slot: end it as well
             const int l2 = local + 1, s2 = l2 & 1;
@@ -1296,7 +1299,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
 
 // ------------------------------------------------------------------------------------------
 // merge of the split-key path: top-k over the kMaxChunks partial lists of one query
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = 1024;
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __restrict__ part_keys,
                                                               const int32_t* __restrict__ part_idx,
@@ -1306,9 +1309,12 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK]
   __shared__ uint32_t hist[kHistBins];
   __shared__ uint32_t mlist[kRankList];
-  __shared__ uint32_t scratch[64];
+  __shared__ uint32_t scratch[3 * (kMergeThreads / 32)];
   __shared__ int sh[8];
   __shared__ int ctr[2];
+  // launched as a programmatic dependent of the score kernel: the partial lists are read
+  // only after that grid completed and its writes are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = blockIdx.x;
   const int nch = tok_nchunks[t];
   if (nch < 2) return;
@@ -1611,9 +1617,21 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
     const int msmem = kMaxChunks * kTopK * 4;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (e != cudaSuccess) return e;
-    merge_kernel<<<a.T, kMergeThreads, msmem, s>>>(ws.part_keys, ws.part_idx, ws.tok_nchunks, a.idx_out,
-                                                    a.score_out);
-    return cudaGetLastError();
+    // programmatic dependent of the score kernel, whose CTAs release it when the work list
+    // runs dry: the merge's launch overlaps the score kernel's last items
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3(a.T);
+    mc.blockDim = dim3(kMergeThreads);
+    mc.dynamicSmemBytes = msmem;
+    mc.stream = s;
+    cudaLaunchAttribute mattr[1];
+    mattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    mattr[0].val.programmaticStreamSerializationAllowed = 1;
+    mc.attrs = mattr;
+    mc.numAttrs = 1;
+    return cudaLaunchKernelEx(&mc, merge_kernel, static_cast<const uint32_t*>(ws.part_keys),
+                              static_cast<const int32_t*>(ws.part_idx), static_cast<const int*>(ws.tok_nchunks),
+                              a.idx_out, a.score_out);
   }
   return launch_score<kPrefillQ, 3, 2, 2, 8, false>(tmQ8, tmK, sp, grid, s);
 }
