@@ -46,7 +46,7 @@ extern "C" {
 typedef enum {
   DSA_OK = 0,
   DSA_ERR_INVALID_ARG = 1,    /* NULL/misaligned pointer, bad size, bad config */
-  DSA_ERR_UNSUPPORTED = 2,    /* a valid request this build does not implement */
+  DSA_ERR_UNSUPPORTED = 2,    /* a valid request this library does not implement */
   DSA_ERR_CUDA = 3,           /* a CUDA runtime/driver call or a launch failed */
   DSA_ERR_OOM = 4,            /* device allocation failed at create */
   DSA_ERR_WORKSPACE = 5,      /* T exceeds the handle's max_tokens */
