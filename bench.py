@@ -7,7 +7,8 @@ A step is one pass of the hot path over one batch: the projections
 (dsa_indexer_project) and the score + top-2,048 (dsa_indexer_topk).  The
 headline workload is the 8,192-token single-sequence prefill; the decode step
 (64 sequences, caches of 16K..128K tokens) is measured in the same run and
-reported under "decode".  Inputs are seeded synthetic tensors resident in HBM;
+reported under "decode"; the projections' share of the prefill step, timed by the
+same events, under "projections".  Inputs are seeded synthetic tensors resident in HBM;
 L2 is flushed (256 MB write) between timed steps, outside the timed events.
 
 With N > 1 (torchrun), every rank runs its own independent batch (weak
@@ -236,9 +237,10 @@ def _setup_decode(d, seed_offset, device):
 
 
 def _time_steps(fn, steps, flush):
-    """Per-step CUDA events (L2 flushed between steps, outside the events);
-    returns (step ms list, inner ms list)."""
-    outer, inner = [], []
+    """Per-step CUDA events (L2 flushed between steps, outside the events); fn records
+    its two events around the score + top-k, after the projections.  Returns the step,
+    score + top-k and projection ms lists."""
+    outer = []
     for _ in range(steps):
         flush()
         e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -247,7 +249,23 @@ def _time_steps(fn, steps, flush):
         e[3].record()
         outer.append(e)
     torch.cuda.synchronize()
-    return ([a[0].elapsed_time(a[3]) for a in outer], [a[1].elapsed_time(a[2]) for a in outer])
+    return ([a[0].elapsed_time(a[3]) for a in outer], [a[1].elapsed_time(a[2]) for a in outer],
+            [a[0].elapsed_time(a[1]) for a in outer])
+
+
+def projection_report(T, ms, peak_tflops, hbm_gbs):
+    """Throughput of dsa_indexer_project over T tokens in ms: the q GEMM (1,536 -> 4,096)
+    and the k|w GEMM (7,168 -> 128 + 32) with its LayerNorm epilogue, run concurrently.
+    Algorithmic flops are the two GEMMs'; algorithmic bytes are the activations read
+    once, the weights read once and q, k, w written once."""
+    flops = 2 * T * (1536 * 4096 + 7168 * 160)
+    nbytes = (T * (7168 * 2 + 1536 * 2 + 4096 * 2 + 128 * 2 + 32 * 4)
+              + (1536 * 4096 + 7168 * 160) * 2)
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "tokens": T, "flop": flops, "bytes": nbytes,
+            "achieved_tflops": round(tflops, 2), "frac_tensor": round(tflops / peak_tflops, 4),
+            "achieved_gbs": round(gbs, 2), "frac_hbm": round(gbs / hbm_gbs, 4)}
 
 
 def _e2e_prefill(st, steps, n_chunks=4):
@@ -337,13 +355,15 @@ def gpu_arm(args, rank, world, local_rank, dist):
     barrier()
     with ClockSampler(device.index) as clk:
         clk.mark_start()
-        step_ms, topk_ms = _time_steps(fn, args.steps, flush)
+        step_ms, topk_ms, proj_ms = _time_steps(fn, args.steps, flush)
         clk.mark_end()
     barrier()
     clocks = clk.summary()
     ms = mx(statistics.mean(step_ms))
     topk_avg = mx(statistics.mean(topk_ms))
+    proj_avg = mx(statistics.mean(proj_ms))
     pairs = st["pairs"]
+    st_tokens = st["hidden"].shape[0]
     value = whole_job_rate(pairs, world, ms) / 1e9
     achieved_tflops = pairs * FLOP_PER_PAIR / (topk_avg * 1e-3) / 1e12
     traffic = _profile_traffic(f"score_topk:{args.workload}")
@@ -371,7 +391,7 @@ def gpu_arm(args, rank, world, local_rank, dist):
 
         _time_steps(dfn, args.warmup, flush)
         barrier()
-        dstep, dtopk = _time_steps(dfn, args.steps, flush)
+        dstep, dtopk, _ = _time_steps(dfn, args.steps, flush)
         barrier()
         dms = mx(statistics.mean(dtopk))
         dstep_ms = mx(statistics.mean(dstep))
@@ -407,6 +427,7 @@ def gpu_arm(args, rank, world, local_rank, dist):
                      "ms_per_launch": round(topk_avg, 4), "peak_source": peaks["source"] + " burst bf16"},
         "e2e": {"value": round(whole_job_rate(pairs, world, e2e_ms) / 1e9, 3), "unit": "Gpairs/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
+        "projections": projection_report(st_tokens, proj_avg, peaks["bf16_tflops"], peaks["hbm_gbs"]),
         "clocks": clocks,
         "gpu_launches": args.steps * 4,
     }
