@@ -112,7 +112,9 @@ dsa_status_t dsa_indexer_destroy(dsa_indexer_t h);
  * The key is k = bf16(gamma * (x - mean) / sqrt(var + eps) + beta) with
  * x = hidden W_k kept in fp32 and the biased variance.  A token whose position
  * lies outside [0, rows of its sequence) gets no key row and sets
- * DSA_ERR_DEVICE_BOUNDS.  T = 0 is a no-op. */
+ * DSA_ERR_DEVICE_BOUNDS.  T = 0 is a no-op.  One call covers at most
+ * 8,388,480 tokens (65,535 tiles of 128 rows): a larger T is refused at launch
+ * and returns DSA_ERR_CUDA, so project longer inputs in several calls. */
 dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
                                  const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
                                  void* key_cache, int64_t cache_rows, const int64_t* cache_offsets, void* q_out,
