@@ -3,17 +3,20 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-A step is one pass of the hot path over one batch: the projections
-(dsa_indexer_project) and the score + top-2,048 (dsa_indexer_topk).  The
-headline workload is the 8,192-token single-sequence prefill; the decode step
-(64 sequences, caches of 16K..128K tokens) is measured in the same run and
-reported under "decode"; the projections' share of the prefill step, timed by the
-same events, under "projections".  Inputs are seeded synthetic tensors resident in HBM;
-L2 is flushed (256 MB write) between timed steps, outside the timed events.
+A step is one pass of the whole hot path over one batch: the projections
+(dsa_indexer_project: q, and k|w with the key LayerNorm) and the score + top-2,048
+(dsa_indexer_topk).  The headline workload is the long-context chunked prefill:
+one 131,072-token sequence processed as 16 chunks of 8,192 queries, each chunk
+projected and then scored against every causal prior key of the cache
+(8,590,000,128 causal pairs per step).  The other four workloads (prefill_3k,
+prefill_8k, prefill_2x32k_heavy, decode_64) are timed in the same run and reported
+under "workloads", each with its own roofline.  Inputs are seeded synthetic tensors
+resident in HBM; L2 is flushed (256 MB write) between timed steps, outside the
+timed events.
 
-With N > 1 (torchrun), every rank runs its own independent batch (weak
-scaling, no collective on the data path); times are the max over ranks.
---impl reference times the CPU oracle on a bounded sample of the same workload.
+With N > 1 (torchrun), every rank runs its own independent batch (weak scaling,
+no collective on the data path); times are the max over ranks.  --impl reference
+times the CPU oracle on bounded samples of the same workload.
 """
 
 from __future__ import annotations
@@ -38,6 +41,14 @@ import workloads as W  # noqa: E402
 METRIC = "indexer score+top-2048 Gpairs/s (prefill), decode GB/s; % of roofline"
 FLOP_PER_PAIR = 2 * 32 * 128           # one (query, key) pair: 32 heads x 128-dim dot products
 L2_FLUSH_BYTES = 256 << 20
+HEADLINE = "chunked_128k"
+PREFILL_WORKLOADS = ["prefill_3k", "prefill_8k", "prefill_2x32k_heavy", "chunked_128k"]
+ALL_WORKLOADS = PREFILL_WORKLOADS + ["decode_64"]
+
+# kernels of this library launched by one call of each entry point (the timed region holds
+# nothing else of ours): project = q GEMM + k|w GEMM with the LayerNorm epilogue;
+# topk = prep + score kernel, plus the merge on the split-key path
+LAUNCHES = {"project": 2, "topk": 2, "topk_split": 3}
 
 
 # ------------------------------------------------------------------------------------------ helpers
@@ -168,89 +179,37 @@ def _cpu_threads():
     return os.cpu_count() or 1
 
 
-# ------------------------------------------------------------------------------------------ GPU arm
+class Spans(list):
+    """CUDA event spans recorded inside one step: (kind, start event, end event)."""
 
-def _setup_prefill(d, name, seed_offset, device):
-    cfg = W.WORKLOADS[name]
-    wts = W.make_weights(cfg["weight_seed"])
-    batch = W.make_prefill(cfg["act_seed"] + seed_offset, cfg["seq_lens"])
-    to = lambda t: t.to(device).contiguous()  # noqa: E731
-    ix = d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta),
-                   max_tokens=max(batch.hidden.shape[0], 256))
-    T = batch.hidden.shape[0]
-    rows = int(batch.cache_offsets[-1])
-    st = dict(ix=ix, T=T, host=batch,
-              hidden=to(batch.hidden), q_latent=to(batch.q_latent), positions=to(batch.positions),
-              qoff=to(batch.q_seq_offsets), coff=to(batch.cache_offsets),
-              cache=torch.zeros((rows, 128), dtype=torch.bfloat16, device=device),
-              q=torch.empty((T, 32, 128), dtype=torch.bfloat16, device=device),
-              w=torch.empty((T, 32), dtype=torch.float32, device=device),
-              idx=torch.empty((T, 2048), dtype=torch.int32, device=device),
-              score=torch.empty((T, 2048), dtype=torch.float32, device=device),
-              pairs=W.causal_pairs(batch.positions))
-    return st
-
-
-def _prefill_step(st, ev=None):
-    ix = st["ix"]
-    ix.project(st["hidden"], st["q_latent"], st["positions"], st["qoff"], st["cache"], st["coff"],
-               q_out=st["q"], w_out=st["w"])
-    if ev is not None:
-        ev[0].record()
-    ix.topk(st["q"], st["w"], st["positions"], st["qoff"], st["cache"], st["coff"], idx_out=st["idx"],
-            score_out=st["score"])
-    if ev is not None:
-        ev[1].record()
-
-
-def _setup_decode(d, seed_offset, device):
-    cfg = W.WORKLOADS["decode_64"]
-    wts = W.make_weights(cfg["weight_seed"])
-    lengths = W.decode_lengths(cfg["act_seed"] + seed_offset, cfg["batch"], cfg["L_min"], cfg["L_max"])
-    batch = W.make_decode(cfg["act_seed"] + seed_offset, lengths=torch.ones_like(lengths))  # new tokens only
-    to = lambda t: t.to(device).contiguous()  # noqa: E731
-    ix = d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta), max_tokens=256)
-    B = cfg["batch"]
-    total = int(lengths.sum())
-    coff = torch.zeros(B + 1, dtype=torch.int64)
-    coff[1:] = torch.cumsum(lengths, 0)
-    # cached keys: LayerNorm (through the library) of N(0,1) pre-norm rows drawn on the device
-    gd = torch.Generator(device=device).manual_seed(2000 + seed_offset)
-    cache = torch.empty((total, 128), dtype=torch.bfloat16, device=device)
-    step = 1 << 20
-    for s in range(0, total, step):
-        n = min(step, total - s)
-        raw = torch.randn((n, 128), generator=gd, device=device, dtype=torch.float32)
-        ix.key_norm(raw, out=cache[s:s + n])
-    torch.cuda.synchronize()
-    positions = (lengths - 1).to(torch.int32)
-    st = dict(ix=ix, T=B, hidden=to(batch.hidden), q_latent=to(batch.q_latent), positions=to(positions),
-              qoff=to(torch.arange(B + 1, dtype=torch.int32)), coff=to(coff), cache=cache,
-              q=torch.empty((B, 32, 128), dtype=torch.bfloat16, device=device),
-              w=torch.empty((B, 32), dtype=torch.float32, device=device),
-              idx=torch.empty((B, 2048), dtype=torch.int32, device=device),
-              score=torch.empty((B, 2048), dtype=torch.float32, device=device),
-              total_keys=total)
-    # algorithmic bytes of the score + top-k: every cached key once, q/w once, indices+scores out
-    st["bytes"] = total * 128 * 2 + B * (32 * 128 * 2 + 32 * 4) + B * 2048 * (4 + 4)
-    return st
+    def span(self, kind, f):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record()
+        f()
+        e.record()
+        self.append((kind, s, e))
 
 
 def _time_steps(fn, steps, flush):
-    """Per-step CUDA events (L2 flushed between steps, outside the events); fn records
-    its two events around the score + top-k, after the projections.  Returns the step,
-    score + top-k and projection ms lists."""
-    outer = []
+    """Per-step CUDA events on the current stream (L2 flushed between steps, outside the
+    events).  fn(spans) runs one step and records its projection and score + top-k calls
+    as spans.  Returns per-step lists: step ms, score + top-k ms, projection ms."""
+    out = []
     for _ in range(steps):
         flush()
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        e[0].record()
-        fn((e[1], e[2]))
-        e[3].record()
-        outer.append(e)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        spans = Spans()
+        e0.record()
+        fn(spans)
+        e1.record()
+        out.append((e0, e1, spans))
     torch.cuda.synchronize()
-    return ([a[0].elapsed_time(a[3]) for a in outer], [a[1].elapsed_time(a[2]) for a in outer],
-            [a[0].elapsed_time(a[1]) for a in outer])
+    step = [a.elapsed_time(b) for a, b, _ in out]
+    topk = [sum(s.elapsed_time(e) for k, s, e in sp if k == "topk") for _, _, sp in out]
+    proj = [sum(s.elapsed_time(e) for k, s, e in sp if k == "project") for _, _, sp in out]
+    return step, topk, proj
 
 
 def projection_report(T, ms, peak_tflops, hbm_gbs):
@@ -268,66 +227,227 @@ def projection_report(T, ms, peak_tflops, hbm_gbs):
             "achieved_gbs": round(gbs, 2), "frac_hbm": round(gbs / hbm_gbs, 4)}
 
 
-def _e2e_prefill(st, steps, n_chunks=4):
-    """Same metric through the public API with host buffers: every step copies the inputs in
-    from pinned host memory and the indices out, in n_chunks chunks of query tokens on a copy
-    stream, so that chunk c+1's inputs travel while chunk c is projected and scored (the
-    chunked-prefill use of the API: each chunk's queries see the keys of every earlier chunk,
-    already in the cache).  Returns (ms per step, H2D bytes, D2H bytes)."""
+def prefill_roofline(pairs, topk_ms, peaks, traffic):
+    """Roofline of the score + top-k over a prefill workload: pairs x 8,192 flop over the
+    summed dsa_indexer_topk time, against the measured burst bf16 peak."""
+    tflops = pairs * FLOP_PER_PAIR / (topk_ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+            "kernel": "score_topk (dsa_indexer_topk: prep + score)", "ms_per_launch": None,
+            "ms_topk_per_step": round(topk_ms, 4), "gpairs_score_topk": round(pairs / (topk_ms * 1e-3) / 1e9, 3),
+            "peak_source": peaks["source"] + " burst bf16 (" + ("of measured" if peaks["source"] == "measured"
+                                                                  else "of fallback") + ")"}
+
+
+# ------------------------------------------------------------------------------------------ GPU arm: workloads
+
+def _make_indexer(d, wts, device, max_tokens):
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    return d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta), max_tokens=max_tokens)
+
+
+def setup_prefill(d, name, seed_offset, device):
+    """Inputs of a prefill workload, resident on the device.  A prefill job is a list of
+    calls ("chunks"): one call for the single-shot prefills, 16 calls of 8,192 queries for
+    the chunked long-context prefill, each scoring against the keys of every earlier chunk."""
+    cfg = W.WORKLOADS[name]
+    wts = W.make_weights(cfg["weight_seed"])
+    seed = cfg["act_seed"] + seed_offset
+    if cfg["kind"] == "chunked":
+        S, C = cfg["seq_len"], cfg["chunk"]
+        parts = [W.make_prefill(seed, [C], start_positions=[c * C], cache_lens=[S], sub=c) for c in range(S // C)]
+        hidden = torch.cat([p.hidden for p in parts])
+        q_latent = torch.cat([p.q_latent for p in parts])
+        positions = torch.cat([p.positions for p in parts])
+        qoffs = [torch.tensor([0, C], dtype=torch.int32) for _ in parts]
+        coff = torch.tensor([0, S], dtype=torch.int64)
+        bounds = [(c * C, (c + 1) * C) for c in range(S // C)]
+        heavy = None
+        seq_offsets = torch.tensor([0, S], dtype=torch.int32)
+    else:
+        batch = W.make_prefill(seed, cfg["seq_lens"])
+        hidden, q_latent, positions = batch.hidden, batch.q_latent, batch.positions
+        T = hidden.shape[0]
+        qoffs = [batch.q_seq_offsets]
+        coff = batch.cache_offsets
+        bounds = [(0, T)]
+        heavy = W.heavy_hitter_rows(seed, coff, cfg["heavy_frac"]) if "heavy_frac" in cfg else None
+        seq_offsets = batch.q_seq_offsets
+    T = hidden.shape[0]
+    chunk_T = max(b - a for a, b in bounds)
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    st = dict(name=name, T=T, bounds=bounds, ix=_make_indexer(d, wts, device, max(chunk_T, 256)),
+              host=dict(hidden=hidden, q_latent=q_latent, positions=positions, qoffs=qoffs, coff=coff),
+              hidden=to(hidden), q_latent=to(q_latent), positions=to(positions),
+              qoffs=[to(q) for q in qoffs], coff=to(coff), seq_offsets=seq_offsets,
+              heavy=None if heavy is None else to(heavy),
+              cache=torch.zeros((int(coff[-1]), 128), dtype=torch.bfloat16, device=device),
+              q=torch.empty((T, 32, 128), dtype=torch.bfloat16, device=device),
+              w=torch.empty((T, 32), dtype=torch.float32, device=device),
+              idx=torch.empty((T, 2048), dtype=torch.int32, device=device),
+              score=torch.empty((T, 2048), dtype=torch.float32, device=device),
+              pairs=W.causal_pairs(positions), weights=wts)
+    return st
+
+
+def prefill_step(st, spans):
+    """One pass of the hot path over the whole workload: per call, the projections (which
+    write the call's keys into the cache) and then the score + top-k."""
+    ix = st["ix"]
+    for (a0, a1), qoff in zip(st["bounds"], st["qoffs"]):
+        spans.span("project", lambda: ix.project(st["hidden"][a0:a1], st["q_latent"][a0:a1],
+                                                 st["positions"][a0:a1], qoff, st["cache"], st["coff"],
+                                                 q_out=st["q"][a0:a1], w_out=st["w"][a0:a1]))
+        if st["heavy"] is not None:
+            # the workload's 1 % heavy-hitter key rows (x4, exact in bf16), applied to the
+            # freshly written cache before scoring; an input-preparation step, outside the spans
+            st["cache"][st["heavy"]] *= 4
+        spans.span("topk", lambda: ix.topk(st["q"][a0:a1], st["w"][a0:a1], st["positions"][a0:a1], qoff,
+                                           st["cache"], st["coff"], idx_out=st["idx"][a0:a1],
+                                           score_out=st["score"][a0:a1]))
+
+
+def setup_decode(d, seed_offset, device):
+    cfg = W.WORKLOADS["decode_64"]
+    wts = W.make_weights(cfg["weight_seed"])
+    lengths = W.decode_lengths(cfg["act_seed"] + seed_offset, cfg["batch"], cfg["L_min"], cfg["L_max"])
+    batch = W.make_decode(cfg["act_seed"] + seed_offset, lengths=torch.ones_like(lengths))  # new tokens only
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    ix = _make_indexer(d, wts, device, 256)
+    B = cfg["batch"]
+    total = int(lengths.sum())
+    coff = torch.zeros(B + 1, dtype=torch.int64)
+    coff[1:] = torch.cumsum(lengths, 0)
+    # cached keys: LayerNorm (through the library) of N(0,1) pre-norm rows drawn on the device
+    gd = torch.Generator(device=device).manual_seed(2000 + seed_offset)
+    cache = torch.empty((total, 128), dtype=torch.bfloat16, device=device)
+    step = 1 << 20
+    for s in range(0, total, step):
+        n = min(step, total - s)
+        raw = torch.randn((n, 128), generator=gd, device=device, dtype=torch.float32)
+        ix.key_norm(raw, out=cache[s:s + n])
+    torch.cuda.synchronize()
+    positions = (lengths - 1).to(torch.int32)
+    st = dict(name="decode_64", ix=ix, T=B, hidden=to(batch.hidden), q_latent=to(batch.q_latent),
+              positions=to(positions), qoff=to(torch.arange(B + 1, dtype=torch.int32)), coff=to(coff), cache=cache,
+              q=torch.empty((B, 32, 128), dtype=torch.bfloat16, device=device),
+              w=torch.empty((B, 32), dtype=torch.float32, device=device),
+              idx=torch.empty((B, 2048), dtype=torch.int32, device=device),
+              score=torch.empty((B, 2048), dtype=torch.float32, device=device),
+              total_keys=total, lengths=lengths)
+    # algorithmic bytes of the score + top-k: every cached key once, q/w once, indices+scores out
+    st["bytes"] = total * 128 * 2 + B * (32 * 128 * 2 + 32 * 4) + B * 2048 * (4 + 4)
+    return st
+
+
+def decode_step(ds, spans):
+    ix = ds["ix"]
+    spans.span("project", lambda: ix.project(ds["hidden"], ds["q_latent"], ds["positions"], ds["qoff"], ds["cache"],
+                                             ds["coff"], q_out=ds["q"], w_out=ds["w"]))
+    spans.span("topk", lambda: ix.topk(ds["q"], ds["w"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"],
+                                       idx_out=ds["idx"], score_out=ds["score"]))
+
+
+def e2e_prefill(st, steps):
+    """The same workload through the public API with host buffers: every step copies each
+    call's inputs in from pinned host memory (on an H2D stream, all calls queued at once so
+    that the copies run ahead of the compute) and each call's indices out (on a D2H stream,
+    queued behind that call), so that call c's indices return while call c+1 is scored and
+    later inputs arrive.  Returns (ms per step, H2D bytes, D2H bytes)."""
     h = st["host"]
     ix = st["ix"]
     T = st["T"]
-    if len(h.q_seq_offsets) != 2:      # one sequence; otherwise copy and compute in one piece
-        n_chunks = 1
-    pin = {k: getattr(h, k).pin_memory() for k in ("hidden", "q_latent", "positions", "q_seq_offsets",
-                                                    "cache_offsets")}
+    pin = {k: h[k].pin_memory() for k in ("hidden", "q_latent", "positions", "coff")}
+    pin_qoffs = [q.pin_memory() for q in h["qoffs"]]
     out = torch.empty((T, 2048), dtype=torch.int32).pin_memory()
-    bi = sum(t.numel() * t.element_size() for t in pin.values())
+    bi = sum(t.numel() * t.element_size() for t in pin.values()) + sum(q.numel() * 4 for q in pin_qoffs)
     bo = out.numel() * out.element_size()
-    bounds = [T * c // n_chunks for c in range(n_chunks + 1)]
     dev = st["hidden"].device
-    qoffs = [torch.tensor([0, bounds[c + 1] - bounds[c]], dtype=torch.int32, device=dev) for c in range(n_chunks)]
-    copy = torch.cuda.Stream(device=dev)
+    h2d = torch.cuda.Stream(device=dev)
+    d2h = torch.cuda.Stream(device=dev)
     main = torch.cuda.current_stream(dev)
     ts = []
     for _ in range(steps):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(main)
-        copy.wait_stream(main)
-        with torch.cuda.stream(copy):
-            st["coff"].copy_(pin["cache_offsets"], non_blocking=True)
-            st["qoff"].copy_(pin["q_seq_offsets"], non_blocking=True)
-        arrived, done = [], []
-        for c in range(n_chunks):
-            a0, a1 = bounds[c], bounds[c + 1]
-            with torch.cuda.stream(copy):
+        h2d.wait_stream(main)
+        d2h.wait_stream(main)
+        arrived = []
+        with torch.cuda.stream(h2d):
+            st["coff"].copy_(pin["coff"], non_blocking=True)
+            for (a0, a1), qd, qh in zip(st["bounds"], st["qoffs"], pin_qoffs):
+                qd.copy_(qh, non_blocking=True)
                 st["hidden"][a0:a1].copy_(pin["hidden"][a0:a1], non_blocking=True)
                 st["q_latent"][a0:a1].copy_(pin["q_latent"][a0:a1], non_blocking=True)
                 st["positions"][a0:a1].copy_(pin["positions"][a0:a1], non_blocking=True)
                 ev = torch.cuda.Event()
-                ev.record(copy)
+                ev.record(h2d)
                 arrived.append(ev)
-        for c in range(n_chunks):
-            a0, a1 = bounds[c], bounds[c + 1]
-            main.wait_event(arrived[c])
-            qoff = st["qoff"] if n_chunks == 1 else qoffs[c]
+        for ((a0, a1), qoff), ev_in in zip(zip(st["bounds"], st["qoffs"]), arrived):
+            main.wait_event(ev_in)
             ix.project(st["hidden"][a0:a1], st["q_latent"][a0:a1], st["positions"][a0:a1], qoff, st["cache"],
                        st["coff"], q_out=st["q"][a0:a1], w_out=st["w"][a0:a1])
+            if st["heavy"] is not None:
+                st["cache"][st["heavy"]] *= 4
             ix.topk(st["q"][a0:a1], st["w"][a0:a1], st["positions"][a0:a1], qoff, st["cache"], st["coff"],
                     idx_out=st["idx"][a0:a1], score_out=st["score"][a0:a1])
-            ev = torch.cuda.Event()
-            ev.record(main)
-            done.append(ev)
-        with torch.cuda.stream(copy):
-            for c in range(n_chunks):
-                copy.wait_event(done[c])
-                out[bounds[c]:bounds[c + 1]].copy_(st["idx"][bounds[c]:bounds[c + 1]], non_blocking=True)
-        main.wait_stream(copy)
+            done = torch.cuda.Event()
+            done.record(main)
+            d2h.wait_event(done)
+            with torch.cuda.stream(d2h):
+                out[a0:a1].copy_(st["idx"][a0:a1], non_blocking=True)
+        main.wait_stream(d2h)
         e1.record(main)
         e1.synchronize()
         ts.append(e0.elapsed_time(e1))
     return statistics.mean(ts), bi, bo
+
+
+def run_prefill(d, name, rank, device, steps, warmup, flush, peaks, mx, clk=None):
+    st = setup_prefill(d, name, rank, device)
+    fn = lambda spans: prefill_step(st, spans)  # noqa: E731
+    _time_steps(fn, warmup, flush)
+    torch.cuda.synchronize()
+    if clk is not None:
+        clk.mark_start()
+    step_ms, topk_ms, proj_ms = _time_steps(fn, steps, flush)
+    if clk is not None:
+        clk.mark_end()
+    ms = mx(statistics.mean(step_ms))
+    topk_avg = mx(statistics.mean(topk_ms))
+    proj_avg = mx(statistics.mean(proj_ms))
+    err = st["ix"].device_error()
+    n_calls = len(st["bounds"])
+    rec = {"workload": name, "metric": "indexer score+top-2048 Gpairs/s (prefill)",
+           "value": None, "unit": "Gpairs/s", "ms_per_step": round(ms, 4), "causal_pairs": st["pairs"],
+           "tokens": st["T"], "calls_per_step": n_calls,
+           "roofline": prefill_roofline(st["pairs"], topk_avg, peaks, _profile_traffic(f"score_topk:{name}")),
+           "projections": projection_report(st["T"], proj_avg, peaks["bf16_tflops"], peaks["hbm_gbs"]),
+           "device_error": err, "gpu_launches_per_step": n_calls * (LAUNCHES["project"] + LAUNCHES["topk"])}
+    rec["roofline"]["ms_per_launch"] = round(topk_avg / n_calls, 4)
+    return st, rec, ms
+
+
+def run_decode(d, rank, device, steps, warmup, flush, peaks, mx):
+    ds = setup_decode(d, rank, device)
+    fn = lambda spans: decode_step(ds, spans)  # noqa: E731
+    _time_steps(fn, warmup, flush)
+    dstep, dtopk, dproj = _time_steps(fn, steps, flush)
+    dms = mx(statistics.mean(dtopk))
+    dstep_ms = mx(statistics.mean(dstep))
+    gbs = ds["bytes"] / (dms * 1e-3) / 1e9
+    rec = {"workload": "decode_64", "metric": "decode GB/s", "value": None, "unit": "GB/s",
+           "ms_score_topk": round(dms, 4), "ms_per_step": round(dstep_ms, 4), "ms_project": round(
+               mx(statistics.mean(dproj)), 4),
+           "keys_scanned": ds["total_keys"], "algorithmic_bytes": ds["bytes"],
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": _profile_traffic("score_topk:decode_64"),
+                        "kernel": "score_topk split-key + merge (dsa_indexer_topk)", "ms_per_launch": round(dms, 4),
+                        "peak_source": peaks["source"] + " HBM copy"},
+           "device_error": ds["ix"].device_error(),
+           "gpu_launches_per_step": LAUNCHES["project"] + LAUNCHES["topk_split"]}
+    return ds, rec, gbs
 
 
 def gpu_arm(args, rank, world, local_rank, dist):
@@ -348,150 +468,219 @@ def gpu_arm(args, rank, world, local_rank, dist):
     def mx(x):
         return max_over_ranks(x, dist, device)
 
-    # ---------------- prefill (headline)
-    st = _setup_prefill(d, args.workload, rank, device)
-    fn = lambda ev: _prefill_step(st, ev)  # noqa: E731
-    _time_steps(fn, args.warmup, flush)
+    # ---------------- headline: every rank runs the same sequence of timed sections
     barrier()
     with ClockSampler(device.index) as clk:
-        clk.mark_start()
-        step_ms, topk_ms, proj_ms = _time_steps(fn, args.steps, flush)
-        clk.mark_end()
+        st, head, ms = run_prefill(d, args.workload, rank, device, args.steps, args.warmup, flush, peaks, mx, clk)
     barrier()
     clocks = clk.summary()
-    ms = mx(statistics.mean(step_ms))
-    topk_avg = mx(statistics.mean(topk_ms))
-    proj_avg = mx(statistics.mean(proj_ms))
-    pairs = st["pairs"]
-    st_tokens = st["hidden"].shape[0]
-    value = whole_job_rate(pairs, world, ms) / 1e9
-    achieved_tflops = pairs * FLOP_PER_PAIR / (topk_avg * 1e-3) / 1e12
-    traffic = _profile_traffic(f"score_topk:{args.workload}")
-    e2e_ms, bi, bo = _e2e_prefill(st, max(2, min(args.steps, 5)))
+    value = whole_job_rate(st["pairs"], world, ms) / 1e9
+    head["value"] = round(value, 3)
+    e2e_ms, bi, bo = e2e_prefill(st, max(2, min(args.steps, 5)))
     e2e_ms = mx(e2e_ms)
-    st["ix"].device_error()
+    cfg = W.WORKLOADS[args.workload]
+    del st
+    torch.cuda.empty_cache()
 
-    # ---------------- decode (second half of the metric)
-    dec = None
-    if not args.skip_decode:
-        del st
+    # ---------------- the other workloads, each with its own roofline
+    subs = {}
+    if not args.headline_only:
+        for name in PREFILL_WORKLOADS:
+            if name == args.workload:
+                continue
+            few = name in ("prefill_2x32k_heavy", "chunked_128k")
+            n = args.steps if few else max(args.steps, 100)
+            s2, rec, ms2 = run_prefill(d, name, rank, device, n, args.warmup, flush, peaks, mx)
+            rec["value"] = round(whole_job_rate(s2["pairs"], world, ms2) / 1e9, 3)
+            rec["steps"] = n
+            subs[name] = rec
+            del s2
+            torch.cuda.empty_cache()
+        n = max(args.steps, 100)
+        ds, rec, gbs = run_decode(d, rank, device, n, args.warmup, flush, peaks, mx)
+        rec["value"] = round(gbs * world, 2)
+        rec["steps"] = n
+        subs["decode_64"] = rec
+        del ds
         torch.cuda.empty_cache()
-        ds = _setup_decode(d, rank, device)
 
-        def dfn(ev):
-            ix = ds["ix"]
-            ix.project(ds["hidden"], ds["q_latent"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"],
-                       q_out=ds["q"], w_out=ds["w"])
-            if ev is not None:
-                ev[0].record()
-            ix.topk(ds["q"], ds["w"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"], idx_out=ds["idx"],
-                    score_out=ds["score"])
-            if ev is not None:
-                ev[1].record()
-
-        _time_steps(dfn, args.warmup, flush)
-        barrier()
-        dstep, dtopk, _ = _time_steps(dfn, args.steps, flush)
-        barrier()
-        dms = mx(statistics.mean(dtopk))
-        dstep_ms = mx(statistics.mean(dstep))
-        gbs = ds["bytes"] / (dms * 1e-3) / 1e9
-        dec = {"workload": "decode_64", "metric": "decode GB/s", "value": round(gbs * world, 2), "unit": "GB/s",
-               "ms_score_topk": round(dms, 4), "ms_per_step": round(dstep_ms, 4),
-               "keys_scanned": ds["total_keys"], "algorithmic_bytes": ds["bytes"],
-               "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": round(gbs / peaks["hbm_gbs"], 4),
-                            "traffic": _profile_traffic("score_topk:decode_64")}}
-        ds["ix"].device_error()
-
+    launches = head["gpu_launches_per_step"] * args.steps
     line = {
         "metric": METRIC,
-        "value": round(value, 3),
+        "value": head["value"],
         "unit": "Gpairs/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms, 4),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) random-init weights)",
-        "config": {"workload": args.workload, "batch": len(W.WORKLOADS[args.workload]["seq_lens"]),
-                   "seq_len": W.WORKLOADS[args.workload]["seq_lens"][0], "heads": 32, "head_dim": 128,
-                   "top_k": 2048, "causal_pairs_per_gpu": pairs, "parallelism": f"independent replicas x{world}",
-                   "l2": "flushed between timed steps (256 MB write)"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": round(achieved_tflops / peaks["bf16_tflops"], 4),
-                     "traffic": traffic, "kernel": "score_topk (dsa_indexer_topk: prep + score)",
-                     "ms_per_launch": round(topk_avg, 4), "peak_source": peaks["source"] + " burst bf16"},
-        "e2e": {"value": round(whole_job_rate(pairs, world, e2e_ms) / 1e9, 3), "unit": "Gpairs/s",
+        "config": {"workload": args.workload,
+                   "batch": 1 if cfg["kind"] == "chunked" else len(cfg["seq_lens"]),
+                   "seq_len": cfg["seq_len"] if cfg["kind"] == "chunked" else cfg["seq_lens"][0],
+                   "chunk": cfg.get("chunk"), "calls_per_step": head["calls_per_step"],
+                   "heads": 32, "head_dim": 128, "top_k": 2048, "causal_pairs_per_gpu": head["causal_pairs"],
+                   "parallelism": f"independent replicas x{world}",
+                   "l2": "flushed between timed steps (256 MB write); inputs larger than L2"},
+        "roofline": head["roofline"],
+        "e2e": {"value": round(whole_job_rate(head["causal_pairs"], world, e2e_ms) / 1e9, 3), "unit": "Gpairs/s",
                 "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "ms_per_step": round(e2e_ms, 4)},
-        "projections": projection_report(st_tokens, proj_avg, peaks["bf16_tflops"], peaks["hbm_gbs"]),
+        "projections": head["projections"],
         "clocks": clocks,
-        "gpu_launches": args.steps * 4,
+        "gpu_launches": launches,
+        "device_error": head["device_error"],
     }
-    if dec is not None:
-        line["decode"] = dec
+    if subs:
+        line["workloads"] = subs
     return line
 
 
-# ------------------------------------------------------------------------------------------ CPU oracle arm
+# ------------------------------------------------------------------------------------------ CPU oracle
 
-def cpu_oracle_sample(name, proj_tokens=256, n_rows=12, seed=0):
-    """The oracle as it stands, on bounded samples of the workload: its projection
-    of `proj_tokens` tokens (seconds per token) and its score + top-k of `n_rows`
-    query rows spread over the positions (seconds per causal pair), extrapolated
-    to the whole workload.  Returns (Gpairs/s, description, seconds spent)."""
+def _oracle_weights(wts):
+    f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
+    return f(wts.W_q), f(wts.W_k), f(wts.W_w), f(wts.gamma), f(wts.beta)
+
+
+def cpu_oracle_workload(name, n_rows=512, proj_tokens=256, seed=0, full=None):
+    """The oracle as it stands, timed on the workload: its projection (seconds per token,
+    from `proj_tokens` tokens or every token) and its score + top-k (seconds per causal
+    pair, from every query row or a stratified sample of `n_rows`: the first and last row
+    of every sequence and chunk, the rows at positions 2,046..2,049, one seeded row per
+    equal stratum), extrapolated to the whole workload where sampled.  The score step's
+    cost does not depend on the key values, so sampled runs score against the oracle's
+    LayerNorm of N(0,1) pre-norm rows (the keys' distribution) instead of projecting every
+    key.  Returns (value, unit, description, seconds spent)."""
     import numpy as np
 
     import oracle
     cfg = W.WORKLOADS[name]
     wts = W.make_weights(cfg["weight_seed"])
-    batch = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
-    T = batch.hidden.shape[0]
+    Wq, Wk, Ww, g, b = _oracle_weights(wts)
     f = lambda t: t.to(torch.float64).numpy()  # noqa: E731
-    Wq, Wk, Ww, g, b = f(wts.W_q), f(wts.W_k), f(wts.W_w), f(wts.gamma), f(wts.beta)
-    hid = f(batch.hidden[:proj_tokens])
-    qlat = f(batch.q_latent[:proj_tokens])
+    spent = 0.0
+    if cfg["kind"] == "decode":
+        lengths = W.decode_lengths(cfg["act_seed"], cfg["batch"], cfg["L_min"], cfg["L_max"])
+        batch = W.make_decode(cfg["act_seed"], lengths=torch.ones_like(lengths))
+        t0 = time.perf_counter()
+        q, k_new, w = oracle.project(f(batch.hidden), f(batch.q_latent), Wq, Wk, Ww, g, b)
+        t_proj = time.perf_counter() - t0
+        t_norm = 0.0
+        t_topk = 0.0
+        for bi, L in enumerate(lengths.tolist()):   # one sequence's cache at a time
+            raw = W.make_decode(cfg["act_seed"] + 1000 + bi, lengths=[L]).raw_keys
+            t0 = time.perf_counter()
+            keys = oracle.key_norm(raw.numpy().astype(np.float64), g, b)
+            keys[L - 1] = k_new[bi]
+            t1 = time.perf_counter()
+            oracle.topk(q[bi:bi + 1], w[bi:bi + 1], np.array([L - 1]), np.array([0, 1]), keys, np.array([0, L]))
+            t_topk += time.perf_counter() - t1
+            t_norm += t1 - t0
+        total = int(lengths.sum())
+        nbytes = total * 128 * 2 + len(lengths) * (32 * 128 * 2 + 32 * 4) + len(lengths) * 2048 * 8
+        spent = t_proj + t_norm + t_topk
+        gbs = nbytes / (t_proj + t_topk) / 1e9
+        desc = (f"decode_64 in full: projection of the 64 new tokens ({t_proj:.2f} s) and score+top-k of the 64 "
+                f"queries over all {total} cached keys ({t_topk:.2f} s; the cache's LayerNorm, {t_norm:.1f} s, is "
+                f"input preparation and not counted); algorithmic bytes {nbytes} as for the GPU")
+        return gbs, "GB/s", desc, spent
+    if cfg["kind"] == "chunked":
+        S, C = cfg["seq_len"], cfg["chunk"]
+        positions = torch.arange(S, dtype=torch.int32)
+        qoff = torch.tensor([0, S], dtype=torch.int32)
+        coff = np.array([0, S])
+        chunk = C
+        tok = W.make_prefill(cfg["act_seed"], [proj_tokens], start_positions=[S - proj_tokens], cache_lens=[S],
+                             sub=S // C - 1)
+        hid_s, qlat_s = tok.hidden, tok.q_latent
+    else:
+        batch = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
+        positions, qoff = batch.positions, batch.q_seq_offsets
+        coff = batch.cache_offsets.numpy()
+        chunk = None
+        hid_s, qlat_s = batch.hidden, batch.q_latent
+    T = positions.numel()
+    full = (T <= 8192) if full is None else full
+    if full:
+        rows = np.arange(T)
+        n_tok = T
+    else:
+        rows = W.stratified_rows(qoff, n_rows, seed=seed, chunk=chunk, positions=positions).numpy()
+        n_tok = min(proj_tokens, hid_s.shape[0])
     t0 = time.perf_counter()
-    oracle.project(hid, qlat, Wq, Wk, Ww, g, b)
-    t_proj = (time.perf_counter() - t0) / proj_tokens
-    # score + top-k rows: keys = the oracle's key norm of seeded pre-norm rows (the
-    # workload's key distribution), q / w of the sampled rows from the oracle projection
-    rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(np.arange(T // 2, T), size=n_rows, replace=False))
-    raw = W.make_decode(cfg["act_seed"], lengths=[T]).raw_keys
-    keys = oracle.key_norm(raw.to(torch.float64).numpy(), g, b)
-    q, _, w = oracle.project(f(batch.hidden[rows]), f(batch.q_latent[rows]), Wq, Wk, Ww, g, b)
-    qq = np.zeros((T, 32, 128))
-    ww = np.zeros((T, 32))
-    qq[rows] = q
-    ww[rows] = w
+    q_s, k_s, w_s = oracle.project(f(hid_s[:n_tok]), f(qlat_s[:n_tok]), Wq, Wk, Ww, g, b)
+    t_proj_tok = (time.perf_counter() - t0) / n_tok
+    spent += t_proj_tok * n_tok
+    seq = oracle.sequence_of(qoff.numpy(), T)
+    if full:
+        keys = k_s
+        qq, ww, pos_r = q_s, w_s, positions.numpy()
+        qoff_r = qoff.numpy()
+        if "heavy_frac" in cfg:
+            keys = keys.copy()
+            keys[W.heavy_hitter_rows(cfg["act_seed"], batch.cache_offsets, cfg["heavy_frac"]).numpy()] *= 4
+    else:
+        rows_cache = int(coff[-1])
+        keys = oracle.key_norm(W.make_decode(cfg["act_seed"], lengths=[rows_cache]).raw_keys.numpy()
+                               .astype(np.float64), g, b)
+        if "heavy_frac" in cfg:
+            keys[W.heavy_hitter_rows(cfg["act_seed"], batch.cache_offsets, cfg["heavy_frac"]).numpy()] *= 4
+        # the sampled rows as a batch of their own: q, w from the oracle's projection of the
+        # sampled tokens (reused cyclically), each row in its own sequence's key range
+        qq = q_s[np.arange(len(rows)) % n_tok]
+        ww = w_s[np.arange(len(rows)) % n_tok]
+        pos_r = positions.numpy()[rows]
+        qoff_r = np.zeros(len(coff), np.int64)
+        qoff_r[1:] = np.cumsum(np.bincount(seq[rows], minlength=len(coff) - 1))
     t0 = time.perf_counter()
-    oracle.topk(qq, ww, batch.positions.numpy(), batch.q_seq_offsets.numpy(), keys, np.array([0, T]), rows=rows)
+    oracle.topk(qq, ww, pos_r, qoff_r, keys, coff)
     t_topk = time.perf_counter() - t0
-    pairs_s = int((batch.positions[rows].to(torch.int64) + 1).sum())
-    total_pairs = W.causal_pairs(batch.positions)
-    t_full = T * t_proj + total_pairs * (t_topk / pairs_s)
-    desc = (f"{name}: projection of {proj_tokens} tokens ({t_proj * 1e3:.2f} ms/token) and score+top-k of "
-            f"{n_rows} query rows ({pairs_s} causal pairs, {t_topk:.2f} s), extrapolated to all {T} tokens "
-            f"/ {total_pairs} pairs ({t_full:.0f} s)")
-    return total_pairs / t_full / 1e9, desc, t_proj * proj_tokens + t_topk
+    spent += t_topk
+    pairs_s = int((positions.numpy()[rows].astype(np.int64) + 1).sum())
+    total_pairs = W.causal_pairs(positions)
+    t_full = T * t_proj_tok + total_pairs * (t_topk / pairs_s)
+    if full:
+        desc = (f"{name} in full: projection of all {T} tokens ({t_proj_tok * T:.1f} s) and score+top-k of all {T} "
+                f"query rows ({total_pairs} causal pairs, {t_topk:.1f} s)")
+    else:
+        desc = (f"{name}: projection of {n_tok} tokens ({t_proj_tok * 1e3:.2f} ms/token) and score+top-k of "
+                f"{len(rows)} stratified query rows (first/last row of every sequence and chunk, positions "
+                f"2046-2049, one seeded row per stratum; {pairs_s} causal pairs, {t_topk:.1f} s), extrapolated to "
+                f"all {T} tokens / {total_pairs} pairs ({t_full:.0f} s)")
+    return total_pairs / t_full / 1e9, "Gpairs/s", desc, spent
+
+
+def cpu_baselines(headline, all_workloads=True):
+    """cpu_baseline of the headline workload and of every other one (rank 0, N=1 only)."""
+    cores = _cpu_threads()
+    out = {}
+    names = [headline] + ([n for n in ALL_WORKLOADS if n != headline] if all_workloads else [])
+    for name in names:
+        v, unit, desc, spent = cpu_oracle_workload(name)
+        out[name] = {"value": float(f"{v:.6g}"), "unit": unit, "cores": cores, "kind": "oracle",
+                     "sample": desc + f"; one process, numpy BLAS on {cores} threads for the matmuls"}
+        print(f"cpu_baseline {name}: {v:.4g} {unit} ({spent:.1f} s)", file=sys.stderr, flush=True)
+    return out
 
 
 def reference_arm(args):
+    """The reference arm: the oracle as it stands on bounded samples of the headline workload
+    (each step: 16 stratified query rows and the projection of 16 tokens, seeded by the step)."""
     vals = []
     desc = ""
-    for _ in range(min(args.warmup, 1)):
-        cpu_oracle_sample(args.workload, proj_tokens=32, n_rows=2)
+    for i in range(min(args.warmup, 1)):
+        cpu_oracle_workload(args.workload, n_rows=4, proj_tokens=4, seed=10_000 + i, full=False)
     wall = 0.0
     for i in range(args.steps):
-        v, desc, spent = cpu_oracle_sample(args.workload, seed=i)
+        v, unit, desc, spent = cpu_oracle_workload(args.workload, n_rows=16, proj_tokens=16, seed=i, full=False)
         vals.append(v)
         wall += spent
     value = statistics.mean(vals)
     cores = _cpu_threads()
+    cfg = W.WORKLOADS[args.workload]
     return {
         "impl": "reference",
         "metric": METRIC,
@@ -506,13 +695,63 @@ def reference_arm(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": args.workload, "batch": len(W.WORKLOADS[args.workload]["seq_lens"]),
-                   "seq_len": W.WORKLOADS[args.workload]["seq_lens"][0], "top_k": 2048},
+        "config": {"workload": args.workload,
+                   "batch": 1 if cfg["kind"] == "chunked" else len(cfg.get("seq_lens", [1])),
+                   "seq_len": cfg.get("seq_len") or cfg["seq_lens"][0], "top_k": 2048},
         "cpu_baseline": {"value": float(f"{value:.6g}"), "unit": "Gpairs/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+                         "sample": f"per step: {desc}; one process, numpy BLAS on {cores} threads"},
         "e2e": {"value": float(f"{value:.6g}"), "unit": "Gpairs/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+
+
+# ------------------------------------------------------------------------------------------ profiling driver
+
+def profile_call(d, spec, repeats):
+    """A small case for ncu captures: one dsa_indexer_topk call of a workload, repeated.
+    spec is WORKLOAD[:CALL]; for the chunked prefill the cache is filled by projecting the
+    chunks up to CALL one at a time, so the device holds one chunk's tensors, the key
+    cache and the workspace (well under 1 GB).  Prints the call's CUDA-event times."""
+    name, _, call = spec.partition(":")
+    cfg = W.WORKLOADS[name]
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    wts = W.make_weights(cfg["weight_seed"])
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    if cfg["kind"] == "chunked":
+        S, C = cfg["seq_len"], cfg["chunk"]
+        c_last = int(call or S // C - 1)
+        ix = _make_indexer(d, wts, device, C)
+        cache = torch.zeros((S, 128), dtype=torch.bfloat16, device=device)
+        coff = to(torch.tensor([0, S], dtype=torch.int64))
+        qoff = to(torch.tensor([0, C], dtype=torch.int32))
+        for c in range(c_last + 1):
+            b = W.make_prefill(cfg["act_seed"], [C], start_positions=[c * C], cache_lens=[S], sub=c)
+            pos = to(b.positions)
+            q, w = ix.project(to(b.hidden), to(b.q_latent), pos, qoff, cache, coff)
+        pairs = W.causal_pairs(b.positions)
+    else:
+        b = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
+        ix = _make_indexer(d, wts, device, max(b.hidden.shape[0], 256))
+        cache = torch.zeros((int(b.cache_offsets[-1]), 128), dtype=torch.bfloat16, device=device)
+        pos, qoff, coff = to(b.positions), to(b.q_seq_offsets), to(b.cache_offsets)
+        q, w = ix.project(to(b.hidden), to(b.q_latent), pos, qoff, cache, coff)
+        if "heavy_frac" in cfg:
+            cache[to(W.heavy_hitter_rows(cfg["act_seed"], b.cache_offsets, cfg["heavy_frac"]))] *= 4
+        pairs = W.causal_pairs(b.positions)
+    idx = torch.empty((q.shape[0], 2048), dtype=torch.int32, device=device)
+    sc = torch.empty((q.shape[0], 2048), dtype=torch.float32, device=device)
+    torch.cuda.synchronize()
+    for i in range(repeats):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ix.topk(q, w, pos, qoff, cache, coff, idx_out=idx, score_out=sc)
+        e1.record()
+        e1.synchronize()
+        ms = e0.elapsed_time(e1)
+        print(f"{spec} call {i}: {ms:.4f} ms, {pairs / ms / 1e6:.2f} Gpairs/s, "
+              f"{pairs * FLOP_PER_PAIR / ms / 1e9:.1f} TFLOP/s", flush=True)
+    assert ix.device_error() == d.DSA_OK
 
 
 # ------------------------------------------------------------------------------------------ main
@@ -520,13 +759,21 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill_8k", choices=["prefill_3k", "prefill_8k", "prefill_2x32k_heavy"])
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=HEADLINE, choices=PREFILL_WORKLOADS)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
-    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other workloads' records")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-call", default=None, metavar="WORKLOAD[:CALL]",
+                    help="only run one score + top-k call of a workload --steps times (for ncu captures)")
     args = ap.parse_args()
+    if args.profile_call:
+        import dsa_lightning_indexer_03_b200 as d
+        from dsa_lightning_indexer_03_b200 import build as B
+        B.build()
+        profile_call(d, args.profile_call, args.steps)
+        return
     args.warmup = max(args.warmup, 3)
 
     rank = int(os.environ.get("RANK", "0"))
@@ -540,16 +787,15 @@ def main():
 
     dist = None
     if world > 1:
-        import datetime
-
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     line = gpu_arm(args, rank, world, local_rank, dist)
-    if rank == 0 and not args.no_cpu_baseline:
-        v, desc, _ = cpu_oracle_sample(args.workload)
-        line["cpu_baseline"] = {"value": float(f"{v:.6g}"), "unit": "Gpairs/s", "cores": _cpu_threads(), "kind": "oracle",
-                                "sample": desc}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baselines(args.workload, all_workloads=not args.headline_only)
+        line["cpu_baseline"] = cb[args.workload]
+        for name, rec in line.get("workloads", {}).items():
+            rec["cpu_baseline"] = cb.get(name)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -53,6 +53,7 @@ SIGNATURES = {
     "dsa_indexer_topk": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _vp, _vp, _u32, _vp]),
     "dsa_indexer_topk_noalloc": (ctypes.c_int, [_i64, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _vp, _vp, _vp]),
     "dsa_indexer_device_error": (ctypes.c_int, [_vp]),
+    "dsa_indexer_noalloc_device_error": (ctypes.c_int, [_vp]),
     "dsa_indexer_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),
     "dsa_indexer_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "dsa_indexer_abi_version": (ctypes.c_int32, []),

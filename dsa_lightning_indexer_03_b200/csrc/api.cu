@@ -15,9 +15,19 @@
 
 using namespace dsa;
 
-namespace {
+uint64_t dsa::wait_timeout_ns() {
+  static const uint64_t t = [] {
+    const char* s = std::getenv("DSA_INDEXER_WAIT_TIMEOUT_MS");
+    if (s && *s) {
+      const long long v = std::atoll(s);
+      if (v > 0) return static_cast<uint64_t>(v) * uint64_t(1000000);
+    }
+    return static_cast<uint64_t>(2000ull * 1000 * 1000);
+  }();
+  return t;
+}
 
-constexpr uint64_t kDefaultTimeoutNs = 2000ull * 1000 * 1000;  // 2 s per pipeline wait
+namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -50,17 +60,7 @@ bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-uint64_t timeout_ns() {
-  static uint64_t t = [] {
-    const char* s = std::getenv("DSA_INDEXER_WAIT_TIMEOUT_MS");
-    if (s && *s) {
-      const long long v = std::atoll(s);
-      if (v > 0) return static_cast<uint64_t>(v) * uint64_t(1000000);
-    }
-    return static_cast<uint64_t>(kDefaultTimeoutNs);
-  }();
-  return t;
-}
+uint64_t timeout_ns() { return dsa::wait_timeout_ns(); }
 
 }  // namespace
 
@@ -287,7 +287,6 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
       (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7))
     return DSA_ERR_INVALID_ARG;
   if (cache_rows < 1 || cache_rows > (int64_t(1) << 31) - (int64_t(1) << 20)) return DSA_ERR_INVALID_ARG;
-  if (flags & DSA_TOPK_SORTED) return DSA_ERR_UNSUPPORTED;
   bool split = (T <= kSplitMaxTokens);
   if (flags & DSA_TOPK_SPLIT) {
     if (T > h->ws.part_tokens) return DSA_ERR_UNSUPPORTED;
@@ -313,6 +312,7 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
   a.idx_out = idx_out;
   a.score_out = score_out;
   a.split = split;
+  a.sorted = (flags & DSA_TOPK_SORTED) != 0;
   a.timeout_ns = timeout_ns();
   if (launch_topk(a, h->ws, tmQ1, tmQ8, tmK, h->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;

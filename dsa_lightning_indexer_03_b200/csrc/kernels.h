@@ -91,6 +91,7 @@ struct TopkArgs {
   int32_t* idx_out;
   float* score_out;
   bool split;
+  bool sorted;       // order each row by (score desc, position asc); short rows stay [0..p, -1...]
   uint64_t timeout_ns;
 };
 
@@ -98,5 +99,9 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
                         const CUtensorMap& tmK, int num_sms, cudaStream_t s);
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s);
+
+// Limit of every bounded pipeline wait in the library's kernels: 2 s, or
+// DSA_INDEXER_WAIT_TIMEOUT_MS milliseconds when that variable is set (read once).
+uint64_t wait_timeout_ns();
 
 }  // namespace dsa

@@ -39,8 +39,6 @@ constexpr size_t kOffCand = kOffNch + align256(size_t(kStaticMaxTokens) * 4);
 constexpr size_t kScratchBytes = kOffCand + align256(kCandEntries * sizeof(uint2));
 static_assert(kScratchBytes == 6473216, "the scratch size is stated in include/dsa_indexer.h");
 
-constexpr int kMaxDevices = 64;
-constexpr uint64_t kWaitTimeoutNs = 2000ull * 1000 * 1000;
 
 }  // namespace
 
@@ -49,10 +47,6 @@ constexpr uint64_t kWaitTimeoutNs = 2000ull * 1000 * 1000;
 static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
 
 namespace {
-
-std::mutex g_mu;
-unsigned char* g_scratch_addr[kMaxDevices] = {};
-int g_sms[kMaxDevices] = {};
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_fn = nullptr;
 std::once_flag g_encode_flag;
@@ -76,22 +70,16 @@ bool tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Device address of the scratch on the current device (looked up on the first call
-// made on that device, with that device current).
+// Device address of the scratch on the current device.  Looked up on every call, with the
+// caller's device current: the lookup costs far less than the launches, and an address kept
+// from an earlier call could belong to a context that no longer exists (after a device reset).
 unsigned char* scratch_on_current_device(int* num_sms) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
-    g_sms[dev] = sms;
-    g_scratch_addr[dev] = static_cast<unsigned char*>(p);
-  }
-  *num_sms = g_sms[dev];
-  return g_scratch_addr[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || p == nullptr) return nullptr;
+  if (cudaDeviceGetAttribute(num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return nullptr;
+  return static_cast<unsigned char*>(p);
 }
 
 bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -149,12 +137,25 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const
   a.idx_out = idx_out;
   a.score_out = score_out;
   a.split = false;
-  a.timeout_ns = kWaitTimeoutNs;
+  a.sorted = false;
+  a.timeout_ns = wait_timeout_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the error word keeps the previous call's bits: start each call from zero
   if (cudaMemsetAsync(ws.err, 0, sizeof(int), s) != cudaSuccess) return DSA_ERR_CUDA;
   // the prep kernel rewrites the work list and resets the work counter on every call
   if (launch_topk(a, ws, tmQ8, tmQ8, tmK, sms < kStaticCtas ? sms : kStaticCtas, s) != cudaSuccess)
     return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+extern "C" dsa_status_t dsa_indexer_noalloc_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DSA_ERR_CUDA;
+  int v = 0;
+  // the error word sits at the start of the scratch; the copy allocates nothing
+  if (cudaMemcpyFromSymbol(&v, g_topk_scratch, sizeof(int), kOffErr, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (v & kErrTimeout) return DSA_ERR_DEVICE_TIMEOUT;
+  if (v & (kErrBounds | kErrOffsets)) return DSA_ERR_DEVICE_BOUNDS;
   return DSA_OK;
 }

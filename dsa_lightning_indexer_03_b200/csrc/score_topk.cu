@@ -740,6 +740,90 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
 }
 
 // ------------------------------------------------------------------------------------------
+// DSA_TOPK_SORTED: orders one row of kTopK selected (ordered score key, position) pairs by
+// score descending, then position ascending, and writes it out.  A group of NT threads
+// (tid = 0..NT-1, named barrier `bar`) runs a bitonic sorting network over 64-bit words
+// (key << 32 | ~position), descending; thread tid holds elements tid*E .. tid*E + E - 1.
+// Compare-exchange steps between elements of one thread run in registers, between threads
+// of one warp through shuffles, and between warps through `stage` (kTopK pairs, global or
+// shared memory), which also holds the input.
+__device__ __forceinline__ uint64_t sort_word(uint2 c) {
+  return (static_cast<uint64_t>(c.x) << 32) | static_cast<uint64_t>(0xFFFFFFFFu - c.y);
+}
+
+// One compare-exchange step (distance J inside bitonic blocks of K elements).
+template <int NT, int K, int J>
+__device__ __forceinline__ void bitonic_step(uint64_t (&v)[kTopK / NT], int tid, uint64_t* s64, int bar) {
+  constexpr int E = kTopK / NT;
+  if constexpr (J < E) {
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int l = r ^ J;
+      if (l > r) {
+        const bool desc = ((tid * E + r) & K) == 0;   // the lower index keeps the larger word
+        const uint64_t a = v[r], b = v[l];
+        if (desc ? (a < b) : (a > b)) {
+          v[r] = b;
+          v[l] = a;
+        }
+      }
+    }
+  } else {
+    if constexpr (J >= 32 * E) {
+#pragma unroll
+      for (int r = 0; r < E; ++r) s64[tid * E + r] = v[r];
+      named_bar_sync(bar, NT);
+    }
+#pragma unroll
+    for (int r = 0; r < E; ++r) {
+      const int i = tid * E + r;
+      uint64_t o;
+      if constexpr (J < 32 * E) {
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v[r] >> 32), J / E);
+        const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(v[r]), J / E);
+        o = (static_cast<uint64_t>(hi) << 32) | lo;
+      } else {
+        o = s64[i ^ J];
+      }
+      const bool desc = (i & K) == 0;
+      const bool keep_max = ((i & J) == 0) == desc;   // lower index of a descending pair
+      v[r] = keep_max ? (v[r] > o ? v[r] : o) : (v[r] < o ? v[r] : o);
+    }
+    if constexpr (J >= 32 * E) named_bar_sync(bar, NT);
+  }
+}
+
+template <int NT, int K, int J>
+__device__ __forceinline__ void bitonic_merge(uint64_t (&v)[kTopK / NT], int tid, uint64_t* s64, int bar) {
+  bitonic_step<NT, K, J>(v, tid, s64, bar);
+  if constexpr (J > 1) bitonic_merge<NT, K, J / 2>(v, tid, s64, bar);
+}
+
+template <int NT, int K>
+__device__ __forceinline__ void bitonic_sort(uint64_t (&v)[kTopK / NT], int tid, uint64_t* s64, int bar) {
+  bitonic_merge<NT, K, K / 2>(v, tid, s64, bar);
+  if constexpr (K < kTopK) bitonic_sort<NT, 2 * K>(v, tid, s64, bar);
+}
+
+template <int NT>
+__device__ void sort_stage_and_emit(uint2* stage, int tid, int bar, int32_t* oi, float* os) {
+  constexpr int E = kTopK / NT;
+  static_assert(E >= 1 && (E & (E - 1)) == 0 && E * NT == kTopK, "power-of-two elements per thread");
+  uint64_t* const s64 = reinterpret_cast<uint64_t*>(stage);
+  uint64_t v[E];
+#pragma unroll
+  for (int r = 0; r < E; ++r) v[r] = sort_word(stage[tid * E + r]);
+  named_bar_sync(bar, NT);   // every entry is in registers before the stage is rewritten
+  bitonic_sort<NT, 2>(v, tid, s64, bar);
+#pragma unroll
+  for (int r = 0; r < E; ++r) {
+    const int i = tid * E + r;
+    __stcs(oi + i, static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(v[r])));
+    if (os) __stcs(os + i, ordered_to_float(static_cast<uint32_t>(v[r] >> 32)));
+  }
+}
+
+// ------------------------------------------------------------------------------------------
 template <int QPW>
 struct WGState {
   uint32_t hist[QPW][kBins1 / 2];  // per query: first-level counts of its candidates (packed)
@@ -824,7 +908,7 @@ __device__ __forceinline__ void sum_over_quad(const float (&part)[4 * QPH], floa
   }
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED>
 __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>::kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       ScoreParams p) {
@@ -1255,6 +1339,14 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
               __stcs(oi + s2, -1);
               if (os) __stcs(os + s2, -INFINITY);
             }
+          } else if constexpr (SORTED) {
+            // the query's other keep set is not read by this selection: it stages the row
+            uint2* const stage = qcand + static_cast<size_t>(jj) * kCandStride + (st.kcur[jj] ^ 1) * kTopK;
+            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+              stage[s2] = make_uint2(key, pos);
+            });
+            named_bar_sync(bar, NTG);
+            sort_stage_and_emit<NTG>(stage, gtid, bar, oi, os);
           } else {
             resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
               __stcs(oi + s2, static_cast<int>(pos));
@@ -1305,8 +1397,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
                                                               const int32_t* __restrict__ part_idx,
                                                               const int* __restrict__ tok_nchunks,
                                                               int32_t* __restrict__ idx_out,
-                                                              float* __restrict__ score_out) {
-  extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK]
+                                                              float* __restrict__ score_out, int sorted) {
+  extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK], then (sorted) kTopK staged pairs
   __shared__ uint32_t hist[kHistBins];
   __shared__ uint32_t mlist[kRankList];
   __shared__ uint32_t scratch[3 * (kMergeThreads / 32)];
@@ -1324,6 +1416,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   v.i = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
   int32_t* oi = idx_out + static_cast<size_t>(t) * kTopK;
   float* os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
+  if (sorted) {
+    uint2* const stage = reinterpret_cast<uint2*>(mkeys + kMaxChunks * kTopK);
+    select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
+                               [&](int slot, uint32_t key, int pos) {
+      stage[slot] = make_uint2(key, static_cast<uint32_t>(pos));
+    });
+    named_bar_sync(1, kMergeThreads);
+    sort_stage_and_emit<kMergeThreads>(stage, threadIdx.x, 1, oi, os);
+    return;
+  }
   select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
                              [&](int slot, uint32_t key, int pos) {
     __stcs(oi + slot, pos);
@@ -1343,6 +1445,8 @@ struct PrepParams {
   const int64_t* cache_offsets;
   int split;
   int num_sms;
+  int32_t* idx_out;   // [T, kTopK]: every row is padded when the offsets are malformed
+  float* score_out;   // [T, kTopK] or null
   TopkWorkspace ws;
 };
 
@@ -1452,6 +1556,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       *ws.work_counter = 0;
     }
     for (int t = threadIdx.x; t < p.T; t += kPrepThreads) ws.tok_nchunks[t] = 0;
+    // no query can be attributed to a sequence: every output row becomes padding
+    const size_t n4 = static_cast<size_t>(p.T) * (kTopK / 4);
+    for (size_t e = threadIdx.x; e < n4; e += kPrepThreads) {
+      reinterpret_cast<int4*>(p.idx_out)[e] = make_int4(-1, -1, -1, -1);
+      if (p.score_out) reinterpret_cast<float4*>(p.score_out)[e] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
     return;
   }
   // 2. validated positions
@@ -1545,11 +1655,11 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
   *status = ok ? 0 : ((err & kErrTimeout) ? 2 : 1);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED>
 cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const ScoreParams& p, int grid,
                          cudaStream_t s) {
   using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
-  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
+  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, SORTED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (C::kRegSplit) {
@@ -1591,6 +1701,8 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   pp.cache_offsets = a.cache_offsets;
   pp.split = a.split ? 1 : 0;
   pp.num_sms = num_sms;
+  pp.idx_out = a.idx_out;
+  pp.score_out = a.score_out;
   pp.ws = ws;
   prep_kernel<<<1, kPrepThreads, 0, s>>>(pp);
   cudaError_t e = cudaGetLastError();
@@ -1612,9 +1724,10 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
   if (a.split) {
-    e = launch_score<1, 5, 4, 2, 4, true>(tmQ1, tmK, sp, grid, s);
+    e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true>(tmQ1, tmK, sp, grid, s)
+                 : launch_score<1, 5, 4, 2, 4, true, false>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
-    const int msmem = kMaxChunks * kTopK * 4;
+    const int msmem = kMaxChunks * kTopK * 4 + (a.sorted ? kTopK * 8 : 0);
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (e != cudaSuccess) return e;
     // programmatic dependent of the score kernel, whose CTAs release it when the work list
@@ -1631,9 +1744,10 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
     mc.numAttrs = 1;
     return cudaLaunchKernelEx(&mc, merge_kernel, static_cast<const uint32_t*>(ws.part_keys),
                               static_cast<const int32_t*>(ws.part_idx), static_cast<const int*>(ws.tok_nchunks),
-                              a.idx_out, a.score_out);
+                              a.idx_out, a.score_out, a.sorted ? 1 : 0);
   }
-  return launch_score<kPrefillQ, 3, 2, 2, 8, false>(tmQ8, tmK, sp, grid, s);
+  return a.sorted ? launch_score<kPrefillQ, 3, 2, 2, 8, false, true>(tmQ8, tmK, sp, grid, s)
+                  : launch_score<kPrefillQ, 3, 2, 2, 8, false, false>(tmQ8, tmK, sp, grid, s);
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s) {

@@ -22,10 +22,11 @@
  *     asynchronous on that stream; the library never synchronises the host,
  *     except dsa_indexer_create / _destroy / _device_error.
  *   - Host-detectable argument errors return a status and launch nothing.
- *     Problems only the device can see (a position outside its sequence's key
- *     cache, malformed offsets, a pipeline wait that ran out) set bits in the
- *     handle's device error word and leave the affected outputs in a defined
- *     padded state; dsa_indexer_device_error() reports and clears them.
+ *     Problems only the device can see set bits in the handle's device error
+ *     word, which dsa_indexer_device_error() reports and clears: a position
+ *     outside its sequence's key cache or malformed offsets (the affected
+ *     output rows are written as padding), or a pipeline wait that ran out (the
+ *     kernel leaves early; rows of unfinished work items are left unwritten).
  *   - A handle may be used from one stream and one host thread at a time (its
  *     workspace is shared by consecutive calls and ordered by that stream, and
  *     dsa_indexer_project forks part of its work onto a stream the handle owns
@@ -139,15 +140,16 @@ dsa_status_t dsa_indexer_key_norm(dsa_indexer_t h, int64_t n, const float* raw_k
  * Query t at position p of sequence b scores keys s = 0..p (inclusive) read
  * from row cache_offsets[b] + s.  Indices are positions inside the sequence.
  * If p + 1 <= top_k the row is exactly [0, 1, ..., p, -1, ...] (scores in
- * the same order, -inf in the padding).  Otherwise the row holds the top_k
- * positions of highest score, in unspecified order (DSA_TOPK_SORTED: score
- * descending, position ascending); among exactly equal scores at the cut any
- * subset may be kept.  The T x S score matrix is never written to memory.
+ * the same order, -inf in the padding), with or without DSA_TOPK_SORTED.
+ * Otherwise the row holds the top_k positions of highest score: in
+ * unspecified order, or with DSA_TOPK_SORTED by score descending, then
+ * position ascending.  Among exactly equal scores at the cut any subset may be
+ * kept.  The T x S score matrix is never written to memory.
  * Flags: DSA_TOPK_SORTED, DSA_TOPK_SPLIT, DSA_TOPK_NO_SPLIT (default: the
  * split-key path when T <= 256).  A query whose position is outside its
  * sequence's cache rows gets an all-padding row and sets
- * DSA_ERR_DEVICE_BOUNDS; malformed offsets set it too and leave the output
- * rows unwritten.  Returns DSA_ERR_WORKSPACE if T or B exceeds max_tokens,
+ * DSA_ERR_DEVICE_BOUNDS; malformed offsets set it too, and then every output
+ * row is padding.  Returns DSA_ERR_WORKSPACE if T or B exceeds max_tokens,
  * and DSA_ERR_UNSUPPORTED for DSA_TOPK_SPLIT with T > 256. */
 dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const float* w,
                               const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
@@ -167,18 +169,27 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
  * the prefill path of dsa_indexer_topk with DSA_TOPK_NO_SPLIT).
  * Limits: T <= 4096 and B <= 4096 (otherwise DSA_ERR_WORKSPACE); the kernels run
  * on at most 8 SMs (the scratch holds 8 per-SM candidate areas), so this is
- * slower than dsa_indexer_topk.  Device-side problems are not reported through
- * a status word (there is no handle): affected rows are padded as documented
- * for dsa_indexer_topk.
- * The first call on a device looks up the scratch's device address with that
- * device current.  All calls on a device share the one scratch array, which keeps
- * the previous call's contents (the call clears what must start at zero): calls
- * whose kernels can overlap on the GPU (e.g. on unordered streams) race and
- * corrupt each other's results; order them on one stream. */
+ * slower than dsa_indexer_topk.  Device-side problems follow dsa_indexer_topk's
+ * rules (bad positions or offsets: padded rows; a wait that ran out: unfinished
+ * rows unwritten) and are recorded in an error word inside the scratch, which
+ * dsa_indexer_noalloc_device_error() reads.
+ * Every call looks up the scratch's device address with the caller's device
+ * current; the first call on a device also loads the library's device code there,
+ * so make that first call before any stream capture.  All calls on a device share
+ * the one scratch array, which keeps the previous call's contents (each call clears
+ * what must start at zero, its error word included): calls whose kernels can
+ * overlap on the GPU (e.g. on unordered streams) race and corrupt each other's
+ * results; order them on one stream. */
 dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const float* w, const int32_t* positions,
                                       const int32_t* q_seq_offsets, int32_t B, const void* key_cache,
                                       int64_t cache_rows, const int64_t* cache_offsets, int32_t* idx_out,
                                       float* score_out, void* stream);
+
+/* Synchronises `stream`, then returns the device-side status recorded by the
+ * last dsa_indexer_topk_noalloc call on the current device: DSA_OK,
+ * DSA_ERR_DEVICE_BOUNDS or DSA_ERR_DEVICE_TIMEOUT (allocates nothing; no
+ * counterpart on the pages, as for dsa_indexer_topk_noalloc). */
+dsa_status_t dsa_indexer_noalloc_device_error(void* stream);
 
 /* Synchronises the device, then returns DSA_OK or the first device-side error
  * recorded since the last call (DSA_ERR_DEVICE_BOUNDS, DSA_ERR_DEVICE_TIMEOUT)

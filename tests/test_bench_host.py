@@ -73,7 +73,8 @@ def test_projection_report_counts_both_gemms_and_the_bytes_once():
 
 
 def test_time_steps_splits_projection_and_topk(monkeypatch):
-    """The events fn records split each step into projection and score + top-k."""
+    """The spans fn records split each step into projection and score + top-k time, summed
+    over the calls of a step (the chunked prefill makes 16 of each)."""
     clock = [0.0]
 
     class FakeEvent:
@@ -86,13 +87,53 @@ def test_time_steps_splits_projection_and_topk(monkeypatch):
         def elapsed_time(self, other):
             return other.t - self.t
 
-    def fn(ev):
-        clock[0] += 2.0          # projections
-        ev[0].record()
-        clock[0] += 5.0          # score + top-k
-        ev[1].record()
+    def advance(dt):
+        def f():
+            clock[0] += dt
+        return f
+
+    def fn(spans):
+        for _ in range(2):
+            spans.span("project", advance(2.0))
+            clock[0] += 0.5          # work between the spans (counted in the step only)
+            spans.span("topk", advance(5.0))
 
     monkeypatch.setattr(bench.torch.cuda, "Event", FakeEvent)
     monkeypatch.setattr(bench.torch.cuda, "synchronize", lambda: None)
     step, topk, proj = bench._time_steps(fn, 3, lambda: None)
-    assert step == [7.0] * 3 and topk == [5.0] * 3 and proj == [2.0] * 3
+    assert step == [15.0] * 3 and topk == [10.0] * 3 and proj == [4.0] * 3
+
+
+def test_prefill_roofline_arithmetic():
+    peaks = dict(bf16_tflops=1650.0, source="measured")
+    r = bench.prefill_roofline(8_590_000_128, 100.0, peaks, None)
+    tflops = 8_590_000_128 * 8192 / 0.1 / 1e12
+    assert abs(r["achieved"] - tflops) < 0.01
+    assert abs(r["frac"] - tflops / 1650.0) < 1e-4
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["gpairs_score_topk"] - 85.9) < 0.001
+
+
+def test_headline_is_the_long_context_chunked_prefill():
+    import workloads as W
+    assert bench.HEADLINE == "chunked_128k"
+    cfg = W.WORKLOADS[bench.HEADLINE]
+    S = cfg["seq_len"]
+    import torch
+    assert W.causal_pairs(torch.arange(S, dtype=torch.int32)) == 8_590_000_128
+    assert set(bench.ALL_WORKLOADS) == set(W.WORKLOADS)
+
+
+def test_stratified_rows_cover_chunk_edges_and_the_topk_boundary():
+    import torch
+
+    import workloads as W
+    S, C = 131072, 8192
+    r = W.stratified_rows(torch.tensor([0, S]), 512, chunk=C, positions=torch.arange(S)).tolist()
+    assert len(r) == 512 and r == sorted(set(r))
+    for c in range(S // C):
+        assert c * C in r and c * C + C - 1 in r
+    for p in (2046, 2047, 2048, 2049):
+        assert p in r
+    # every 1/64 of the range holds a sampled row
+    assert len({t * 64 // S for t in r}) == 64

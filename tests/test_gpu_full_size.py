@@ -91,7 +91,7 @@ def test_prefill_8k_end_to_end(dsa):
     check_rows_valid(idx, pos)
     keys = oracle.project_keys(f64(batch.hidden), f64(wts.W_k), f64(wts.gamma), f64(wts.beta))
     assert_proj_close(f64(cache), keys, "k")
-    rows = sample_rows(T, 40, must=(0, 2046, 2047, 2048, 4095, T - 1))
+    rows = W.stratified_rows(batch.q_seq_offsets, 256, seed=1, positions=batch.positions).numpy()
     oq, _, ow = oracle_project(wts, batch.hidden[rows], batch.q_latent[rows])
     assert_proj_close(f64(q[rows]).reshape(len(rows), -1), oq.reshape(len(rows), -1), "q")
     assert_proj_close(f64(w[rows]), ow, "w")
@@ -99,7 +99,7 @@ def test_prefill_8k_end_to_end(dsa):
                              batch.cache_offsets.numpy())
     recall, _ = check_topk(idx[rows].cpu().numpy(), sc[rows].cpu().numpy(), rows, batch.positions.numpy()[rows],
                            I, A)
-    print(f"prefill_8k sampled end-to-end recall {recall:.6f}")
+    print(f"prefill_8k end to end: {len(rows)} stratified rows against the oracle, recall {recall:.6f}")
 
 
 def test_prefill_2x32k_heavy(dsa):
@@ -117,7 +117,19 @@ def test_prefill_2x32k_heavy(dsa):
     torch.cuda.synchronize()
     assert ix.device_error() == dsa.DSA_OK
     check_rows_valid(idx, pos)
-    rows = sample_rows(T, 24, must=(0, 2047, 2048, 32767, 32768, 32768 + 2048, T - 1))
+    strat = W.stratified_rows(batch.q_seq_offsets, 128, seed=2, positions=batch.positions).numpy()
+    # and 128 rows whose selection holds heavy-hitter keys (the x4 rows)
+    seq_all = oracle.sequence_of(batch.q_seq_offsets.numpy(), T)
+    heavy_pos = torch.zeros(int(batch.cache_offsets[-1]), dtype=torch.bool, device="cuda")
+    heavy_pos[_cuda(heavy)] = True
+    base = _cuda(batch.cache_offsets[torch.as_tensor(seq_all)]).unsqueeze(1)
+    sel_rows = (idx.to(torch.int64) + base).clamp(min=0)
+    has_heavy = (heavy_pos[sel_rows] & (idx >= 0)).any(1).cpu().numpy()
+    cand = np.setdiff1d(np.nonzero(has_heavy)[0], strat)
+    rng = np.random.default_rng(3)
+    hh = rng.choice(cand, size=min(128, len(cand)), replace=False)
+    rows = np.unique(np.concatenate([strat, hh]))
+    assert len(hh) == 128, "at least 128 queries select heavy-hitter keys"
     oq, ok_, ow = oracle_project(wts, batch.hidden[rows], batch.q_latent[rows])
     # projections of the sampled tokens (their key rows, before the heavy-hitter scaling)
     kr = f64(cache[_cuda(torch.as_tensor(rows))])
@@ -131,7 +143,8 @@ def test_prefill_2x32k_heavy(dsa):
                              batch.cache_offsets.numpy())
     recall, _ = check_topk(idx[rows].cpu().numpy(), sc[rows].cpu().numpy(), rows, batch.positions.numpy()[rows],
                            I, A)
-    print(f"prefill_2x32k_heavy sampled recall {recall:.6f}")
+    print(f"prefill_2x32k_heavy: {len(rows)} rows ({len(hh)} selecting heavy hitters) against the oracle, "
+          f"recall {recall:.6f}")
 
 
 def test_decode_64(dsa):
@@ -173,7 +186,7 @@ def test_decode_64(dsa):
     assert_proj_close(f64(q).reshape(B, -1), oq.reshape(B, -1), "q")
     assert_proj_close(f64(w), ow, "w")
     assert_proj_close(f64(cache[_cuda(torch.as_tensor(last))]), ok_, "new k")
-    rows = np.array([0, 5, 17, 31, 42, 63])
+    rows = np.arange(B)
     I, A = [], []
     for b in rows:   # one sequence's cache at a time (the whole cache in float64 would be ~5 GB)
         lo, hi = int(coff[b]), int(coff[b + 1])
@@ -182,7 +195,7 @@ def test_decode_64(dsa):
         I += Ib
         A += Ab
     recall, _ = check_topk(idx[rows].cpu().numpy(), sc[rows].cpu().numpy(), rows, positions.numpy()[rows], I, A)
-    print(f"decode_64 sampled recall {recall:.6f}")
+    print(f"decode_64: all {B} rows against the oracle, recall {recall:.6f}")
 
 
 def test_chunked_128k(dsa):
@@ -202,16 +215,20 @@ def test_chunked_128k(dsa):
         torch.cuda.synchronize()
         assert ix.device_error() == dsa.DSA_OK
         check_rows_valid(idx, pos)
-        if c in (0, 7, S // C - 1):
-            rows = sample_rows(C, 4, must=(C - 1,))
-            keep[c] = (batch, rows, q[rows].cpu(), w[rows].cpu(), idx[rows].cpu(), sc[rows].cpu())
+        rows = W.stratified_rows(torch.tensor([0, C]), 32, seed=100 + c, positions=batch.positions).numpy()
+        keep[c] = (batch, rows, q[rows].cpu(), w[rows].cpu(), idx[rows].cpu(), sc[rows].cpu())
+    keys = f64(cache)
+    n_rows, recalls = 0, []
     for c, (batch, rows, qs, ws, ids, scs) in keep.items():
+        assert 0 in rows and C - 1 in rows and len(rows) >= 32
         oq, ok_, ow = oracle_project(wts, batch.hidden[rows], batch.q_latent[rows])
         assert_proj_close(f64(qs).reshape(len(rows), -1), oq.reshape(len(rows), -1), f"chunk {c} q")
         assert_proj_close(f64(ws), ow, f"chunk {c} w")
         assert_proj_close(f64(cache[_cuda(torch.as_tensor(c * C + rows))]), ok_, f"chunk {c} k")
         pos_rows = batch.positions.numpy()[rows]
-        _, _, I, A = oracle_rows(f64(qs), f64(ws), pos_rows, np.zeros(len(rows)), f64(cache),
-                                 np.array([0, S]))
+        _, _, I, A = oracle_rows(f64(qs), f64(ws), pos_rows, np.zeros(len(rows)), keys, np.array([0, S]))
         recall, _ = check_topk(ids.numpy(), scs.numpy(), c * C + rows, pos_rows, I, A)
-        print(f"chunked_128k chunk {c} sampled recall {recall:.6f}")
+        n_rows += len(rows)
+        recalls.append(recall)
+    print(f"chunked_128k: {n_rows} rows (every chunk, its first and last included) against the oracle, "
+          f"recall min {min(recalls):.6f} mean {np.mean(recalls):.6f}")

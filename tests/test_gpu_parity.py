@@ -8,7 +8,7 @@ import torch
 
 import oracle
 import workloads as W
-from _parity import (assert_proj_close, check_topk, f64, oracle_project, oracle_topk_rows)
+from _parity import (assert_proj_close, check_sorted, check_topk, f64, oracle_project, oracle_topk_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -187,6 +187,54 @@ def test_topk_without_scores(dsa):
     a = np.sort(idx.cpu().numpy(), axis=1)
     b = np.sort(ref_idx.cpu().numpy(), axis=1)
     assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("flags", [1, 1 | 2, 1 | 4])
+def test_topk_sorted_rows(dsa, flags):
+    # DSA_TOPK_SORTED on the prefill path (default / NO_SPLIT) and on the split-key path, with
+    # queries whose prefix is shorter and longer than 2,048; with and without score output
+    if flags & 2:
+        lens = [5000, 9000, 40000, 2048, 2049, 130]
+        B = len(lens)
+        q, keys, w = W.make_scoring_inputs(21, B, sum(lens))
+        positions = torch.tensor([n - 1 for n in lens], dtype=torch.int32)
+        qoff = torch.arange(B + 1, dtype=torch.int32)
+    else:
+        lens = [3000, 37, 2600]
+        B = len(lens)
+        q, keys, w = W.make_scoring_inputs(22, sum(lens), sum(lens))
+        positions = torch.cat([torch.arange(n, dtype=torch.int32) for n in lens])
+        qoff = _offsets(lens, torch.int32)
+    wts = W.make_weights(9, hidden_dim=128, q_latent_dim=64)
+    ix = _indexer(dsa, wts)
+    coff = _offsets(lens, torch.int64)
+    gi, gs = _run_topk(dsa, ix, q, w, positions, qoff, keys, coff, flags)
+    T = gi.shape[0]
+    rows = np.arange(T) if T <= 64 else np.unique(np.concatenate([np.arange(0, T, 11), [2046, 2047, 2048, T - 1]]))
+    _, _, I, A = _oracle_rows(q, w, positions, qoff, keys, coff, rows)
+    check_topk(gi[rows], gs[rows], rows, positions.numpy()[rows], I, A)
+    open_pairs = check_sorted(gi[rows], gs[rows], rows, positions.numpy()[rows], I, A)
+    # without scores the order is the same (the sort key is the kernel's own score)
+    idx2, _ = ix.topk(_cuda(q), _cuda(w), _cuda(positions), _cuda(qoff), _cuda(keys), _cuda(coff),
+                      return_scores=False, flags=flags)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx2.cpu().numpy(), gi)
+    print(f"sorted rows flags={flags}: {len(rows)} rows, {open_pairs} neighbour pairs inside the band")
+
+
+def test_malformed_offsets_pad_every_row(dsa):
+    wts = W.make_weights(10, hidden_dim=128, q_latent_dim=64)
+    ix = _indexer(dsa, wts)
+    T = 200
+    q, keys, w = W.make_scoring_inputs(23, T, T)
+    positions = torch.arange(T, dtype=torch.int32)
+    qoff = torch.tensor([0, 150, 100, T], dtype=torch.int32)    # not monotone
+    coff = torch.tensor([0, 100, 150, T], dtype=torch.int64)
+    for flags in (0, 2):
+        idx, sc = ix.topk(_cuda(q), _cuda(w), _cuda(positions), _cuda(qoff), _cuda(keys), _cuda(coff), flags=flags)
+        torch.cuda.synchronize()
+        assert ix.device_error() == dsa.DSA_ERR_DEVICE_BOUNDS
+        assert bool((idx == -1).all()) and bool(torch.isneginf(sc).all())
 
 
 # ------------------------------------------------------------------------------------------ end to end

@@ -7,6 +7,11 @@ scratch in the library's static device memory, so this test checks that two
 calls in a row -- the second reusing the scratch the first left behind --
 return what the handle-based entry point returns for the same inputs.
 
+The rows are also checked against the CPU oracle (sampled rows, the parity
+rule of the other tests), and the cases reach the limits that size the
+static scratch: 4,096 queries in 4,096 sequences, and 4,096 queries of one
+sequence whose prefixes all exceed 2,048 keys.
+
 This file is collected last on purpose: a failure here leaves every other
 test already run.  It passes both alone in a fresh process and after the
 rest of the suite."""
@@ -17,7 +22,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
+from _parity import check_topk, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -37,7 +44,8 @@ def _p(t):
 
 
 def _case(seed, lens, starts=None):
-    """Score + top-k inputs for sequences of `lens` query tokens (on the GPU)."""
+    """Score + top-k inputs for sequences of `lens` query tokens (on the GPU); sequence b
+    holds starts[b] + lens[b] key rows and its queries sit at positions starts[b] ..."""
     starts = starts or [0] * len(lens)
     T = sum(lens)
     rows = [s + n for s, n in zip(starts, lens)]
@@ -48,7 +56,8 @@ def _case(seed, lens, starts=None):
     coff = torch.zeros(len(lens) + 1, dtype=torch.int64)
     coff[1:] = torch.cumsum(torch.tensor(rows), 0)
     c = lambda t: t.to("cuda").contiguous()  # noqa: E731
-    return dict(T=T, B=len(lens), q=c(q), w=c(w), pos=c(positions), qoff=c(qoff), keys=c(keys), coff=c(coff))
+    return dict(T=T, B=len(lens), q=c(q), w=c(w), pos=c(positions), qoff=c(qoff), keys=c(keys), coff=c(coff),
+                host=dict(q=q, w=w, pos=positions, qoff=qoff, keys=keys, coff=coff))
 
 
 def _with_handle(lib, x):
@@ -106,14 +115,67 @@ def _same_selection(a_idx, a_sc, b_idx, b_sc):
                 assert m[i] == s
 
 
+def _against_oracle(x, idx, sc, rows):
+    """Sampled rows of a no-alloc result against the CPU oracle (same rule as the other tests)."""
+    h = x["host"]
+    _, _, I, A = oracle.topk(f64(h["q"]), f64(h["w"]), h["pos"].numpy(), h["qoff"].numpy(), f64(h["keys"]),
+                             h["coff"].numpy(), 2048, rows=rows, keep_scores=True)
+    recall, _ = check_topk(idx[rows], sc[rows], rows, h["pos"].numpy()[rows], I, A)
+    return recall
+
+
+def _rows(x, n, seed):
+    rng = np.random.default_rng(seed)
+    T = x["T"]
+    return np.unique(np.concatenate([rng.choice(T, size=min(n, T), replace=False), [0, T - 1]]))
+
+
 def test_no_alloc_matches_handle_entry_on_two_calls_in_a_row(lib):
     first = _case(41, [3000])                              # one sequence, long and short prefixes
     second = _case(42, [700, 2600, 1, 45], [0, 100, 0, 5])  # ragged batch, offset positions
-    for x in (first, second):
+    for k, x in enumerate((first, second)):
         ref_idx, ref_sc = _with_handle(lib, x)
         got_idx, got_sc = _no_alloc(lib, x)
         assert not np.any(got_idx == -7)   # every output slot was written
         _same_selection(ref_idx, ref_sc, got_idx, got_sc)
+        recall = _against_oracle(x, got_idx, got_sc, _rows(x, 300, k))
+        print(f"no-alloc call {k}: recall against the oracle {recall:.6f}")
+    assert lib.dsa_indexer_noalloc_device_error(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+
+
+def test_no_alloc_at_the_limits_of_its_scratch(lib):
+    # 4,096 sequences of one query each (the work list's owner bases then live in the scratch,
+    # not in shared memory): 64 of them with prefixes of 2,049..2,600 keys, the rest short
+    rng = np.random.default_rng(7)
+    starts = rng.integers(0, 12, 4096)
+    long_ = rng.choice(4096, 64, replace=False)
+    starts[long_] = rng.integers(2048, 2600, 64)
+    many = _case(44, [1] * 4096, [int(v) for v in starts])
+    # 4,096 queries of one sequence, at positions 3,000..7,095: every prefix is long, so the
+    # streaming selection runs for every item of the longest work list the scratch holds
+    deep = _case(45, [4096], [3000])
+    for k, (x, rows) in enumerate(((many, np.unique(np.concatenate([long_, np.arange(0, 4096, 97)]))),
+                                   (deep, _rows(deep, 120, 9)))):
+        ref_idx, ref_sc = _with_handle(lib, x)
+        got_idx, got_sc = _no_alloc(lib, x)
+        assert not np.any(got_idx == -7)
+        _same_selection(ref_idx, ref_sc, got_idx, got_sc)
+        recall = _against_oracle(x, got_idx, got_sc, rows)
+        print(f"no-alloc limit case {k}: recall against the oracle {recall:.6f}")
+    assert lib.dsa_indexer_noalloc_device_error(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+
+
+def test_no_alloc_pads_rows_and_reports_malformed_offsets(lib):
+    x = _case(46, [100, 50, 50])
+    x["qoff"] = torch.tensor([0, 150, 100, 200], dtype=torch.int32, device="cuda")   # not monotone
+    idx, sc = _no_alloc(lib, x)
+    assert np.all(idx == -1) and np.all(np.isneginf(sc))
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.dsa_indexer_noalloc_device_error(stream) == 7   # DSA_ERR_DEVICE_BOUNDS
+    # the next call starts from a clear error word
+    y = _case(47, [300])
+    _no_alloc(lib, y)
+    assert lib.dsa_indexer_noalloc_device_error(stream) == 0
 
 
 def test_no_alloc_rejects_sizes_beyond_its_scratch(lib):

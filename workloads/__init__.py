@@ -24,4 +24,5 @@ from .generate import (  # noqa: F401
     heavy_hitter_rows,
     causal_pairs,
     make_scoring_inputs,
+    stratified_rows,
 )

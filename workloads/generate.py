@@ -176,3 +176,39 @@ def make_scoring_inputs(seed: int, n_queries: int, n_keys: int, n_heads: int = 3
 def causal_pairs(positions: torch.Tensor) -> int:
     """Number of (query, key) pairs a causal pass scores: sum over queries of pos + 1."""
     return int(positions.to(torch.int64).sum()) + int(positions.numel())
+
+
+def stratified_rows(q_seq_offsets, n: int, seed: int = 0, chunk: int | None = None,
+                    positions=None) -> "torch.Tensor":
+    """Query rows (global token indices) that sample a workload for checking or timing.
+
+    Always included: the first and last token of every sequence, the first and last
+    token of every `chunk`-token chunk (when given), and the tokens at positions
+    2,046..2,049 (where a prefix reaches the 2,048 kept tokens), when present.  The
+    rest, up to n rows, is one seeded draw per equal stratum of the token range, so
+    that every part of the prefix-length range is represented.  Sorted, unique."""
+    offs = [int(v) for v in torch.as_tensor(q_seq_offsets).tolist()]
+    T = offs[-1]
+    must = set()
+    for b in range(len(offs) - 1):
+        if offs[b + 1] > offs[b]:
+            must.update((offs[b], offs[b + 1] - 1))
+    if chunk:
+        for c0 in range(0, T, chunk):
+            must.update((c0, min(c0 + chunk, T) - 1))
+    if positions is not None:
+        pos = torch.as_tensor(positions).to(torch.int64)
+        hit = torch.nonzero((pos >= 2046) & (pos <= 2049)).flatten().tolist()
+        must.update(hit)
+    must = sorted(t for t in must if 0 <= t < T)
+    rest = max(0, min(n, T) - len(must))
+    g = _gen(seed, 21)
+    picked = set(must)
+    if rest:
+        edges = torch.linspace(0, T, rest + 1).round().to(torch.int64).tolist()
+        for i in range(rest):
+            lo, hi = edges[i], max(edges[i + 1], edges[i] + 1)
+            picked.add(int(torch.randint(lo, min(hi, T), (1,), generator=g)))
+    while len(picked) < min(n, T):   # a draw that hit an included row: draw again
+        picked.add(int(torch.randint(0, T, (1,), generator=g)))
+    return torch.tensor(sorted(picked), dtype=torch.int64)
