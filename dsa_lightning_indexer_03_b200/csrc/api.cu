@@ -160,7 +160,8 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
        h->alloc(&ws.tok_nchunks, size_t(T)) &&
        h->alloc(&ws.cand, size_t(ws.cand_slots) * kPrefillQ * kCandStride) &&
        h->alloc(&ws.part_keys, size_t(ws.part_tokens) * kMaxChunks * kTopK) &&
-       h->alloc(&ws.part_idx, size_t(ws.part_tokens) * kMaxChunks * kTopK) && h->alloc(&ws.err, 4);
+       h->alloc(&ws.part_idx, size_t(ws.part_tokens) * kMaxChunks * kTopK) &&
+       h->alloc(&ws.part_hist, size_t(ws.part_tokens) * 2048) && h->alloc(&ws.err, 4);
   if (!ok) {
     delete h;
     return DSA_ERR_OOM;
@@ -173,6 +174,8 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
   }
   cudaStream_t s = nullptr;
   cudaError_t e = cudaMemset(ws.err, 0, sizeof(int));
+  // the merge of the split-key path clears the counts it used; they start at zero
+  if (e == cudaSuccess) e = cudaMemset(ws.part_hist, 0, size_t(ws.part_tokens) * 2048 * sizeof(uint32_t));
   // tensor-core layouts: W_q^T [4096, QL]; [W_k | W_w]^T [160, HD]
   if (e == cudaSuccess) e = launch_transpose_bf16(static_cast<const __nv_bfloat16*>(W_q), QL, H * D, h->WqT, 0, s);
   if (e == cudaSuccess) e = launch_transpose_bf16(static_cast<const __nv_bfloat16*>(W_k), HD, D, h->WkwT, 0, s);
@@ -315,6 +318,23 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
   a.sorted = (flags & DSA_TOPK_SORTED) != 0;
   a.timeout_ns = timeout_ns();
   if (launch_topk(a, h->ws, tmQ1, tmQ8, tmK, h->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_indexer_topk_reuse(dsa_indexer_t h, int64_t n_draft, const int32_t* anchor_rows, int64_t n_src,
+                                    const int32_t* src_idx, const float* src_score, int32_t* idx_out,
+                                    float* score_out, void* stream) {
+  if (!h || n_draft < 0 || n_src < 0) return DSA_ERR_INVALID_ARG;
+  if (n_draft == 0) return DSA_OK;
+  if (n_draft > (int64_t(1) << 30) || n_src > (int64_t(1) << 30)) return DSA_ERR_INVALID_ARG;
+  if (!anchor_rows || !src_idx || !idx_out || n_src == 0) return DSA_ERR_INVALID_ARG;
+  if ((score_out != nullptr) != (src_score != nullptr)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(src_idx) || !aligned16(idx_out) || (src_score && !aligned16(src_score)) ||
+      (score_out && !aligned16(score_out)) || (reinterpret_cast<uintptr_t>(anchor_rows) & 3))
+    return DSA_ERR_INVALID_ARG;
+  if (launch_reuse_rows(static_cast<int>(n_draft), anchor_rows, static_cast<int>(n_src), src_idx, src_score, idx_out,
+                        score_out, h->ws.err, h->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return DSA_ERR_CUDA;
   return DSA_OK;
 }

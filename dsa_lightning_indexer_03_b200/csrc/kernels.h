@@ -75,6 +75,7 @@ struct TopkWorkspace {
   int cand_slots;    // CTA slots (x kPrefillQ queries each)
   uint32_t* part_keys;
   int32_t* part_idx;
+  uint32_t* part_hist;  // [part_tokens][2048] bin counts of the partial lists; zero between calls
   int part_tokens;
   int* err;
 };
@@ -97,6 +98,11 @@ struct TopkArgs {
 
 cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtensorMap& tmQ1, const CUtensorMap& tmQ8,
                         const CUtensorMap& tmK, int num_sms, cudaStream_t s);
+
+// dst rows d = 0..n-1 := src row anchor[d] (indices, and scores when both score pointers are
+// given; an anchor outside [0, n_src) gives a padding row and sets kErrBounds)
+cudaError_t launch_reuse_rows(int n, const int32_t* anchor, int n_src, const int32_t* src_idx, const float* src_score,
+                              int32_t* dst_idx, float* dst_score, int* err, int num_sms, cudaStream_t s);
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s);
 

@@ -122,6 +122,7 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const
   ws.cand_slots = kStaticCtas;
   ws.part_keys = nullptr;
   ws.part_idx = nullptr;
+  ws.part_hist = nullptr;
   ws.part_tokens = 0;
 
   TopkArgs a{};

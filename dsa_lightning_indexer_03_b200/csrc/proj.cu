@@ -12,7 +12,10 @@
 // Kernel shape: one 128-row output tile per CTA; warp 0 issues TMA loads of
 // 64-wide K slices of A and B into a STAGES-deep ring (128-byte swizzle),
 // warp 1 issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM accumulator,
-// warps 2..5 drain TMEM (tcgen05.ld 32x32b) in the epilogue.
+// warps 2..5 drain TMEM (tcgen05.ld 32x32b) in the epilogue.  The k|w GEMM
+// (proj_kw_cluster_kernel) splits its 7,168-deep contraction over a cluster of
+// CTAs that reduce their partial tiles through distributed shared memory before
+// the LayerNorm epilogue, so that every token count keeps many SMs streaming.
 
 #include "kernels.h"
 
@@ -246,6 +249,254 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ---------------------------------------------------------------- k|w projection, split over a cluster
+// The k|w GEMM is bound by reading `hidden` (14,336 bytes per token): one CTA per 128-token
+// tile streams the whole 7,168-wide contraction through one SM.  Here a cluster of CS CTAs
+// shares each 128-token tile: CTA r accumulates k-blocks [r*nk/CS, (r+1)*nk/CS) in its TMEM,
+// stores its partial [128 x 160] fp32 tile in its shared memory, and after a cluster barrier
+// reduces 128/CS of the tile's rows over all CS partials through distributed shared memory
+// (ld.shared::cluster), then applies the key LayerNorm, the bf16 cast and the key-cache
+// scatter to those rows and stores their head weights.  Each row is handled by CS threads
+// (128/CS key columns and 32/CS weight columns each); the LayerNorm's sums over the row are
+// shuffles inside those CS lanes.
+constexpr int kPartStride = 164;   // floats per row of the partial tile (conflict-free float4 stores)
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+template <int CS, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    proj_kw_cluster_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                           ProjParams p) {
+  constexpr int BN = 160;
+  constexpr int kRows = kBM / CS;        // rows of the tile this CTA finishes
+  constexpr int kKeyCols = 128 / CS;     // key columns per thread
+  constexpr int kWCols = 32 / CS;        // weight columns per thread
+  static_assert(CS == 2 || CS == 4 || CS == 8, "cluster of 2, 4 or 8");
+  static_assert(kBM * kPartStride * 4 <= STAGES * ProjSmem<BN, STAGES>::kStageBytes, "partial fits the ring");
+  using L = ProjSmem<BN, STAGES>;
+  constexpr uint32_t kTmemCols = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * kABytes;
+  float* part = reinterpret_cast<float*>(smem);   // [kBM][kPartStride], over the ring once it is drained
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  float* s_gamma = reinterpret_cast<float*>(smem + L::kGammaOff);
+  float* s_beta = s_gamma + 128;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int m0 = blockIdx.y * kBM;
+  const int nk_all = p.K / kBK;
+  const int kb0 = static_cast<int>(rank) * nk_all / CS, kb1 = (static_cast<int>(rank) + 1) * nk_all / CS;
+  const int nk = kb1 - kb0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x >= 64) {
+    const int i = threadIdx.x - 64;
+    s_gamma[i] = p.kw.gamma[i];
+    s_beta[i] = p.kw.beta[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const WaitCtl wc{p.err, abort_flag, p.timeout_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES && !mbar_wait(&empty[s], ((i / STAGES) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(&full[s], L::kStageBytes);
+        tma_load_2d(sA + s * kABytes, &tmA, &full[s], (kb0 + i) * kBK, m0);
+        tma_load_2d(sB + s * L::kBBytes, &tmB, &full[s], (kb0 + i) * kBK, 0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        for (int i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+          drain_wait(&full[i % STAGES], (i / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, BN);
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&full[s], (i / STAGES) & 1, wc)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * kABytes);
+        const uint32_t b = smem_u32(sB + s * L::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          umma_bf16(tmem, umma_desc_sw128(a + kk * 32), umma_desc_sw128(b + kk * 32), idesc, (i | kk) != 0);
+        umma_commit(&empty[s]);
+      }
+      umma_commit(acc_full);
+      umma_commit(mma_done);
+      drain_wait(mma_done, 0);
+    }
+  } else {
+    // this CTA's partial tile: TMEM lane = row, into shared memory (the ring is free: every
+    // load issued was consumed by an MMA, and acc_full follows every MMA)
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0, wc));
+    tc_fence_after();
+    float4* prow = reinterpret_cast<float4*>(part + row * kPartStride);
+    if (ok && nk > 0) {
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32cols(tbase + c * 32, r);
+        tmem_ld_wait(r);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          prow[c * 8 + v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                        __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+      }
+    } else {
+      for (int v = 0; v < BN / 4; ++v) prow[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  __syncwarp();
+  cluster_sync_all();   // every partial of the cluster is in place
+  if (warp >= 2) {
+    const int e = threadIdx.x - 64;
+    const int rl = e / CS, t = e % CS;                 // row of this CTA's share, thread within the row
+    const int trow = static_cast<int>(rank) * kRows + rl;  // row inside the tile
+    float xk[kKeyCols], xw[kWCols];
+#pragma unroll
+    for (int i = 0; i < kKeyCols; ++i) xk[i] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kWCols; ++i) xw[i] = 0.f;
+    const uint32_t base = smem_u32(part + trow * kPartStride);
+#pragma unroll 1
+    for (int src = 0; src < CS; ++src) {
+      const uint32_t rb = map_shared_rank(base, static_cast<uint32_t>(src));
+#pragma unroll
+      for (int v = 0; v < kKeyCols / 4; ++v) {
+        const float4 f = ld_dsmem_f4(rb + (t * kKeyCols + 4 * v) * 4);
+        xk[4 * v] += f.x;
+        xk[4 * v + 1] += f.y;
+        xk[4 * v + 2] += f.z;
+        xk[4 * v + 3] += f.w;
+      }
+#pragma unroll
+      for (int v = 0; v < kWCols / 4; ++v) {
+        const float4 f = ld_dsmem_f4(rb + (128 + t * kWCols + 4 * v) * 4);
+        xw[4 * v] += f.x;
+        xw[4 * v + 1] += f.y;
+        xw[4 * v + 2] += f.z;
+        xw[4 * v + 3] += f.w;
+      }
+    }
+    // LayerNorm over the 128 key columns of the row, spread over its CS threads
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < kKeyCols; ++i) sum += xk[i];
+#pragma unroll
+    for (int o = 1; o < CS; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float mean = sum * (1.0f / 128.0f);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < kKeyCols; ++i) {
+      const float d = xk[i] - mean;
+      ss = fmaf(d, d, ss);
+    }
+#pragma unroll
+    for (int o = 1; o < CS; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rstd = rsqrtf(ss * (1.0f / 128.0f) + p.kw.eps);
+    const int tok = m0 + trow;
+    if (tok < p.M) {
+      const int pos = p.kw.positions[tok];
+      int lo = 0, hi = p.kw.B - 1;   // sequence of the token: the last b with q_seq_offsets[b] <= tok
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.kw.q_seq_offsets[mid] <= tok) lo = mid;
+        else hi = mid - 1;
+      }
+      const int64_t cb = p.kw.cache_offsets[lo];
+      const int64_t len = p.kw.cache_offsets[lo + 1] - cb;
+      if (pos >= 0 && pos < len && cb >= 0 && cb + pos < p.kw.cache_rows) {
+        uint4* d4 = reinterpret_cast<uint4*>(p.kw.key_cache + static_cast<size_t>(cb + pos) * kHeadDim +
+                                             t * kKeyCols);
+#pragma unroll
+        for (int v = 0; v < kKeyCols / 8; ++v) {
+          float y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int d = t * kKeyCols + 8 * v + i;
+            y[i] = fmaf((xk[8 * v + i] - mean) * rstd, s_gamma[d], s_beta[d]);
+          }
+          uint4 pk;
+          pk.x = pack_bf16x2(y[0], y[1]);
+          pk.y = pack_bf16x2(y[2], y[3]);
+          pk.z = pack_bf16x2(y[4], y[5]);
+          pk.w = pack_bf16x2(y[6], y[7]);
+          d4[v] = pk;
+        }
+      } else if (t == 0) {
+        atomicOr(p.err, kErrBounds);
+      }
+      float4* w4 = reinterpret_cast<float4*>(p.kw.w_out + static_cast<size_t>(tok) * kHeads + t * kWCols);
+#pragma unroll
+      for (int v = 0; v < kWCols / 4; ++v)
+        w4[v] = make_float4(xw[4 * v], xw[4 * v + 1], xw[4 * v + 2], xw[4 * v + 3]);
+    }
+  }
+  __syncwarp();
+  cluster_sync_all();   // no CTA leaves while a peer may still read its partial
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // ---------------------------------------------------------------- key LayerNorm on its own
 __global__ void __launch_bounds__(256) key_norm_kernel(int64_t n, const float* __restrict__ raw,
                                                        __nv_bfloat16* __restrict__ out, const float* __restrict__ gamma,
@@ -313,6 +564,27 @@ cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M,
   return launch_proj<256, 4, EPI_Q>(tmA, tmB, p, N / 256, s);
 }
 
+template <int CS>
+cudaError_t launch_kw_cluster(const CUtensorMap& tmA, const CUtensorMap& tmB, const ProjParams& p, cudaStream_t s) {
+  using L = ProjSmem<160, 5>;
+  auto kern = proj_kw_cluster_kernel<CS, 5>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, (p.M + kBM - 1) / kBM);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p);
+}
+
 cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K, const ProjKwEpilogue& e,
                            cudaStream_t s) {
   ProjParams p{};
@@ -321,6 +593,11 @@ cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K
   p.kw = e;
   p.err = e.err;
   p.timeout_ns = e.timeout_ns;
+  const int nk = K / kBK;
+  // the contraction is split over a cluster of CTAs when it is long enough to share
+  if (nk >= 8) return launch_kw_cluster<8>(tmA, tmB, p, s);
+  if (nk >= 4) return launch_kw_cluster<4>(tmA, tmB, p, s);
+  if (nk >= 2) return launch_kw_cluster<2>(tmA, tmB, p, s);
   return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
 }
 

@@ -51,6 +51,7 @@ struct ScoreParams {
   uint2* cand;                  // [slots][QMAX][kCandStride] (key, position) pairs
   uint32_t* part_keys;          // [T][kMaxChunks][kTopK]
   int32_t* part_idx;
+  uint32_t* part_hist;          // [T][kBins1]: first-level bin counts of each query's partial lists
   int* err;
   uint64_t timeout_ns;
 };
@@ -88,7 +89,6 @@ __device__ __forceinline__ uint32_t group_suffix_excl(uint32_t v, int tid, uint3
 }
 
 constexpr int kHistBins = 1024;   // histogram bins of one selection round
-constexpr int kRankList = 256;    // boundary-bin keys ranked directly (merge path)
 
 // k-th largest of the order-preserving keys that a group of NT threads visits, among those
 // inside the window [lo, hi] (1 <= k <= their number; keys outside are ignored).
@@ -160,238 +160,11 @@ __device__ uint32_t kth_largest(const uint32_t* keys, int n, int k, uint32_t lo,
 }
 
 // ------------------------------------------------------------------------------------------
-// Selection over dense lists (the merge of the split-key path's partial lists).
-
-
-// A dense list of n slots (n a multiple of 4); slots with position < 0 are empty.
-struct FlatCands {
-  const uint32_t* k;
-  const int32_t* i;
-  template <bool kKeys, bool kIdx>
-  __device__ __forceinline__ uint32_t load4(int s0, uint4& kv, int4& iv) const {
-    if (kKeys) kv = *reinterpret_cast<const uint4*>(k + s0);
-    if (kIdx) {
-      iv = *reinterpret_cast<const int4*>(i + s0);
-      return (iv.x >= 0 ? 1u : 0u) | (iv.y >= 0 ? 2u : 0u) | (iv.z >= 0 ? 4u : 0u) | (iv.w >= 0 ? 8u : 0u);
-    }
-    return 0xFu;
-  }
-};
-
 __device__ __forceinline__ uint32_t u4_get(const uint4& v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 __device__ __forceinline__ int i4_get(const int4& v, int j) {
   return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
-}
-
-// Emits the top k of the occupied slots: every key > kth and the first (k - n_above)
-// keys equal to kth.  sink(slot, key, pos) is called once per kept entry with a
-// distinct slot in [0, k).  ctr[0..1] are shared counters zeroed beforehand.
-template <int NT, class View, class Sink>
-__device__ void emit_view(const View& v, const uint32_t* skeys, int n, int k, uint32_t kth, int n_above, int* ctr,
-                          int tid, Sink sink) {
-  const int lane = tid & 31;
-  const int ties = k - n_above;
-  const uint32_t lt = lanemask_lt();
-#pragma unroll 12
-  for (int base = 0; base < n / 4; base += NT) {
-    const int g = base + tid;
-    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
-    int4 ii = make_int4(-1, -1, -1, -1);
-    uint32_t m = 0;
-    if (g < n / 4) {
-      kk = reinterpret_cast<const uint4*>(skeys)[g];
-      uint4 dummy;
-      m = v.template load4<false, true>(4 * g, dummy, ii);
-    }
-    uint32_t bg[4], be[4];
-    int tg = 0, te = 0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t key = u4_get(kk, j);
-      const bool valid = (m >> j) & 1u;
-      bg[j] = __ballot_sync(0xffffffffu, valid && key > kth);
-      be[j] = __ballot_sync(0xffffffffu, valid && key == kth);
-      tg += __popc(bg[j]);
-      te += __popc(be[j]);
-    }
-    if (tg | te) {
-      int b0 = 0, b1 = 0;
-      if (lane == 0) {
-        if (tg) b0 = atomicAdd(&ctr[0], tg);
-        if (te) b1 = atomicAdd(&ctr[1], te);
-      }
-      b0 = __shfl_sync(0xffffffffu, b0, 0);
-      b1 = __shfl_sync(0xffffffffu, b1, 0);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if ((bg[j] >> lane) & 1u) sink(b0 + __popc(bg[j] & lt), u4_get(kk, j), i4_get(ii, j));
-        if ((be[j] >> lane) & 1u) {
-          const int r = b1 + __popc(be[j] & lt);
-          if (r < ties) sink(n_above + r, u4_get(kk, j), i4_get(ii, j));
-        }
-        b0 += __popc(bg[j]);
-        b1 += __popc(be[j]);
-      }
-    }
-  }
-}
-
-// Histogram bin of a key for the selection's first round: bins of equal width in
-// score value between the smallest and largest candidate (a monotone map from the
-// ordered keys, so the bin holding the k-th largest can be found exactly).
-__device__ __forceinline__ int value_bin(uint32_t key, float lo_f, float scale) {
-  const float x = (ordered_to_float(key) - lo_f) * scale;
-  int b = __float2int_rz(x);
-  b = b < 0 ? 0 : (b > kHistBins - 1 ? kHistBins - 1 : b);
-  return x == x ? b : 0;
-}
-
-// Selects the top kTopK occupied slots of a view (which holds at least kTopK):
-// 1. stage the keys of the n slots into shared memory (empty slots as 0) and find
-//    the occupied keys' range;
-// 2. histogram the keys into kHistBins bins of equal width in score value and
-//    locate the bin that holds the kTopK-th largest;
-// 3. gather that bin's keys into `list` and find the exact kTopK-th largest K* there
-//    by counting ranks (a crowded bin falls back to kth_largest over all keys);
-// 4. emit every key > K* and the first kTopK - n_above keys equal to K* through
-//    sink(slot, key, pos).  Returns K*.
-template <int NT, class View, class Sink>
-__device__ uint32_t select_topk(const View& v, int n, uint32_t* skeys, uint32_t* hist, uint32_t* list, int list_cap,
-                                uint32_t* scratch, int* sh, int* ctr, int tid, int bar, Sink sink) {
-  const int lane = tid & 31, wid = tid >> 5;
-  // 1. stage + range; the histogram is cleared and the counters zeroed in the same phase
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll 12
-  for (int g = tid; g < n / 4; g += NT) {
-    uint4 k;
-    int4 unused;
-    const uint32_t m = v.template load4<true, false>(4 * g, k, unused);
-    reinterpret_cast<uint4*>(skeys)[g] = k;
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      if ((m >> j) & 1u) {
-        lo = min(lo, u4_get(k, j));
-        hi = max(hi, u4_get(k, j));
-      }
-  }
-  for (int i = tid; i < kHistBins; i += NT) hist[i] = 0;
-  if (tid == 0) {
-    ctr[0] = 0;
-    ctr[1] = 0;
-    sh[5] = 0;
-  }
-  lo = __reduce_min_sync(0xffffffffu, lo);
-  hi = __reduce_max_sync(0xffffffffu, hi);
-  if (lane == 0) {
-    scratch[wid] = lo;
-    scratch[NT / 32 + wid] = hi;
-  }
-  named_bar_sync(bar, NT);
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) {
-    lo = min(lo, scratch[w]);
-    hi = max(hi, scratch[NT / 32 + w]);
-  }
-  const float lo_f = ordered_to_float(lo), hi_f = ordered_to_float(hi);
-  float scale = (hi_f > lo_f) ? static_cast<float>(kHistBins) / (hi_f - lo_f) : 0.f;
-  if (!(scale < 3.0e38f)) scale = 0.f;
-
-  // 2. value-binned histogram of the occupied keys (empty slots hold key 0)
-#pragma unroll 4
-  for (int g = tid; g < n / 4; g += NT) {
-    const uint4 k = reinterpret_cast<const uint4*>(skeys)[g];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t key = u4_get(k, j);
-      if (key >= lo && key != 0u) atomicAdd(&hist[value_bin(key, lo_f, scale)], 1u);
-    }
-  }
-  named_bar_sync(bar, NT);
-  int above;
-  int bstar;
-  {
-    constexpr int kBPT = kHistBins / NT;
-    const int b0 = tid * kBPT;
-    uint32_t c[kBPT];
-    uint32_t s = 0;
-#pragma unroll
-    for (int i = 0; i < kBPT; ++i) {
-      c[i] = hist[b0 + i];
-      s += c[i];
-    }
-    // suffix sum over threads: warp shuffles + one exchange of warp totals
-    uint32_t x = s;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, x, off);
-      if (lane + off < 32) x += y;
-    }
-    if (lane == 0) scratch[2 * (NT / 32) + wid] = x;
-    named_bar_sync(bar, NT);
-    uint32_t above_t = x - s;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w)
-      if (w > wid) above_t += scratch[2 * (NT / 32) + w];
-    const uint32_t need = kTopK;
-    if (above_t < need && need <= above_t + s) {
-      uint32_t cum = above_t;
-#pragma unroll
-      for (int i = kBPT - 1; i >= 0; --i) {
-        if (cum + c[i] >= need) {
-          sh[0] = b0 + i;
-          sh[1] = static_cast<int>(cum);
-          break;
-        }
-        cum += c[i];
-      }
-    }
-    named_bar_sync(bar, NT);
-    bstar = sh[0];
-    above = sh[1];
-  }
-  // 3. gather the boundary bin and rank its keys
-#pragma unroll 4
-  for (int g = tid; g < n / 4; g += NT) {
-    const uint4 k = reinterpret_cast<const uint4*>(skeys)[g];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t key = u4_get(k, j);
-      if (key >= lo && key != 0u && value_bin(key, lo_f, scale) == bstar) {
-        const int o = atomicAdd(&sh[5], 1);
-        if (o < list_cap) list[o] = key;
-      }
-    }
-  }
-  named_bar_sync(bar, NT);
-  const int m = sh[5];
-  const int need2 = kTopK - above;
-  uint32_t kth;
-  int n_above;
-  if (m <= list_cap) {
-    for (int e = tid; e < m; e += NT) {
-      const uint32_t xk = list[e];
-      int greater = 0, equal = 0;
-      for (int j = 0; j < m; ++j) {
-        const uint32_t y = list[j];
-        greater += y > xk;
-        equal += y == xk;
-      }
-      if (greater < need2 && need2 <= greater + equal) {  // every finder writes the same values
-        sh[2] = static_cast<int>(xk);
-        sh[3] = greater;
-      }
-    }
-    named_bar_sync(bar, NT);
-    kth = static_cast<uint32_t>(sh[2]);
-    n_above = above + sh[3];
-  } else {
-    kth = kth_largest<NT>(skeys, n, kTopK, lo, hi, hist, scratch, sh, tid, bar, &n_above);
-  }
-  // 4. emit
-  emit_view<NT>(v, skeys, n, kTopK, kth, n_above, ctr, tid, sink);
-  return kth;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1356,7 +1129,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
         } else {
           uint32_t* pk = p.part_keys + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
           int32_t* pi = p.part_idx + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
+          uint32_t* const h = st.hist[jj];
           if (n_valid <= kTopK) {
+            // every candidate is kept; h already counts exactly these
             if (gtid == 0) st.ctr[0] = 0;
             named_bar_sync(bar, NTG);
             collect<NTG>(v, st.ctr, gtid, [&](int rank, uint2 x) {
@@ -1368,10 +1143,20 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
               pi[e] = -1;
             }
           } else {
-            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+            // h is cleared before the first kept entry is emitted and counts the kept entries
+            resolve_topk<NTG>(v, h, true, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
               pk[s2] = key;
               pi[s2] = static_cast<int>(pos);
+              count_key(h, key >> kBinShift);
             });
+          }
+          named_bar_sync(bar, NTG);
+          // add the partial list's bin counts to the query's totals, which the merge reads
+          uint32_t* const qh = p.part_hist + static_cast<size_t>(t) * kBins1;
+          for (int i = gtid; i < kBins1 / 2; i += NTG) {
+            const uint32_t wd = h[i];
+            if (wd & 0xFFFFu) atomicAdd(&qh[2 * i], wd & 0xFFFFu);
+            if (wd >> 16) atomicAdd(&qh[2 * i + 1], wd >> 16);
           }
         }
         named_bar_sync(bar, NTG);
@@ -1390,47 +1175,169 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
 
 
 // ------------------------------------------------------------------------------------------
-// merge of the split-key path: top-k over the kMaxChunks partial lists of one query
+// merge of the split-key path: top-k over the partial lists of one query's key chunks.
+// Every chunk added the first-level bin counts of the entries it kept to the query's
+// histogram, so the bin b1 holding the kTopK-th largest entry is found from those counts
+// alone.  One pass over the partial lists then writes every entry above b1 to its output
+// slot and gathers b1's entries into shared memory, where the exact kTopK-th largest key K*
+// is found (kth_largest) and the entries of b1 above K*, then the first ties, are written.
+// The histogram is cleared after use, ready for the next call.
 constexpr int kMergeThreads = 1024;
+constexpr int kMergeList = 8192;   // boundary-bin entries held in shared memory
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __restrict__ part_keys,
                                                               const int32_t* __restrict__ part_idx,
                                                               const int* __restrict__ tok_nchunks,
+                                                              uint32_t* __restrict__ part_hist,
                                                               int32_t* __restrict__ idx_out,
                                                               float* __restrict__ score_out, int sorted) {
-  extern __shared__ uint32_t mkeys[];  // [kMaxChunks * kTopK], then (sorted) kTopK staged pairs
+  extern __shared__ uint32_t msm[];   // list keys [kMergeList], list positions [kMergeList], stage [kTopK] pairs
+  uint32_t* const lkeys = msm;
+  int32_t* const lidx = reinterpret_cast<int32_t*>(msm + kMergeList);
+  uint2* const stage = reinterpret_cast<uint2*>(msm + 2 * kMergeList);
   __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t mlist[kRankList];
-  __shared__ uint32_t scratch[3 * (kMergeThreads / 32)];
+  __shared__ uint32_t scratch[kMergeThreads / 32];
   __shared__ int sh[8];
-  __shared__ int ctr[2];
-  // launched as a programmatic dependent of the score kernel: the partial lists are read
-  // only after that grid completed and its writes are visible
+  __shared__ int ctr[4];
+  // launched as a programmatic dependent of the score kernel: the partial lists and the
+  // counts are read only after that grid completed and its writes are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int t = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int nch = tok_nchunks[t];
-  if (nch < 2) return;
+  if (nch < 2) return;   // written by the score kernel itself; no counts were added
   const int n = nch * kTopK;
-  FlatCands v;
-  v.k = part_keys + static_cast<size_t>(t) * kMaxChunks * kTopK;
-  v.i = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
-  int32_t* oi = idx_out + static_cast<size_t>(t) * kTopK;
-  float* os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
-  if (sorted) {
-    uint2* const stage = reinterpret_cast<uint2*>(mkeys + kMaxChunks * kTopK);
-    select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
-                               [&](int slot, uint32_t key, int pos) {
-      stage[slot] = make_uint2(key, static_cast<uint32_t>(pos));
-    });
-    named_bar_sync(1, kMergeThreads);
-    sort_stage_and_emit<kMergeThreads>(stage, threadIdx.x, 1, oi, os);
-    return;
+  const uint32_t* const keys = part_keys + static_cast<size_t>(t) * kMaxChunks * kTopK;
+  const int32_t* const pos = part_idx + static_cast<size_t>(t) * kMaxChunks * kTopK;
+  uint32_t* const qh = part_hist + static_cast<size_t>(t) * kBins1;
+  int32_t* const oi = idx_out + static_cast<size_t>(t) * kTopK;
+  float* const os = score_out ? score_out + static_cast<size_t>(t) * kTopK : nullptr;
+  auto out = [&](int slot, uint32_t key, int p) {
+    if (sorted) {
+      stage[slot] = make_uint2(key, static_cast<uint32_t>(p));
+    } else {
+      __stcs(oi + slot, p);
+      if (os) __stcs(os + slot, ordered_to_float(key));
+    }
+  };
+  if (tid < 4) ctr[tid] = 0;
+  // 1. boundary bin from the counts (two bins per thread), then clear them
+  constexpr int kBPT = kBins1 / kMergeThreads;
+  static_assert(kBPT == 2, "two bins per thread");
+  uint32_t c[kBPT];
+  uint32_t csum = 0;
+#pragma unroll
+  for (int i = 0; i < kBPT; ++i) {
+    c[i] = qh[kBPT * tid + i];
+    csum += c[i];
   }
-  select_topk<kMergeThreads>(v, n, mkeys, hist, mlist, kRankList, scratch, sh, ctr, threadIdx.x, 1,
-                             [&](int slot, uint32_t key, int pos) {
-    __stcs(oi + slot, pos);
-    if (os) __stcs(os + slot, ordered_to_float(key));
-  });
+#pragma unroll
+  for (int i = 0; i < kBPT; ++i) qh[kBPT * tid + i] = 0u;
+  if (tid == 0) {
+    sh[0] = 0;
+    sh[1] = 0;
+  }
+  const uint32_t above_t = group_suffix_excl<kMergeThreads>(csum, tid, scratch, 1);
+  if (above_t < static_cast<uint32_t>(kTopK) && static_cast<uint32_t>(kTopK) <= above_t + csum) {
+    uint32_t cum = above_t;
+#pragma unroll
+    for (int i = kBPT - 1; i >= 0; --i) {
+      if (cum + c[i] >= static_cast<uint32_t>(kTopK)) {
+        sh[0] = kBPT * tid + i;
+        sh[1] = static_cast<int>(cum);
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  named_bar_sync(1, kMergeThreads);
+  const uint32_t b1 = static_cast<uint32_t>(min(max(sh[0], 0), kBins1 - 1));
+  const int above = min(max(sh[1], 0), kTopK);
+  // 2. one pass: entries above b1 to their slots, b1's entries to the list
+  const uint32_t lt = lanemask_lt();
+#pragma unroll 2
+  for (int base = 0; base < n / 4; base += kMergeThreads) {
+    const int g = base + tid;
+    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
+    int4 ii = make_int4(-1, -1, -1, -1);
+    if (g < n / 4) {
+      kk = reinterpret_cast<const uint4*>(keys)[g];
+      ii = reinterpret_cast<const int4*>(pos)[g];
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = u4_get(kk, j);
+      const int p = i4_get(ii, j);
+      const uint32_t bin = key >> kBinShift;
+      const bool up = p >= 0 && bin > b1, mid = p >= 0 && bin == b1;
+      const uint32_t bu = __ballot_sync(0xffffffffu, up), bm = __ballot_sync(0xffffffffu, mid);
+      if (bu | bm) {
+        int ou = 0, om = 0;
+        if (lane == 0) {
+          if (bu) ou = atomicAdd(&ctr[0], __popc(bu));
+          if (bm) om = atomicAdd(&ctr[1], __popc(bm));
+        }
+        ou = __shfl_sync(0xffffffffu, ou, 0) + __popc(bu & lt);
+        om = __shfl_sync(0xffffffffu, om, 0) + __popc(bm & lt);
+        if (up && ou < kTopK) out(ou, key, p);
+        if (mid && om < kMergeList) {
+          lkeys[om] = key;
+          lidx[om] = p;
+        }
+      }
+    }
+  }
+  named_bar_sync(1, kMergeThreads);
+  const int m = ctr[1];
+  const int need = kTopK - above;
+  const uint32_t lo = b1 << kBinShift, hi = lo + ((1u << kBinShift) - 1u);
+  int n_above;
+  uint32_t kth;
+  // 3. the exact need-th largest key of the boundary bin
+  if (m <= kMergeList) {
+    kth = kth_largest<kMergeThreads>(lkeys, m, need, lo, hi, hist, scratch, sh, tid, 1, &n_above);
+  } else {
+    // more boundary entries than the list holds: visit them in the partial lists
+    auto visit = [&](auto f) {
+      for (int e = tid; e < n; e += kMergeThreads)
+        if (pos[e] >= 0 && (keys[e] >> kBinShift) == b1) f(keys[e]);
+    };
+    kth = kth_window<kMergeThreads>(visit, need, lo, hi, hist, scratch, sh, tid, 1, &n_above);
+  }
+  // 4. the boundary bin's entries above K*, then the first ties
+  const int ties = need - n_above;
+  auto fin = [&](uint32_t key, int p, bool ok) {
+    const bool gt = ok && key > kth, eq = ok && key == kth;
+    const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    if (bg | be) {
+      int og = 0, oe = 0;
+      if (lane == 0) {
+        if (bg) og = atomicAdd(&ctr[2], __popc(bg));
+        if (be) oe = atomicAdd(&ctr[3], __popc(be));
+      }
+      og = __shfl_sync(0xffffffffu, og, 0) + __popc(bg & lt);
+      oe = __shfl_sync(0xffffffffu, oe, 0) + __popc(be & lt);
+      if (gt && above + og < kTopK) out(above + og, key, p);
+      if (eq && oe < ties) out(above + n_above + oe, key, p);
+    }
+  };
+  if (m <= kMergeList) {
+    for (int base = 0; base < m; base += kMergeThreads) {
+      const int e = base + tid;
+      const bool ok = e < m;
+      fin(ok ? lkeys[e] : 0u, ok ? lidx[e] : -1, ok);
+    }
+  } else {
+    for (int base = 0; base < n; base += kMergeThreads) {
+      const int e = base + tid;
+      const bool ok = e < n && pos[e] >= 0 && (keys[e] >> kBinShift) == b1;
+      fin(ok ? keys[e] : 0u, ok ? pos[e] : -1, ok);
+    }
+  }
+  if (sorted) {
+    named_bar_sync(1, kMergeThreads);
+    sort_stage_and_emit<kMergeThreads>(stage, tid, 1, oi, os);
+  }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -1720,6 +1627,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.cand = ws.cand;
   sp.part_keys = ws.part_keys;
   sp.part_idx = ws.part_idx;
+  sp.part_hist = ws.part_hist;
   sp.err = ws.err;
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
@@ -1727,7 +1635,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
     e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true>(tmQ1, tmK, sp, grid, s)
                  : launch_score<1, 5, 4, 2, 4, true, false>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
-    const int msmem = kMaxChunks * kTopK * 4 + (a.sorted ? kTopK * 8 : 0);
+    const int msmem = 2 * kMergeList * 4 + kTopK * 8;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (e != cudaSuccess) return e;
     // programmatic dependent of the score kernel, whose CTAs release it when the work list
@@ -1744,7 +1652,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
     mc.numAttrs = 1;
     return cudaLaunchKernelEx(&mc, merge_kernel, static_cast<const uint32_t*>(ws.part_keys),
                               static_cast<const int32_t*>(ws.part_idx), static_cast<const int*>(ws.tok_nchunks),
-                              a.idx_out, a.score_out, a.sorted ? 1 : 0);
+                              ws.part_hist, a.idx_out, a.score_out, a.sorted ? 1 : 0);
   }
   return a.sorted ? launch_score<kPrefillQ, 3, 2, 2, 8, false, true>(tmQ8, tmK, sp, grid, s)
                   : launch_score<kPrefillQ, 3, 2, 2, 8, false, false>(tmQ8, tmK, sp, grid, s);

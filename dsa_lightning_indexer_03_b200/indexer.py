@@ -146,6 +146,27 @@ class Indexer:
               "dsa_indexer_topk")
         return idx_out, score_out
 
+    def topk_reuse(self, anchor_rows, src_idx, src_score=None, idx_out=None, score_out=None, stream=None):
+        """Rows of earlier dsa_indexer_topk results reused by speculative draft tokens: row d of
+        the output is row anchor_rows[d] of src_idx (and src_score, when given)."""
+        dev = self.device
+        _need(anchor_rows, "anchor_rows", torch.int32, dev)
+        _need(src_idx, "src_idx", torch.int32, dev)
+        n = anchor_rows.numel()
+        if idx_out is None:
+            idx_out = torch.empty((n, self.top_k), dtype=torch.int32, device=dev)
+        _need(idx_out, "idx_out", torch.int32, dev)
+        if src_score is not None:
+            _need(src_score, "src_score", torch.float32, dev)
+            if score_out is None:
+                score_out = torch.empty((n, self.top_k), dtype=torch.float32, device=dev)
+        if score_out is not None:
+            _need(score_out, "score_out", torch.float32, dev)
+        check(self._lib.dsa_indexer_topk_reuse(self._h, n, _ptr(anchor_rows), src_idx.shape[0], _ptr(src_idx),
+                                               _ptr(src_score), _ptr(idx_out), _ptr(score_out), _stream(stream)),
+              "dsa_indexer_topk_reuse")
+        return idx_out, score_out
+
     def device_error(self) -> int:
         """Synchronises and returns (then clears) the handle's device error status."""
         with torch.cuda.device(self.device):

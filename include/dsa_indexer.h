@@ -157,6 +157,23 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
                               int32_t* idx_out,
                               float* score_out, uint32_t flags, void* stream);
 
+/* Index reuse across speculative draft steps ('MTP' row of the page "Kimi K3.1
+ * Pro vs GLM-5": GLM-5.2 reuses the first step's top-k indices in its later
+ * draft steps).  Draft token d takes the selection of its anchor: row
+ * anchor_rows[d] of a [n_src, top_k] result of dsa_indexer_topk (the first
+ * step's queries), copied bit for bit.
+ *   anchor_rows int32 [n_draft], each in [0, n_src)
+ *   src_idx     int32 [n_src, top_k];  src_score fp32 [n_src, top_k] or NULL
+ *   idx_out     int32 [n_draft, top_k]; score_out fp32 [n_draft, top_k] or NULL
+ *               (scores are copied when both score pointers are given; giving
+ *               only one of them is DSA_ERR_INVALID_ARG)
+ * The output must not overlap the source.  An anchor outside [0, n_src) gives
+ * an all-padding row (-1, -inf) and sets DSA_ERR_DEVICE_BOUNDS.  Asynchronous on
+ * `stream`; n_draft = 0 is a no-op. */
+dsa_status_t dsa_indexer_topk_reuse(dsa_indexer_t h, int64_t n_draft, const int32_t* anchor_rows, int64_t n_src,
+                                    const int32_t* src_idx, const float* src_score, int32_t* idx_out,
+                                    float* score_out, void* stream);
+
 /* Allocation-free score + top-k (no counterpart on the pages; it exists for the
  * library's users).  Some callers cannot let a library allocate device memory:
  * a framework whose memory pool already holds the device's whole budget, or a

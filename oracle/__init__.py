@@ -21,4 +21,5 @@ from .indexer_oracle import (  # noqa: F401
     sequence_of,
     topk,
     sort_selected,
+    reuse_topk,
 )

@@ -238,3 +238,26 @@ def sort_selected(idx_row, I):
     out = -np.ones_like(idx_row)
     out[: len(valid)] = valid[order]
     return out
+
+
+# --------------------------------------------------------------------------
+# index reuse across speculative draft steps
+# --------------------------------------------------------------------------
+
+def reuse_topk(idx, score, anchor_rows):
+    """Selections of speculative draft tokens ('MTP' row, page "Kimi K3.1 Pro vs GLM-5":
+    GLM-5.2 reuses the first step's top-k indices in its later draft steps).
+
+    idx [n_src, top_k] and score [n_src, top_k] are the first step's selections; draft
+    token d takes row anchor_rows[d] unchanged.  An anchor outside [0, n_src) has no
+    selection to reuse: its row is all padding (-1, -inf)."""
+    idx = np.asarray(idx)
+    score = np.asarray(score, np.float64)
+    a = np.asarray(anchor_rows, np.int64)
+    n_src, k = idx.shape
+    ok = (a >= 0) & (a < n_src)
+    out_i = np.full((len(a), k), -1, dtype=np.int64)
+    out_s = np.full((len(a), k), -np.inf)
+    out_i[ok] = idx[a[ok]]
+    out_s[ok] = score[a[ok]]
+    return out_i, out_s

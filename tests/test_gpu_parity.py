@@ -237,6 +237,35 @@ def test_malformed_offsets_pad_every_row(dsa):
         assert bool((idx == -1).all()) and bool(torch.isneginf(sc).all())
 
 
+def test_topk_reuse_for_draft_steps(dsa):
+    # first step: 6 anchor queries selected by dsa_indexer_topk (checked against the oracle);
+    # draft steps: 14 tokens that reuse an anchor's row, one with an anchor out of range
+    wts = W.make_weights(12, hidden_dim=128, q_latent_dim=64)
+    ix = _indexer(dsa, wts)
+    lens = [3000, 5000, 2100, 700, 9000, 4096]
+    B = len(lens)
+    q, keys, w = W.make_scoring_inputs(24, B, sum(lens))
+    positions = torch.tensor([n - 1 for n in lens], dtype=torch.int32)
+    qoff = torch.arange(B + 1, dtype=torch.int32)
+    coff = _offsets(lens, torch.int64)
+    gi, gs = _run_topk(dsa, ix, q, w, positions, qoff, keys, coff, 0)
+    _, _, I, A = _oracle_rows(q, w, positions, qoff, keys, coff, np.arange(B))
+    check_topk(gi, gs, np.arange(B), positions.numpy(), I, A)
+    anchors = torch.tensor([0, 0, 0, 1, 1, 2, 3, 3, 3, 3, 4, 5, 5, 5], dtype=torch.int32)
+    anchors[7] = 17   # no such anchor: a padding row and a bounds report
+    src_i, src_s = _cuda(torch.from_numpy(gi)), _cuda(torch.from_numpy(gs))
+    ri, rs = ix.topk_reuse(_cuda(anchors), src_i, src_s)
+    ri2, rs2 = ix.topk_reuse(_cuda(anchors), src_i)
+    torch.cuda.synchronize()
+    assert ix.device_error() == dsa.DSA_ERR_DEVICE_BOUNDS
+    oi, os_ = oracle.reuse_topk(gi, gs, anchors.numpy())
+    assert np.array_equal(ri.cpu().numpy(), oi) and np.array_equal(ri2.cpu().numpy(), oi)
+    assert rs2 is None
+    got_s = rs.cpu().numpy()
+    assert np.array_equal(got_s[np.isfinite(os_)], os_[np.isfinite(os_)])
+    assert np.all(np.isneginf(got_s[~np.isfinite(os_)]))
+
+
 # ------------------------------------------------------------------------------------------ end to end
 
 def test_end_to_end_prefill_3k(dsa):

@@ -371,3 +371,31 @@ def test_planted_layernorm_mistakes_fail_the_closed_form():
     assert np.allclose(oracle.layer_norm(x, ones, zeros, 1e-6), ref, atol=1e-10)
     assert not np.allclose(unbiased, ref, atol=1e-6)
     assert not np.allclose(rms, ref, atol=1e-6)
+
+
+# ---------------------------------------------------------------- index reuse (draft steps)
+
+def test_reuse_gives_every_draft_its_anchors_bruteforce_selection():
+    # the first step's selection of each anchor comes from brute-force scoring of its prefix;
+    # a draft token at a later position reuses exactly that row ('MTP' row, GLM-5.2)
+    rng = np.random.default_rng(31)
+    H, D, k, T = 2, 4, 3, 9
+    q = rng.standard_normal((T, H, D))
+    w = rng.standard_normal((T, H))
+    keys = rng.standard_normal((T, D))
+    pos = np.arange(T)
+    anchors = np.array([4, 6])
+    idx, sc = oracle.topk(q[anchors], w[anchors], pos[anchors], np.array([0, 2]), keys, np.array([0, T]),
+                          top_k=k)
+    drafts = np.array([0, 0, 0, 1, 1, 5])      # anchor row of each draft token; 5 has none
+    ri, rs = oracle.reuse_topk(idx, sc, drafts)
+    for d, a in enumerate(drafts):
+        if a >= len(anchors):
+            assert np.all(ri[d] == -1) and np.all(np.isneginf(rs[d]))
+            continue
+        p = pos[anchors[a]]
+        best = max(itertools.combinations(range(p + 1), k),
+                   key=lambda c: (sorted((sum(w[anchors[a], h] * max(0.0, q[anchors[a], h] @ keys[s])
+                                              for h in range(H)) for s in c)), [-s for s in c]))
+        assert set(ri[d].tolist()) == set(best)
+        assert ri[d].max() <= p      # causal for the anchor, hence for every later draft position
