@@ -22,4 +22,9 @@ from .indexer_oracle import (  # noqa: F401
     topk,
     sort_selected,
     reuse_topk,
+    E4M3_MAX,
+    e4m3_round,
+    quantize_fp8,
+    fp8_index_scores,
+    topk_fp8,
 )

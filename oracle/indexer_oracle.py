@@ -261,3 +261,91 @@ def reuse_topk(idx, score, anchor_rows):
     out_i[ok] = idx[a[ok]]
     out_s[ok] = score[a[ok]]
     return out_i, out_s
+
+
+# --------------------------------------------------------------------------
+# FP8 indexer-key cache ('FP8 -> FP4 training' row, page "Kimi K3.1 Pro vs GLM-5":
+# vLLM and SGLang cache the indexer keys in FP8 by default)
+# --------------------------------------------------------------------------
+
+E4M3_MAX = 448.0   # largest finite e4m3 value: 2^8 * 1.75
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Round values to the nearest FP8 e4m3 value (1 sign, 4 exponent bits with bias 7,
+    3 mantissa bits; no infinities), ties to even, saturating at +-448.  A value in
+    [2^(e-1), 2^e) with e - 1 >= -6 is rounded to a multiple of 2^(e-4); below 2^-6 the
+    spacing stays 2^-9 (subnormals).  Returned as float64 (exact)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.zeros_like(x)
+    nz = (x != 0.0) & np.isfinite(x)
+    v = x[nz]
+    _, e = np.frexp(v)                   # |v| in [2^(e-1), 2^e)
+    q = np.maximum(e - 4, -9)
+    y = np.ldexp(np.rint(np.ldexp(v, -q)), q)
+    out[nz] = np.clip(y, -E4M3_MAX, E4M3_MAX)
+    return out
+
+
+def quantize_fp8(v, axis: int = -1):
+    """FP8 e4m3 codes and fp32 scale of rows of float32-representable values, one scale per
+    row (the pages fix no granularity; one scale per 128-value key row, and per head of a
+    query, is the reading taken):
+        amax  = max |v| over the row
+        scale = fp32(amax / 448),  inv = fp32(448 / amax)      (both 0 when amax = 0)
+        code  = e4m3(fp32(v * inv))
+    so that code * scale approximates v.  Every operation is a single float32 rounding, as
+    on the device.  Returns (codes as float64 on the e4m3 grid, scale as float64)."""
+    v = np.asarray(v, dtype=np.float32)
+    amax = np.max(np.abs(v), axis=axis, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        scale = np.where(amax > 0, (amax / np.float32(E4M3_MAX)).astype(np.float32), np.float32(0))
+        inv = np.where(amax > 0, (np.float32(E4M3_MAX) / amax).astype(np.float32), np.float32(0))
+    prod = (v * inv).astype(np.float32)
+    codes = e4m3_round(prod.astype(np.float64))
+    return codes, np.squeeze(scale, axis=axis).astype(np.float64)
+
+
+def fp8_index_scores(q8_t, sq_t, w_t, k8, sk):
+    """Scores of one query against FP8 keys: with q_h ~ q8_h * sq_h and k_s ~ k8_s * sk_s
+    (positive scales),
+        I[s] = sum_h w_h * max(0, (q8_h sq_h) . (k8_s sk_s))
+             = sk_s * sum_h (w_h sq_h) * max(0, q8_h . k8_s),
+    and the tolerance scale A[s] = sk_s * sum_h |w_h sq_h| |q8_h . k8_s|."""
+    logits = np.asarray(k8, np.float64) @ np.asarray(q8_t, np.float64).T          # [n, H]
+    wq = np.asarray(w_t, np.float64) * np.asarray(sq_t, np.float64)
+    sk = np.asarray(sk, np.float64)
+    I = sk * (np.maximum(logits, 0.0) @ wq)
+    A = sk * (np.abs(logits) @ np.abs(wq))
+    return I, A
+
+
+def topk_fp8(q8, sq, w, positions, q_seq_offsets, k8, sk, cache_offsets, top_k: int = TOP_K, rows=None,
+             keep_scores: bool = False):
+    """As topk, over FP8 queries q8 [T, H, D] with per-head scales sq [T, H] and FP8 keys
+    k8 [rows, D] with per-row scales sk [rows]."""
+    q8 = np.asarray(q8, np.float64)
+    positions = np.asarray(positions, np.int64)
+    cache_offsets = np.asarray(cache_offsets, np.int64)
+    T = q8.shape[0]
+    seq = sequence_of(q_seq_offsets, T)
+    rows = np.arange(T) if rows is None else np.asarray(rows, np.int64)
+    idx = np.empty((len(rows), top_k), dtype=np.int64)
+    score = np.empty((len(rows), top_k), dtype=np.float64)
+    all_I, all_A = [], []
+    for r, t in enumerate(rows):
+        b = seq[t]
+        p = positions[t]
+        base = cache_offsets[b]
+        if p < 0 or base + p >= cache_offsets[b + 1]:
+            raise ValueError(f"query {t}: position {p} outside its sequence's cache rows")
+        I, A = fp8_index_scores(q8[t], sq[t], w[t], k8[base: base + p + 1], sk[base: base + p + 1])
+        sel = select_topk(I, top_k)
+        idx[r] = sel
+        score[r] = np.where(sel >= 0, I[np.maximum(sel, 0)], -np.inf)
+        if keep_scores:
+            all_I.append(I)
+            all_A.append(A)
+    if keep_scores:
+        return idx, score, all_I, all_A
+    return idx, score

@@ -399,3 +399,81 @@ def test_reuse_gives_every_draft_its_anchors_bruteforce_selection():
                                               for h in range(H)) for s in c)), [-s for s in c]))
         assert set(ri[d].tolist()) == set(best)
         assert ri[d].max() <= p      # causal for the anchor, hence for every later draft position
+
+
+# ---------------------------------------------------------------- FP8 key cache
+
+def test_e4m3_round_matches_torch_conversion_inside_the_range():
+    rng = np.random.default_rng(41)
+    mant = rng.uniform(1.0, 2.0, 100_000)
+    ex = rng.integers(-12, 9, 100_000)
+    x = (np.ldexp(mant, ex) * rng.choice([-1, 1], 100_000)).astype(np.float32).astype(np.float64)
+    x = x[np.abs(x) <= 448.0]
+    want = torch.tensor(x, dtype=torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.e4m3_round(x), want)
+
+
+def test_e4m3_grid_and_ties():
+    # the 126 finite positive codes: 7 subnormals k 2^-9, then (1 + m/8) 2^(e-7)
+    grid = [k * 2.0 ** -9 for k in range(1, 8)] + [(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16)
+                                                      for m in range(8) if not (e == 15 and m == 7)]
+    assert len(grid) == 126 and max(grid) == 448.0
+    g = np.array(grid)
+    assert np.array_equal(oracle.e4m3_round(g), g)
+    # midpoints go to the even mantissa; beyond 448 saturates
+    assert oracle.e4m3_round(np.array([0.59375]))[0] == 0.625       # between 0.5625 (odd) and 0.625
+    assert oracle.e4m3_round(np.array([1.0625]))[0] == 1.0          # between 1.0 (even) and 1.125
+    assert oracle.e4m3_round(np.array([3 * 2.0 ** -10]))[0] == 2.0 ** -8   # subnormal tie to even
+    assert oracle.e4m3_round(np.array([1000.0, -500.0])).tolist() == [448.0, -448.0]
+
+
+def test_quantize_fp8_bounds_and_exact_max():
+    rng = np.random.default_rng(42)
+    v = rng.standard_normal((500, 128)).astype(np.float32)
+    codes, scale = oracle.quantize_fp8(v)
+    assert codes.shape == v.shape and scale.shape == (500,)
+    assert np.all(np.abs(codes) <= 448.0)
+    # the row maximum lands on 448 (up to one float32 rounding of v * inv)
+    am = np.argmax(np.abs(v), axis=1)
+    assert np.all(np.abs(codes[np.arange(500), am]) == 448.0)
+    # relative error of a normal-range value is at most half a mantissa step (2^-4)
+    deq = codes * scale[:, None]
+    big = np.abs(v) >= 2.0 ** -6 * scale[:, None]
+    assert np.all(np.abs(deq - v)[big] <= 2.0 ** -4 * np.abs(v)[big] * (1 + 1e-6))
+    z, zs = oracle.quantize_fp8(np.zeros((2, 8), np.float32))
+    assert np.all(z == 0) and np.all(zs == 0)
+
+
+def test_fp8_scores_equal_scores_of_the_dequantised_operands():
+    # the scale factoring (s_k out of the ReLU, s_q into the head weight) is exact algebra:
+    # compare with index_scores of code * scale
+    rng = np.random.default_rng(43)
+    H, D, n = 4, 16, 50
+    q = rng.standard_normal((H, D)).astype(np.float32)
+    k = rng.standard_normal((n, D)).astype(np.float32)
+    w = rng.standard_normal(H)
+    q8, sq = oracle.quantize_fp8(q)
+    k8, sk = oracle.quantize_fp8(k)
+    I, A = oracle.fp8_index_scores(q8, sq, w, k8, sk)
+    I2, A2 = oracle.index_scores(q8 * sq[:, None], w, k8 * sk[:, None])
+    assert np.allclose(I, I2, rtol=1e-12, atol=1e-12) and np.allclose(A, A2, rtol=1e-12, atol=1e-12)
+    # planted mistake: the key scale left out
+    bad = (np.maximum(k8 @ q8.T, 0.0) @ (w * sq))
+    assert not np.allclose(bad, I2)
+
+
+def test_fp8_selection_tracks_the_bf16_selection():
+    # quantisation moves scores by a few percent of A: the FP8 top-k keeps almost all of the
+    # bf16 top-k on N(0,1) data (the recall the engines accept by caching keys in FP8)
+    rng = np.random.default_rng(44)
+    T, S = 3, 6000
+    q = oracle.bf16_round(rng.standard_normal((T, 32, 128)))
+    k = oracle.bf16_round(rng.standard_normal((S, 128)))
+    w = rng.standard_normal((T, 32))
+    pos = np.array([S - 1, S - 2, 4000])
+    idx_b, _ = oracle.topk(q, w, pos, np.array([0, T]), k, np.array([0, S]))
+    q8, sq = oracle.quantize_fp8(q.astype(np.float32))
+    k8, sk = oracle.quantize_fp8(k.astype(np.float32))
+    idx_f, _ = oracle.topk_fp8(q8, sq, w, pos, np.array([0, T]), k8, sk, np.array([0, S]))
+    for r in range(T):
+        assert len(np.intersect1d(idx_b[r], idx_f[r])) / 2048 > 0.9
