@@ -227,16 +227,18 @@ def projection_report(T, ms, peak_tflops, hbm_gbs):
             "achieved_gbs": round(gbs, 2), "frac_hbm": round(gbs / hbm_gbs, 4)}
 
 
-def prefill_roofline(pairs, topk_ms, peaks, traffic):
+def prefill_roofline(pairs, topk_ms, peaks, traffic, fp8=False):
     """Roofline of the score + top-k over a prefill workload: pairs x 8,192 flop over the
-    summed dsa_indexer_topk time, against the measured burst bf16 peak."""
+    summed dsa_indexer_topk time, against the measured burst bf16 peak (for FP8 operands,
+    that peak times the nominal fp8 / bf16 ratio of 2)."""
     tflops = pairs * FLOP_PER_PAIR / (topk_ms * 1e-3) / 1e12
-    return {"bound": "tensor", "achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": round(tflops / peaks["bf16_tflops"], 4), "traffic": traffic,
+    peak = peaks["bf16_tflops"] * (2 if fp8 else 1)
+    return {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(tflops / peak, 4), "traffic": traffic,
             "kernel": "score_topk (dsa_indexer_topk: prep + score)", "ms_per_launch": None,
             "ms_topk_per_step": round(topk_ms, 4), "gpairs_score_topk": round(pairs / (topk_ms * 1e-3) / 1e9, 3),
-            "peak_source": peaks["source"] + " burst bf16 (" + ("of measured" if peaks["source"] == "measured"
-                                                                  else "of fallback") + ")"}
+            "peak_source": peaks["source"] + " burst bf16" + (" x 2 (fp8)" if fp8 else "") + " (" +
+                           ("of measured" if peaks["source"] == "measured" else "of fallback") + ")"}
 
 
 # ------------------------------------------------------------------------------------------ GPU arm: workloads
@@ -246,7 +248,7 @@ def _make_indexer(d, wts, device, max_tokens):
     return d.Indexer(to(wts.W_q), to(wts.W_k), to(wts.W_w), to(wts.gamma), to(wts.beta), max_tokens=max_tokens)
 
 
-def setup_prefill(d, name, seed_offset, device):
+def setup_prefill(d, name, seed_offset, device, fp8=False):
     """Inputs of a prefill workload, resident on the device.  A prefill job is a list of
     calls ("chunks"): one call for the single-shot prefills, 16 calls of 8,192 queries for
     the chunked long-context prefill, each scoring against the keys of every earlier chunk."""
@@ -286,7 +288,13 @@ def setup_prefill(d, name, seed_offset, device):
               w=torch.empty((T, 32), dtype=torch.float32, device=device),
               idx=torch.empty((T, 2048), dtype=torch.int32, device=device),
               score=torch.empty((T, 2048), dtype=torch.float32, device=device),
-              pairs=W.causal_pairs(positions), weights=wts)
+              pairs=W.causal_pairs(positions), weights=wts, fp8=fp8)
+    if fp8:
+        rows = int(coff[-1])
+        st["cache"] = torch.zeros((rows, 128), dtype=torch.uint8, device=device)
+        st["kscale"] = torch.zeros((rows,), dtype=torch.float32, device=device)
+        st["q"] = torch.empty((T, 32, 128), dtype=torch.uint8, device=device)
+        st["qscale"] = torch.empty((T, 32), dtype=torch.float32, device=device)
     return st
 
 
@@ -294,6 +302,15 @@ def prefill_step(st, spans):
     """One pass of the hot path over the whole workload: per call, the projections (which
     write the call's keys into the cache) and then the score + top-k."""
     ix = st["ix"]
+    if st["fp8"]:
+        for (a0, a1), qoff in zip(st["bounds"], st["qoffs"]):
+            spans.span("project", lambda: ix.project_fp8(
+                st["hidden"][a0:a1], st["q_latent"][a0:a1], st["positions"][a0:a1], qoff, st["cache"], st["kscale"],
+                st["coff"], q_out=st["q"][a0:a1], q_scale=st["qscale"][a0:a1], w_out=st["w"][a0:a1]))
+            spans.span("topk", lambda: ix.topk_fp8(
+                st["q"][a0:a1], st["qscale"][a0:a1], st["w"][a0:a1], st["positions"][a0:a1], qoff, st["cache"],
+                st["kscale"], st["coff"], idx_out=st["idx"][a0:a1], score_out=st["score"][a0:a1]))
+        return
     for (a0, a1), qoff in zip(st["bounds"], st["qoffs"]):
         spans.span("project", lambda: ix.project(st["hidden"][a0:a1], st["q_latent"][a0:a1],
                                                  st["positions"][a0:a1], qoff, st["cache"], st["coff"],
@@ -307,7 +324,7 @@ def prefill_step(st, spans):
                                            score_out=st["score"][a0:a1]))
 
 
-def setup_decode(d, seed_offset, device):
+def setup_decode(d, seed_offset, device, fp8=False):
     cfg = W.WORKLOADS["decode_64"]
     wts = W.make_weights(cfg["weight_seed"])
     lengths = W.decode_lengths(cfg["act_seed"] + seed_offset, cfg["batch"], cfg["L_min"], cfg["L_max"])
@@ -335,13 +352,33 @@ def setup_decode(d, seed_offset, device):
               idx=torch.empty((B, 2048), dtype=torch.int32, device=device),
               score=torch.empty((B, 2048), dtype=torch.float32, device=device),
               total_keys=total, lengths=lengths)
-    # algorithmic bytes of the score + top-k: every cached key once, q/w once, indices+scores out
-    st["bytes"] = total * 128 * 2 + B * (32 * 128 * 2 + 32 * 4) + B * 2048 * (4 + 4)
+    st["fp8"] = fp8
+    if fp8:
+        # the FP8 cache of the same keys: e4m3 codes and one scale per row
+        st["cache"], st["kscale"] = ix.quantize_keys_fp8(cache)
+        del cache
+        st["q"] = torch.empty((B, 32, 128), dtype=torch.uint8, device=device)
+        st["qscale"] = torch.empty((B, 32), dtype=torch.float32, device=device)
+        torch.cuda.synchronize()
+    # algorithmic bytes of the score + top-k: every cached key once (with its scale for FP8),
+    # q (and its head scales) and w once, indices + scores out
+    if fp8:
+        st["bytes"] = total * (128 + 4) + B * (32 * 128 + 32 * 4 + 32 * 4) + B * 2048 * (4 + 4)
+    else:
+        st["bytes"] = total * 128 * 2 + B * (32 * 128 * 2 + 32 * 4) + B * 2048 * (4 + 4)
     return st
 
 
 def decode_step(ds, spans):
     ix = ds["ix"]
+    if ds["fp8"]:
+        spans.span("project", lambda: ix.project_fp8(ds["hidden"], ds["q_latent"], ds["positions"], ds["qoff"],
+                                                     ds["cache"], ds["kscale"], ds["coff"], q_out=ds["q"],
+                                                     q_scale=ds["qscale"], w_out=ds["w"]))
+        spans.span("topk", lambda: ix.topk_fp8(ds["q"], ds["qscale"], ds["w"], ds["positions"], ds["qoff"],
+                                               ds["cache"], ds["kscale"], ds["coff"], idx_out=ds["idx"],
+                                               score_out=ds["score"]))
+        return
     spans.span("project", lambda: ix.project(ds["hidden"], ds["q_latent"], ds["positions"], ds["qoff"], ds["cache"],
                                              ds["coff"], q_out=ds["q"], w_out=ds["w"]))
     spans.span("topk", lambda: ix.topk(ds["q"], ds["w"], ds["positions"], ds["qoff"], ds["cache"], ds["coff"],
@@ -404,8 +441,8 @@ def e2e_prefill(st, steps):
     return statistics.mean(ts), bi, bo
 
 
-def run_prefill(d, name, rank, device, steps, warmup, flush, peaks, mx, clk=None):
-    st = setup_prefill(d, name, rank, device)
+def run_prefill(d, name, rank, device, steps, warmup, flush, peaks, mx, clk=None, fp8=False):
+    st = setup_prefill(d, name, rank, device, fp8)
     fn = lambda spans: prefill_step(st, spans)  # noqa: E731
     _time_steps(fn, warmup, flush)
     torch.cuda.synchronize()
@@ -419,30 +456,32 @@ def run_prefill(d, name, rank, device, steps, warmup, flush, peaks, mx, clk=None
     proj_avg = mx(statistics.mean(proj_ms))
     err = st["ix"].device_error()
     n_calls = len(st["bounds"])
-    rec = {"workload": name, "metric": "indexer score+top-2048 Gpairs/s (prefill)",
+    rec = {"workload": name + ("_fp8" if fp8 else ""), "metric": "indexer score+top-2048 Gpairs/s (prefill)",
            "value": None, "unit": "Gpairs/s", "ms_per_step": round(ms, 4), "causal_pairs": st["pairs"],
            "tokens": st["T"], "calls_per_step": n_calls,
-           "roofline": prefill_roofline(st["pairs"], topk_avg, peaks, _profile_traffic(f"score_topk:{name}")),
+           "roofline": prefill_roofline(st["pairs"], topk_avg, peaks, _profile_traffic(f"score_topk:{name}"), fp8),
            "projections": projection_report(st["T"], proj_avg, peaks["bf16_tflops"], peaks["hbm_gbs"]),
            "device_error": err, "gpu_launches_per_step": n_calls * (LAUNCHES["project"] + LAUNCHES["topk"])}
     rec["roofline"]["ms_per_launch"] = round(topk_avg / n_calls, 4)
     return st, rec, ms
 
 
-def run_decode(d, rank, device, steps, warmup, flush, peaks, mx):
-    ds = setup_decode(d, rank, device)
+def run_decode(d, rank, device, steps, warmup, flush, peaks, mx, fp8=False):
+    ds = setup_decode(d, rank, device, fp8)
     fn = lambda spans: decode_step(ds, spans)  # noqa: E731
     _time_steps(fn, warmup, flush)
     dstep, dtopk, dproj = _time_steps(fn, steps, flush)
     dms = mx(statistics.mean(dtopk))
     dstep_ms = mx(statistics.mean(dstep))
     gbs = ds["bytes"] / (dms * 1e-3) / 1e9
-    rec = {"workload": "decode_64", "metric": "decode GB/s", "value": None, "unit": "GB/s",
+    rec = {"workload": "decode_64" + ("_fp8" if fp8 else ""), "metric": "decode GB/s", "value": None, "unit": "GB/s",
+           "keys_per_s": round(ds["total_keys"] / (dms * 1e-3) / 1e9, 3),
            "ms_score_topk": round(dms, 4), "ms_per_step": round(dstep_ms, 4), "ms_project": round(
                mx(statistics.mean(dproj)), 4),
            "keys_scanned": ds["total_keys"], "algorithmic_bytes": ds["bytes"],
            "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                        "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": _profile_traffic("score_topk:decode_64"),
+                        "frac": round(gbs / peaks["hbm_gbs"], 4),
+                        "traffic": _profile_traffic("score_topk:decode_64" + ("_fp8" if fp8 else "")),
                         "kernel": "score_topk split-key + merge (dsa_indexer_topk)", "ms_per_launch": round(dms, 4),
                         "peak_source": peaks["source"] + " HBM copy"},
            "device_error": ds["ix"].device_error(),
@@ -497,11 +536,19 @@ def gpu_arm(args, rank, world, local_rank, dist):
             del s2
             torch.cuda.empty_cache()
         n = max(args.steps, 100)
-        ds, rec, gbs = run_decode(d, rank, device, n, args.warmup, flush, peaks, mx)
-        rec["value"] = round(gbs * world, 2)
+        for fp8 in (False, True):
+            ds, rec, gbs = run_decode(d, rank, device, n, args.warmup, flush, peaks, mx, fp8)
+            rec["value"] = round(gbs * world, 2)
+            rec["steps"] = n
+            subs[rec["workload"]] = rec
+            del ds
+            torch.cuda.empty_cache()
+        # the FP8 cache on the 8,192-token prefill (FP8 tensor-core scoring)
+        s2, rec, ms2 = run_prefill(d, "prefill_8k", rank, device, n, args.warmup, flush, peaks, mx, fp8=True)
+        rec["value"] = round(whole_job_rate(s2["pairs"], world, ms2) / 1e9, 3)
         rec["steps"] = n
-        subs["decode_64"] = rec
-        del ds
+        subs[rec["workload"]] = rec
+        del s2
         torch.cuda.empty_cache()
 
     launches = head["gpu_launches_per_step"] * args.steps
@@ -795,7 +842,8 @@ def main():
         cb = cpu_baselines(args.workload, all_workloads=not args.headline_only)
         line["cpu_baseline"] = cb[args.workload]
         for name, rec in line.get("workloads", {}).items():
-            rec["cpu_baseline"] = cb.get(name)
+            if name in cb:
+                rec["cpu_baseline"] = cb[name]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

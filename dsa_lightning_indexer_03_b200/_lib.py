@@ -52,6 +52,11 @@ SIGNATURES = {
     "dsa_indexer_key_norm": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp]),
     "dsa_indexer_topk": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _vp, _vp, _u32, _vp]),
     "dsa_indexer_topk_noalloc": (ctypes.c_int, [_i64, _vp, _vp, _vp, _vp, _i32, _vp, _i64, _vp, _vp, _vp, _vp]),
+    "dsa_indexer_project_fp8": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
+                                                _vp, _vp]),
+    "dsa_indexer_quantize_keys_fp8": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp]),
+    "dsa_indexer_topk_fp8": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
+                                             _u32, _vp]),
     "dsa_indexer_topk_reuse": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp]),
     "dsa_indexer_device_error": (ctypes.c_int, [_vp]),
     "dsa_indexer_noalloc_device_error": (ctypes.c_int, [_vp]),

@@ -43,16 +43,17 @@ bool load_encode() {
   return g_encode != nullptr;
 }
 
-// 2-D bf16 tensor [rows, inner] (row-major, row stride inner*2 bytes), 128-byte swizzled
-// boxes of box_inner x box_rows elements.
+// 2-D bf16 (or, with `bytes`, 1-byte FP8) tensor [rows, inner] (row-major, dense rows),
+// 128-byte swizzled boxes of box_inner x box_rows elements.
 bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
-               uint32_t box_rows) {
+               uint32_t box_rows, bool bytes = false) {
   if (!load_encode()) return false;
   cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {inner * (bytes ? 1 : 2)};
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = g_encode(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                        const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -215,29 +216,41 @@ dsa_status_t dsa_indexer_destroy(dsa_indexer_t h) {
   return DSA_OK;
 }
 
-dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
-                                 const int32_t* positions, const int32_t* q_seq_offsets, int32_t B, void* key_cache,
-                                 int64_t cache_rows, const int64_t* cache_offsets, void* q_out, float* w_out,
-                                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of dsa_indexer_project and dsa_indexer_project_fp8: key_cache / q_out are bf16
+// for the former; key8 + key_scale and q8 + q_scale for the latter.
+dsa_status_t project_impl(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
+                          const int32_t* positions, const int32_t* q_seq_offsets, int32_t B, void* key_cache,
+                          float* key_scale, int64_t cache_rows, const int64_t* cache_offsets, void* q_out,
+                          float* q_scale, float* w_out, void* stream, bool fp8) {
   if (!h) return DSA_ERR_INVALID_ARG;
   if (T < 0 || T > (int64_t(1) << 26) || B < 1) return DSA_ERR_INVALID_ARG;
   if (T == 0) return DSA_OK;
   if (!hidden || !q_latent || !positions || !q_seq_offsets || !key_cache || !cache_offsets || !q_out || !w_out)
+    return DSA_ERR_INVALID_ARG;
+  if (fp8 && (!key_scale || !q_scale || (reinterpret_cast<uintptr_t>(key_scale) & 3) ||
+              (reinterpret_cast<uintptr_t>(q_scale) & 3)))
     return DSA_ERR_INVALID_ARG;
   if (!aligned16(hidden) || !aligned16(q_latent) || !aligned16(key_cache) || !aligned16(q_out) ||
       !aligned16(w_out) || (reinterpret_cast<uintptr_t>(positions) & 3) ||
       (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7))
     return DSA_ERR_INVALID_ARG;
   if (cache_rows < 1 || cache_rows > (int64_t(1) << 31) - (int64_t(1) << 20)) return DSA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const dsa_indexer_config_t& c = h->cfg;
+  if (fp8 && c.hidden_dim < 128) return DSA_ERR_UNSUPPORTED;   // the FP8 key epilogue is the split-K one
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tmX, tmQL;
   if (!make_tmap(&tmX, hidden, c.hidden_dim, uint64_t(T), 64, 128) ||
       !make_tmap(&tmQL, q_latent, c.q_latent_dim, uint64_t(T), 64, 128))
     return DSA_ERR_INVALID_ARG;
   ProjKwEpilogue e{};
   e.M = static_cast<int>(T);
-  e.key_cache = static_cast<__nv_bfloat16*>(key_cache);
+  e.key_cache = fp8 ? nullptr : static_cast<__nv_bfloat16*>(key_cache);
+  e.key8 = fp8 ? static_cast<uint8_t*>(key_cache) : nullptr;
+  e.key_scale = fp8 ? key_scale : nullptr;
   e.cache_rows = cache_rows;
   e.w_out = w_out;
   e.positions = positions;
@@ -254,12 +267,106 @@ dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden,
   if (cudaEventRecord(h->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(h->side, h->ev_fork, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
   const cudaError_t ekw = launch_proj_kw(tmX, h->tm_WkwT, c.hidden_dim, e, h->side);
-  const cudaError_t eq = launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
-                                       static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s);
+  const cudaError_t eq =
+      fp8 ? launch_proj_q8(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
+                           static_cast<uint8_t*>(q_out), q_scale, h->ws.err, timeout_ns(), s)
+          : launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
+                          static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s);
   // join even if a launch failed, so that the side stream never runs ahead unordered
   if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess || cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
   if (ekw != cudaSuccess || eq != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+// Shared body of dsa_indexer_topk and dsa_indexer_topk_fp8.
+dsa_status_t topk_impl(dsa_indexer_t h, int64_t T, const void* q, const float* q_scale, const float* w,
+                       const int32_t* positions, const int32_t* q_seq_offsets, int32_t B, const void* key_cache,
+                       const float* key_scale, int64_t cache_rows, const int64_t* cache_offsets, int32_t* idx_out,
+                       float* score_out, uint32_t flags, void* stream, bool fp8) {
+  if (!h) return DSA_ERR_INVALID_ARG;
+  if (T < 0 || B < 1) return DSA_ERR_INVALID_ARG;
+  if ((flags & DSA_TOPK_SPLIT) && (flags & DSA_TOPK_NO_SPLIT)) return DSA_ERR_INVALID_ARG;
+  if (flags & ~(DSA_TOPK_SORTED | DSA_TOPK_SPLIT | DSA_TOPK_NO_SPLIT)) return DSA_ERR_INVALID_ARG;
+  if (T == 0) return DSA_OK;
+  if (T > h->cfg.max_tokens || B > h->cfg.max_tokens) return DSA_ERR_WORKSPACE;
+  if (!q || !w || !positions || !q_seq_offsets || !key_cache || !cache_offsets || !idx_out) return DSA_ERR_INVALID_ARG;
+  if (fp8 && (!q_scale || !key_scale || (reinterpret_cast<uintptr_t>(q_scale) & 3) ||
+              (reinterpret_cast<uintptr_t>(key_scale) & 3)))
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(w) || !aligned16(key_cache) || !aligned16(idx_out) ||
+      (score_out && !aligned16(score_out)) || (reinterpret_cast<uintptr_t>(positions) & 3) ||
+      (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7))
+    return DSA_ERR_INVALID_ARG;
+  if (cache_rows < 1 || cache_rows > (int64_t(1) << 31) - (int64_t(1) << 20)) return DSA_ERR_INVALID_ARG;
+  bool split = (T <= kSplitMaxTokens);
+  if (flags & DSA_TOPK_SPLIT) {
+    if (T > h->ws.part_tokens) return DSA_ERR_UNSUPPORTED;
+    split = true;
+  }
+  if (flags & DSA_TOPK_NO_SPLIT) split = false;
+  if (split && T > h->ws.part_tokens) split = false;
+  // a box row is 128 bytes: 64 bf16 (two boxes per 128-dim row) or 128 FP8 codes (one)
+  const uint32_t bi = fp8 ? 128 : 64;
+  CUtensorMap tmQ1, tmQ8, tmK;
+  if (!make_tmap(&tmQ1, q, kHeadDim, uint64_t(T) * kHeads, bi, kHeads, fp8) ||
+      !make_tmap(&tmQ8, q, kHeadDim, uint64_t(T) * kHeads, bi, kHeads * kPrefillQ, fp8) ||
+      !make_tmap(&tmK, key_cache, kHeadDim, uint64_t(cache_rows), bi, kKeyTile, fp8))
+    return DSA_ERR_INVALID_ARG;
+  TopkArgs a{};
+  a.T = static_cast<int>(T);
+  a.B = B;
+  a.cache_rows = cache_rows;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.w = w;
+  a.positions = positions;
+  a.q_seq_offsets = q_seq_offsets;
+  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
+  a.cache_offsets = cache_offsets;
+  a.idx_out = idx_out;
+  a.score_out = score_out;
+  a.split = split;
+  a.sorted = (flags & DSA_TOPK_SORTED) != 0;
+  a.fp8 = fp8;
+  a.q_scale = fp8 ? q_scale : nullptr;
+  a.key_scale = fp8 ? key_scale : nullptr;
+  a.timeout_ns = timeout_ns();
+  if (launch_topk(a, h->ws, tmQ1, tmQ8, tmK, h->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dsa_status_t dsa_indexer_project(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
+                                 const int32_t* positions, const int32_t* q_seq_offsets, int32_t B, void* key_cache,
+                                 int64_t cache_rows, const int64_t* cache_offsets, void* q_out, float* w_out,
+                                 void* stream) {
+  return project_impl(h, T, hidden, q_latent, positions, q_seq_offsets, B, key_cache, nullptr, cache_rows,
+                      cache_offsets, q_out, nullptr, w_out, stream, false);
+}
+
+dsa_status_t dsa_indexer_project_fp8(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
+                                     const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                                     void* key_cache_fp8, float* key_scale, int64_t cache_rows,
+                                     const int64_t* cache_offsets, void* q_fp8, float* q_scale, float* w_out,
+                                     void* stream) {
+  return project_impl(h, T, hidden, q_latent, positions, q_seq_offsets, B, key_cache_fp8, key_scale, cache_rows,
+                      cache_offsets, q_fp8, q_scale, w_out, stream, true);
+}
+
+dsa_status_t dsa_indexer_quantize_keys_fp8(dsa_indexer_t h, int64_t n, const void* keys, void* key_cache_fp8,
+                                           float* key_scale, void* stream) {
+  if (!h || n < 0) return DSA_ERR_INVALID_ARG;
+  if (n == 0) return DSA_OK;
+  if (!keys || !key_cache_fp8 || !key_scale || !aligned16(keys) || !aligned16(key_cache_fp8) ||
+      (reinterpret_cast<uintptr_t>(key_scale) & 3) || n > (int64_t(1) << 34))
+    return DSA_ERR_INVALID_ARG;
+  if (launch_quantize_keys_fp8(n, static_cast<const __nv_bfloat16*>(keys), static_cast<uint8_t*>(key_cache_fp8),
+                               key_scale, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DSA_ERR_CUDA;
   return DSA_OK;
 }
 
@@ -278,48 +385,17 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
                               const int32_t* q_seq_offsets, int32_t B, const void* key_cache, int64_t cache_rows,
                               const int64_t* cache_offsets, int32_t* idx_out, float* score_out, uint32_t flags,
                               void* stream) {
-  if (!h) return DSA_ERR_INVALID_ARG;
-  if (T < 0 || B < 1) return DSA_ERR_INVALID_ARG;
-  if ((flags & DSA_TOPK_SPLIT) && (flags & DSA_TOPK_NO_SPLIT)) return DSA_ERR_INVALID_ARG;
-  if (flags & ~(DSA_TOPK_SORTED | DSA_TOPK_SPLIT | DSA_TOPK_NO_SPLIT)) return DSA_ERR_INVALID_ARG;
-  if (T == 0) return DSA_OK;
-  if (T > h->cfg.max_tokens || B > h->cfg.max_tokens) return DSA_ERR_WORKSPACE;
-  if (!q || !w || !positions || !q_seq_offsets || !key_cache || !cache_offsets || !idx_out) return DSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(w) || !aligned16(key_cache) || !aligned16(idx_out) ||
-      (score_out && !aligned16(score_out)) || (reinterpret_cast<uintptr_t>(positions) & 3) ||
-      (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7))
-    return DSA_ERR_INVALID_ARG;
-  if (cache_rows < 1 || cache_rows > (int64_t(1) << 31) - (int64_t(1) << 20)) return DSA_ERR_INVALID_ARG;
-  bool split = (T <= kSplitMaxTokens);
-  if (flags & DSA_TOPK_SPLIT) {
-    if (T > h->ws.part_tokens) return DSA_ERR_UNSUPPORTED;
-    split = true;
-  }
-  if (flags & DSA_TOPK_NO_SPLIT) split = false;
-  if (split && T > h->ws.part_tokens) split = false;
-  CUtensorMap tmQ1, tmQ8, tmK;
-  if (!make_tmap(&tmQ1, q, kHeadDim, uint64_t(T) * kHeads, 64, kHeads) ||
-      !make_tmap(&tmQ8, q, kHeadDim, uint64_t(T) * kHeads, 64, kHeads * kPrefillQ) ||
-      !make_tmap(&tmK, key_cache, kHeadDim, uint64_t(cache_rows), 64, kKeyTile))
-    return DSA_ERR_INVALID_ARG;
-  TopkArgs a{};
-  a.T = static_cast<int>(T);
-  a.B = B;
-  a.cache_rows = cache_rows;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.w = w;
-  a.positions = positions;
-  a.q_seq_offsets = q_seq_offsets;
-  a.key_cache = static_cast<const __nv_bfloat16*>(key_cache);
-  a.cache_offsets = cache_offsets;
-  a.idx_out = idx_out;
-  a.score_out = score_out;
-  a.split = split;
-  a.sorted = (flags & DSA_TOPK_SORTED) != 0;
-  a.timeout_ns = timeout_ns();
-  if (launch_topk(a, h->ws, tmQ1, tmQ8, tmK, h->num_sms, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  return DSA_OK;
+  return topk_impl(h, T, q, nullptr, w, positions, q_seq_offsets, B, key_cache, nullptr, cache_rows, cache_offsets,
+                   idx_out, score_out, flags, stream, false);
+}
+
+dsa_status_t dsa_indexer_topk_fp8(dsa_indexer_t h, int64_t T, const void* q_fp8, const float* q_scale, const float* w,
+                                  const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                                  const void* key_cache_fp8, const float* key_scale, int64_t cache_rows,
+                                  const int64_t* cache_offsets, int32_t* idx_out, float* score_out, uint32_t flags,
+                                  void* stream) {
+  return topk_impl(h, T, q_fp8, q_scale, w, positions, q_seq_offsets, B, key_cache_fp8, key_scale, cache_rows,
+                   cache_offsets, idx_out, score_out, flags, stream, true);
 }
 
 dsa_status_t dsa_indexer_topk_reuse(dsa_indexer_t h, int64_t n_draft, const int32_t* anchor_rows, int64_t n_src,

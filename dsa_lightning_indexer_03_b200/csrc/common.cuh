@@ -202,6 +202,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::f8f6f4 with FP8 e4m3 A and B (format code 0 in both
+// fields), fp32 accumulator, both operands K-major.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
+  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
                "r"(ncols)
@@ -266,6 +273,33 @@ __device__ __forceinline__ void umma_tile_k128(uint32_t d_tmem, uint32_t a_addr,
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%10];\n\t}"
       ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(0), "n"(A_HALF >> 4), "n"(B_HALF >> 4),
       "r"(smem_u32(bar0)), "r"(smem_u32(bar1))
+      : "memory");
+}
+
+// One 128-key tile of FP8 e4m3 operands: each 128-dim row is one 128-byte swizzle row, so the
+// contraction is 4 tcgen05.mma.kind::f8f6f4 of K = 32 (32 bytes each), the first overwriting
+// D; then commits to both barriers.
+__device__ __forceinline__ void umma_tile_k128_e4m3(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr,
+                                                    uint32_t idesc, uint64_t* bar0, uint64_t* bar1) {
+  const uint64_t ad = umma_desc_sw128(a_addr), bd = umma_desc_sw128(b_addr);
+  const uint32_t alo = static_cast<uint32_t>(ad), ahi = static_cast<uint32_t>(ad >> 32);
+  const uint32_t blo = static_cast<uint32_t>(bd), bhi = static_cast<uint32_t>(bd >> 32);
+  asm volatile(
+      "{\n\t.reg .pred p0, p1;\n\t.reg .b32 al, bl;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p0, %6, %6;\n\t"
+      "setp.eq.b32 p1, %6, %6;\n\t"
+      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, p0;\n\t"
+      "add.u32 al, %1, 2;\n\tadd.u32 bl, %3, 2;\n\tmov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, p1;\n\t"
+      "add.u32 al, %1, 4;\n\tadd.u32 bl, %3, 4;\n\tmov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, p1;\n\t"
+      "add.u32 al, %1, 6;\n\tadd.u32 bl, %3, 6;\n\tmov.b64 a, {al, %2};\n\tmov.b64 b, {bl, %4};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %5, p1;\n\t"
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}"
+      ::"r"(d_tmem), "r"(alo), "r"(ahi), "r"(blo), "r"(bhi), "r"(idesc), "r"(0), "r"(smem_u32(bar0)),
+      "r"(smem_u32(bar1))
       : "memory");
 }
 

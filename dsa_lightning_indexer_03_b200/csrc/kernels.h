@@ -20,6 +20,8 @@ struct ProjKwEpilogue {
   const int32_t* q_seq_offsets;   // [B+1]
   int B;
   const int64_t* cache_offsets;   // [B+1]
+  uint8_t* key8;                  // FP8 cache instead of key_cache when set: e4m3 codes [cache_rows, 128]
+  float* key_scale;               // FP8 cache: [cache_rows] scale of each row
   const float* gamma;             // [128]
   const float* beta;              // [128]
   float eps;
@@ -34,6 +36,14 @@ cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M,
 // [k~ | w] = A[M,K] * Bt[160,K]^T with the key LayerNorm / scatter epilogue; tmB box {64,160}
 cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K, const ProjKwEpilogue& e,
                            cudaStream_t s);
+
+// q8_out[M, N] = e4m3 codes of bf16(A * Bt^T) per 128-column head, q_scale[M, N/128]
+cudaError_t launch_proj_q8(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N, uint8_t* q8_out,
+                           float* q_scale, int* err, uint64_t timeout_ns, cudaStream_t s);
+
+// FP8 e4m3 codes and scales of n bf16 key rows (one scale per row)
+cudaError_t launch_quantize_keys_fp8(int64_t n, const __nv_bfloat16* keys, uint8_t* out, float* scale,
+                                     cudaStream_t s);
 
 cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,
                             const float* beta, float eps, cudaStream_t s);
@@ -93,6 +103,9 @@ struct TopkArgs {
   float* score_out;
   bool split;
   bool sorted;       // order each row by (score desc, position asc); short rows stay [0..p, -1...]
+  bool fp8;          // q and key_cache hold FP8 e4m3 codes with the scales below
+  const float* q_scale;    // FP8: [T, 32] per query head
+  const float* key_scale;  // FP8: [cache_rows] per key row
   uint64_t timeout_ns;
 };
 

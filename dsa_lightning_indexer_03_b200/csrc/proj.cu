@@ -17,6 +17,8 @@
 // CTAs that reduce their partial tiles through distributed shared memory before
 // the LayerNorm epilogue, so that every token count keeps many SMs streaming.
 
+#include <cuda_fp8.h>
+
 #include "kernels.h"
 
 namespace dsa {
@@ -27,12 +29,14 @@ constexpr int kBK = 64;
 constexpr int kABytes = kBM * kBK * 2;  // 16 KB per stage
 constexpr uint64_t kDrainNs = 200ull * 1000 * 1000;
 
-enum { EPI_Q = 0, EPI_KW = 1 };
+enum { EPI_Q = 0, EPI_KW = 1, EPI_Q8 = 2 };
 
 struct ProjParams {
   int M, K;
   __nv_bfloat16* q_out;  // EPI_Q
   int ldq;
+  uint8_t* q8_out;       // EPI_Q8: FP8 e4m3 codes [M, ldq]
+  float* q_scale;        // EPI_Q8: [M, ldq / 128], one scale per query head
   ProjKwEpilogue kw;     // EPI_KW
   int* err;
   uint64_t timeout_ns;
@@ -51,6 +55,23 @@ struct ProjSmem {
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// FP8 e4m3 codes of four values (round to nearest even, saturating at +-448), first value
+// in the lowest byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return (lo & 0xFFFFu) | (hi << 16);
+}
+
+// Scale and inverse scale of a row whose largest magnitude is amax: amax / 448 and
+// 448 / amax (both 0 for an all-zero row); codes are e4m3(x * inv), values code * scale.
+__device__ __forceinline__ void fp8_row_scale(float amax, float* scale, float* inv) {
+  *scale = amax > 0.f ? __fdiv_rn(amax, 448.f) : 0.f;
+  *inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
 }
 
 // waits without looking at the abort flag (used only to drain in-flight work)
@@ -174,6 +195,43 @@ __global__ void __launch_bounds__(192, 1)
               d4[v] = pk;
             }
           }
+        }
+      } else if constexpr (EPI == EPI_Q8) {
+        // per head (128 columns): q = bf16(acc), then FP8 codes with the head's scale
+#pragma unroll 1
+        for (int hh = 0; hh < BN / 128; ++hh) {
+          float amax = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld_32cols(tbase + hh * 128 + c * 32, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(round_bf16(__uint_as_float(r[i]))));
+          }
+          float scale, inv;
+          fp8_row_scale(amax, &scale, &inv);
+          const int head = (n0 >> 7) + hh;
+          uint8_t* dst = p.q8_out + static_cast<size_t>(row) * p.ldq + head * 128;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld_32cols(tbase + hh * 128 + c * 32, r);
+            tmem_ld_wait(r);
+            if (row < p.M) {
+              uint32_t w8[8];
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                w8[v] = pack_e4m3x4(__fmul_rn(round_bf16(__uint_as_float(r[4 * v])), inv),
+                                    __fmul_rn(round_bf16(__uint_as_float(r[4 * v + 1])), inv),
+                                    __fmul_rn(round_bf16(__uint_as_float(r[4 * v + 2])), inv),
+                                    __fmul_rn(round_bf16(__uint_as_float(r[4 * v + 3])), inv));
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+              d4[0] = make_uint4(w8[0], w8[1], w8[2], w8[3]);
+              d4[1] = make_uint4(w8[4], w8[5], w8[6], w8[7]);
+            }
+          }
+          if (row < p.M) p.q_scale[static_cast<size_t>(row) * (p.ldq >> 7) + head] = scale;
         }
       } else {
         // key: LayerNorm over columns 0..127 of this token's row, fp32 math
@@ -449,6 +507,23 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
     for (int o = 1; o < CS; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rstd = rsqrtf(ss * (1.0f / 128.0f) + p.kw.eps);
+    // FP8 cache: k = bf16(LayerNorm), then e4m3 codes with the row's scale (the shuffles run
+    // on every lane, before the per-token branch)
+    const bool fp8 = p.kw.key8 != nullptr;
+    float y8[kKeyCols];
+    float scale8 = 0.f, inv8 = 0.f;
+    if (fp8) {
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < kKeyCols; ++i) {
+        const int d = t * kKeyCols + i;
+        y8[i] = round_bf16(fmaf((xk[i] - mean) * rstd, s_gamma[d], s_beta[d]));
+        amax = fmaxf(amax, fabsf(y8[i]));
+      }
+#pragma unroll
+      for (int o = 1; o < CS; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      fp8_row_scale(amax, &scale8, &inv8);
+    }
     const int tok = m0 + trow;
     if (tok < p.M) {
       const int pos = p.kw.positions[tok];
@@ -460,7 +535,20 @@ __global__ void __launch_bounds__(192, 1)
       }
       const int64_t cb = p.kw.cache_offsets[lo];
       const int64_t len = p.kw.cache_offsets[lo + 1] - cb;
-      if (pos >= 0 && pos < len && cb >= 0 && cb + pos < p.kw.cache_rows) {
+      const bool in_cache = pos >= 0 && pos < len && cb >= 0 && cb + pos < p.kw.cache_rows;
+      if (fp8) {
+        if (in_cache) {
+          uint32_t* d32 = reinterpret_cast<uint32_t*>(p.kw.key8 + static_cast<size_t>(cb + pos) * kHeadDim +
+                                                      t * kKeyCols);
+#pragma unroll
+          for (int v = 0; v < kKeyCols / 4; ++v)
+            d32[v] = pack_e4m3x4(__fmul_rn(y8[4 * v], inv8), __fmul_rn(y8[4 * v + 1], inv8),
+                                 __fmul_rn(y8[4 * v + 2], inv8), __fmul_rn(y8[4 * v + 3], inv8));
+          if (t == 0) p.kw.key_scale[cb + pos] = scale8;
+        } else if (t == 0) {
+          atomicOr(p.err, kErrBounds);
+        }
+      } else if (in_cache) {
         uint4* d4 = reinterpret_cast<uint4*>(p.kw.key_cache + static_cast<size_t>(cb + pos) * kHeadDim +
                                              t * kKeyCols);
 #pragma unroll
@@ -520,6 +608,28 @@ __global__ void __launch_bounds__(256) key_norm_kernel(int64_t n, const float* _
   pk.x = pack_bf16x2(fmaf(d0 * rstd, g.x, b.x), fmaf(d1 * rstd, g.y, b.y));
   pk.y = pack_bf16x2(fmaf(d2 * rstd, g.z, b.z), fmaf(d3 * rstd, g.w, b.w));
   reinterpret_cast<uint2*>(out + row * kHeadDim)[lane] = pk;
+}
+
+// ---------------------------------------------------------------- bf16 key rows -> FP8 cache rows
+// One warp per 128-value row: each lane converts 4 values; the row's largest magnitude comes
+// from a warp reduction.
+__global__ void __launch_bounds__(256) quantize_keys_fp8_kernel(int64_t n, const __nv_bfloat16* __restrict__ keys,
+                                                                uint8_t* __restrict__ out, float* __restrict__ scale) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n) return;
+  const uint2 raw = reinterpret_cast<const uint2*>(keys + row * kHeadDim)[lane];
+  const __nv_bfloat162 b0 = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  const __nv_bfloat162 b1 = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  const float v0 = __low2float(b0), v1 = __high2float(b0), v2 = __low2float(b1), v3 = __high2float(b1);
+  float amax = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  float sc, inv;
+  fp8_row_scale(amax, &sc, &inv);
+  reinterpret_cast<uint32_t*>(out + row * kHeadDim)[lane] =
+      pack_e4m3x4(__fmul_rn(v0, inv), __fmul_rn(v1, inv), __fmul_rn(v2, inv), __fmul_rn(v3, inv));
+  if (lane == 0) scale[row] = sc;
 }
 
 // ---------------------------------------------------------------- weight re-layout at create
@@ -599,6 +709,27 @@ cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K
   if (nk >= 4) return launch_kw_cluster<4>(tmA, tmB, p, s);
   if (nk >= 2) return launch_kw_cluster<2>(tmA, tmB, p, s);
   return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
+}
+
+cudaError_t launch_proj_q8(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N, uint8_t* q8_out,
+                           float* q_scale, int* err, uint64_t timeout_ns, cudaStream_t s) {
+  ProjParams p{};
+  p.M = M;
+  p.K = K;
+  p.q8_out = q8_out;
+  p.q_scale = q_scale;
+  p.ldq = N;
+  p.err = err;
+  p.timeout_ns = timeout_ns;
+  return launch_proj<256, 4, EPI_Q8>(tmA, tmB, p, N / 256, s);
+}
+
+cudaError_t launch_quantize_keys_fp8(int64_t n, const __nv_bfloat16* keys, uint8_t* out, float* scale,
+                                     cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 7) / 8;
+  quantize_keys_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(n, keys, out, scale);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,

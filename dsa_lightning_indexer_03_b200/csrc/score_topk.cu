@@ -52,6 +52,8 @@ struct ScoreParams {
   uint32_t* part_keys;          // [T][kMaxChunks][kTopK]
   int32_t* part_idx;
   uint32_t* part_hist;          // [T][kBins1]: first-level bin counts of each query's partial lists
+  const float* q_scale;         // FP8: [T, 32] scale of each query head (folded into its weight)
+  const float* key_scale;       // FP8: [cache_rows] scale of each key row (multiplies the score)
   int* err;
   uint64_t timeout_ns;
 };
@@ -623,8 +625,11 @@ struct WGState {
 // queries (ALT = false) or, with ALT, take whole items in turn (group g takes the items
 // the CTA receives at positions g, g + 2, ...): one group's end-of-item selection then
 // overlaps the other group's tiles.
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, int EB = 2>
 struct ScoreCfg {
+  // EB = bytes per element of q and of the keys: 2 (bf16, kind::f16 MMA) or 1 (FP8 e4m3,
+  // kind::f8f6f4 MMA).  A 128-dim row is EB 128-byte swizzle rows ("halves") wide.
+  static constexpr int kHalves = EB;
   static constexpr int kQPW = ALT ? QMAX : QMAX / NWG;  // queries of one epilogue group
   static constexpr int kConsumers = ALT ? EW : NWG * EW; // warps that consume each tile
   static constexpr int kQPH = kQPW / (EW / 4);        // queries of one epilogue warp
@@ -639,11 +644,11 @@ struct ScoreCfg {
   static constexpr int kTmemNeed = kTotalBufs * kAccCols;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kQHalf = QMAX * kHeads * 128;  // bytes of one 64-column half of the Q tile
+  static constexpr int kQHalf = QMAX * kHeads * 128;  // bytes of one 128-byte-wide half of the Q tile
   static constexpr int kKHalf = kKeyTile * 128;       // 16 KB
-  static constexpr int kKStage = 2 * kKHalf;
+  static constexpr int kKStage = kHalves * kKHalf;
   static constexpr int kQOff = 0;
-  static constexpr int kKOff = 2 * kQHalf;
+  static constexpr int kKOff = kHalves * kQHalf;
   static constexpr int kWGOff = kKOff + STAGES * kKStage;
   static constexpr int kWGBytes = (static_cast<int>(sizeof(WGState<kQPW>)) + 15) / 16 * 16;
   static constexpr int kBarOff = kWGOff + NWG * kWGBytes;
@@ -681,11 +686,12 @@ __device__ __forceinline__ void sum_over_quad(const float (&part)[4 * QPH], floa
   }
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED>
-__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>::kThreads, 1)
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB>
+__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>::kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       ScoreParams p) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>;
+  constexpr bool kFp8 = EB == 1;
   constexpr int QPW = C::kQPW;
   constexpr int QPH = C::kQPH;
   constexpr int NTG = C::kGroupThreads;
@@ -778,9 +784,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
         const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
         if (kt1 <= kt0) continue;
         if (qloads > 0 && !mbar_wait(q_empty, (qloads - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(q_full, 2 * C::kQHalf);
+        mbar_arrive_expect_tx(q_full, C::kHalves * C::kQHalf);
         tma_load_2d_hint(sQ, &tmQ, q_full, 0, wi.t0 * kHeads, pol_q);
-        tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * kHeads, pol_q);
+        if constexpr (!kFp8) tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * kHeads, pol_q);
         ++qloads;
         const int row0 = static_cast<int>(p.cache_offsets[wi.b]);
         bool ok = true;
@@ -793,7 +799,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
           mbar_arrive_expect_tx(&full[s], C::kKStage);
           uint8_t* dst = sK + s * C::kKStage;
           tma_load_2d_hint(dst, &tmK, &full[s], 0, row0 + kt * kKeyTile, pol_k);
-          tma_load_2d_hint(dst + C::kKHalf, &tmK, &full[s], 64, row0 + kt * kKeyTile, pol_k);
+          if constexpr (!kFp8) tma_load_2d_hint(dst + C::kKHalf, &tmK, &full[s], 64, row0 + kt * kKeyTile, pol_k);
         }
         if (!ok) break;
       }
@@ -821,7 +827,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
         if (!mbar_wait(q_full, qloads & 1, wc)) break;
         ++qloads;
         tc_fence_after();
-        const uint32_t idesc = umma_idesc_bf16(kKeyTile, wi.nq * kHeads);
+        const uint32_t idesc = kFp8 ? umma_idesc_e4m3(kKeyTile, wi.nq * kHeads) : umma_idesc_bf16(kKeyTile, wi.nq * kHeads);
         const bool second = ALT && (local & 1);   // with ALT, the CTA's odd items go to group 1
         bool ok = true;
         for (int kt = kt0; kt < kt1; ++kt, ++kstage) {
@@ -836,8 +842,12 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
             break;
           }
           tc_fence_after();
-          umma_tile_k128<C::kKHalf, C::kQHalf>(tmem + ab * C::kAccCols, smem_u32(sK + s * C::kKStage), qa, idesc,
-                                              &empty[s], &acc_full[ab]);
+          if constexpr (kFp8)
+            umma_tile_k128_e4m3(tmem + ab * C::kAccCols, smem_u32(sK + s * C::kKStage), qa, idesc, &empty[s],
+                                &acc_full[ab]);
+          else
+            umma_tile_k128<C::kKHalf, C::kQHalf>(tmem + ab * C::kAccCols, smem_u32(sK + s * C::kKStage), qa, idesc,
+                                                &empty[s], &acc_full[ab]);
         }
         umma_commit(q_empty);
         if (!ok) break;
@@ -911,7 +921,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
       if (it >= 0) {
         for (int i = gtid; i < QPW * kHeads; i += NTG) {
           const int jj = i / kHeads, j = qbase + jj;
-          st.w[jj][i % kHeads] = (j < wi.nq) ? p.w[static_cast<size_t>(wi.t0 + j) * kHeads + (i % kHeads)] : 0.f;
+          const size_t wix = static_cast<size_t>(wi.t0 + j) * kHeads + (i % kHeads);
+          // FP8: the query head's scale joins its weight (sum_h w_h s_h ReLU(q8_h . k8))
+          st.w[jj][i % kHeads] = (j < wi.nq) ? (kFp8 ? p.w[wix] * p.q_scale[wix] : p.w[wix]) : 0.f;
         }
       }
       if (named_bar_or(bar, NTG, it < 0)) break;   // every thread of the group leaves together
@@ -919,6 +931,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
       const int nloc = min(QPW, wi.nq - qbase);    // queries of the group present in this item
       const int nmine = min(QPH, nloc - j0);        // ... and scored by this warp (may be <= 0)
       const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
+      const int64_t kbase = kFp8 ? p.cache_offsets[wi.b] : 0;   // first key-cache row of the sequence
       // an item of at most kWarpApp / 32 tiles cannot fill an append area: no capacity checks
       const bool long_item = (kt1 - kt0) * 32 > kWarpApp;
       int cnt_r[QPH], pos_r[QPH];
@@ -976,6 +989,13 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>
             }
           float score[QPH];
           sum_over_quad<QPH>(part, score, lane);
+          if constexpr (kFp8) {
+            // the key row's scale (positive) multiplies every head's ReLU term; rows past the
+            // item's last scored key are masked and not read
+            const float sk = s_pos < wi.k_end ? __ldg(p.key_scale + kbase + s_pos) : 0.f;
+#pragma unroll
+            for (int j = 0; j < QPH; ++j) score[j] *= sk;
+          }
           // admit (key, position) into this warp's area of each of its queries and count it;
           // the append counts stay warp-uniform in registers
 #pragma unroll
@@ -1562,11 +1582,11 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
   *status = ok ? 0 : ((err & kErrTimeout) ? 2 : 1);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB>
 cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const ScoreParams& p, int grid,
                          cudaStream_t s) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT>;
-  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, SORTED>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>;
+  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, SORTED, EB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (C::kRegSplit) {
@@ -1628,12 +1648,18 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.part_keys = ws.part_keys;
   sp.part_idx = ws.part_idx;
   sp.part_hist = ws.part_hist;
+  sp.q_scale = a.q_scale;
+  sp.key_scale = a.key_scale;
   sp.err = ws.err;
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
   if (a.split) {
-    e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true>(tmQ1, tmK, sp, grid, s)
-                 : launch_score<1, 5, 4, 2, 4, true, false>(tmQ1, tmK, sp, grid, s);
+    if (a.fp8)   // 16 KB key tiles: twice the stages keep the same bytes in flight
+      e = a.sorted ? launch_score<1, 10, 4, 2, 4, true, true, 1>(tmQ1, tmK, sp, grid, s)
+                   : launch_score<1, 10, 4, 2, 4, true, false, 1>(tmQ1, tmK, sp, grid, s);
+    else
+      e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true, 2>(tmQ1, tmK, sp, grid, s)
+                   : launch_score<1, 5, 4, 2, 4, true, false, 2>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
     const int msmem = 2 * kMergeList * 4 + kTopK * 8;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
@@ -1654,8 +1680,11 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
                               static_cast<const int32_t*>(ws.part_idx), static_cast<const int*>(ws.tok_nchunks),
                               ws.part_hist, a.idx_out, a.score_out, a.sorted ? 1 : 0);
   }
-  return a.sorted ? launch_score<kPrefillQ, 3, 2, 2, 8, false, true>(tmQ8, tmK, sp, grid, s)
-                  : launch_score<kPrefillQ, 3, 2, 2, 8, false, false>(tmQ8, tmK, sp, grid, s);
+  if (a.fp8)
+    return a.sorted ? launch_score<kPrefillQ, 6, 2, 2, 8, false, true, 1>(tmQ8, tmK, sp, grid, s)
+                    : launch_score<kPrefillQ, 6, 2, 2, 8, false, false, 1>(tmQ8, tmK, sp, grid, s);
+  return a.sorted ? launch_score<kPrefillQ, 3, 2, 2, 8, false, true, 2>(tmQ8, tmK, sp, grid, s)
+                  : launch_score<kPrefillQ, 3, 2, 2, 8, false, false, 2>(tmQ8, tmK, sp, grid, s);
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s) {

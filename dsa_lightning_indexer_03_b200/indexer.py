@@ -146,6 +146,81 @@ class Indexer:
               "dsa_indexer_topk")
         return idx_out, score_out
 
+    # ------------------------------------------------------------------ FP8 key cache
+    def project_fp8(self, hidden, q_latent, positions, q_seq_offsets, key_cache_fp8, key_scale, cache_offsets,
+                    q_out=None, q_scale=None, w_out=None, stream=None):
+        """FP8 projections: e4m3 codes q [T, n_heads, head_dim] (uint8) with per-head scales
+        [T, n_heads] and w [T, n_heads] fp32; each token's key goes to key_cache_fp8 (uint8
+        [rows, head_dim]) with its scale in key_scale (fp32 [rows])."""
+        dev = self.device
+        T = hidden.shape[0]
+        _need(hidden, "hidden", torch.bfloat16, dev)
+        _need(q_latent, "q_latent", torch.bfloat16, dev)
+        _need(positions, "positions", torch.int32, dev)
+        _need(q_seq_offsets, "q_seq_offsets", torch.int32, dev)
+        _need(key_cache_fp8, "key_cache_fp8", torch.uint8, dev)
+        _need(key_scale, "key_scale", torch.float32, dev)
+        _need(cache_offsets, "cache_offsets", torch.int64, dev)
+        if q_out is None:
+            q_out = torch.empty((T, self.n_heads, self.head_dim), dtype=torch.uint8, device=dev)
+        if q_scale is None:
+            q_scale = torch.empty((T, self.n_heads), dtype=torch.float32, device=dev)
+        if w_out is None:
+            w_out = torch.empty((T, self.n_heads), dtype=torch.float32, device=dev)
+        _need(q_out, "q_out", torch.uint8, dev)
+        _need(q_scale, "q_scale", torch.float32, dev)
+        _need(w_out, "w_out", torch.float32, dev)
+        B = q_seq_offsets.numel() - 1
+        check(self._lib.dsa_indexer_project_fp8(self._h, T, _ptr(hidden), _ptr(q_latent), _ptr(positions),
+                                                _ptr(q_seq_offsets), B, _ptr(key_cache_fp8), _ptr(key_scale),
+                                                key_cache_fp8.shape[0], _ptr(cache_offsets), _ptr(q_out),
+                                                _ptr(q_scale), _ptr(w_out), _stream(stream)),
+              "dsa_indexer_project_fp8")
+        return q_out, q_scale, w_out
+
+    def quantize_keys_fp8(self, keys, out=None, scale=None, stream=None):
+        """FP8 codes (uint8 [n, head_dim]) and per-row scales (fp32 [n]) of bf16 key rows."""
+        dev = self.device
+        _need(keys, "keys", torch.bfloat16, dev)
+        n = keys.shape[0]
+        if out is None:
+            out = torch.empty((n, self.head_dim), dtype=torch.uint8, device=dev)
+        if scale is None:
+            scale = torch.empty((n,), dtype=torch.float32, device=dev)
+        _need(out, "out", torch.uint8, dev)
+        _need(scale, "scale", torch.float32, dev)
+        check(self._lib.dsa_indexer_quantize_keys_fp8(self._h, n, _ptr(keys), _ptr(out), _ptr(scale),
+                                                      _stream(stream)), "dsa_indexer_quantize_keys_fp8")
+        return out, scale
+
+    def topk_fp8(self, q, q_scale, w, positions, q_seq_offsets, key_cache_fp8, key_scale, cache_offsets,
+                 idx_out=None, score_out=None, return_scores: bool = True, flags: int = 0, stream=None):
+        """topk over FP8 queries and an FP8 key cache."""
+        dev = self.device
+        T = q.shape[0]
+        _need(q, "q", torch.uint8, dev)
+        _need(q_scale, "q_scale", torch.float32, dev)
+        _need(w, "w", torch.float32, dev)
+        _need(positions, "positions", torch.int32, dev)
+        _need(q_seq_offsets, "q_seq_offsets", torch.int32, dev)
+        _need(key_cache_fp8, "key_cache_fp8", torch.uint8, dev)
+        _need(key_scale, "key_scale", torch.float32, dev)
+        _need(cache_offsets, "cache_offsets", torch.int64, dev)
+        if idx_out is None:
+            idx_out = torch.empty((T, self.top_k), dtype=torch.int32, device=dev)
+        _need(idx_out, "idx_out", torch.int32, dev)
+        if score_out is None and return_scores:
+            score_out = torch.empty((T, self.top_k), dtype=torch.float32, device=dev)
+        if score_out is not None:
+            _need(score_out, "score_out", torch.float32, dev)
+        B = q_seq_offsets.numel() - 1
+        check(self._lib.dsa_indexer_topk_fp8(self._h, T, _ptr(q), _ptr(q_scale), _ptr(w), _ptr(positions),
+                                             _ptr(q_seq_offsets), B, _ptr(key_cache_fp8), _ptr(key_scale),
+                                             key_cache_fp8.shape[0], _ptr(cache_offsets), _ptr(idx_out),
+                                             _ptr(score_out), int(flags), _stream(stream)),
+              "dsa_indexer_topk_fp8")
+        return idx_out, score_out
+
     def topk_reuse(self, anchor_rows, src_idx, src_score=None, idx_out=None, score_out=None, stream=None):
         """Rows of earlier dsa_indexer_topk results reused by speculative draft tokens: row d of
         the output is row anchor_rows[d] of src_idx (and src_score, when given)."""

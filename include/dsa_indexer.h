@@ -157,6 +157,47 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
                               int32_t* idx_out,
                               float* score_out, uint32_t flags, void* stream);
 
+/* ---- FP8 indexer-key cache ('FP8 -> FP4 training' row of the page "Kimi K3.1
+ * Pro vs GLM-5": vLLM and SGLang cache the indexer keys in FP8 by default).
+ * The key cache holds FP8 e4m3 codes [cache_rows, head_dim] (one byte each,
+ * 128-byte rows) and one fp32 scale per row; queries hold e4m3 codes
+ * [T, n_heads, head_dim] and one fp32 scale per (token, head).  A row x of
+ * float values is stored as scale = amax / 448 (0 for an all-zero row) and
+ * codes e4m3(x * (448 / amax)), rounded to nearest even with saturation; the
+ * value represented is code * scale.  x is the bf16 key (after the LayerNorm)
+ * or the bf16 query head, so the FP8 cache stores what the bf16 path would,
+ * rounded once more.  Scores become
+ *     I[t,s] = key_scale[s] * sum_h (w[t,h] * q_scale[t,h]) * ReLU(q8[t,h] . k8[s])
+ * (the positive scales factor out of the ReLU), computed on the tensor cores
+ * with kind::f8f6f4 MMAs; decode reads 132 bytes per cached key instead of 256.
+ * Requires hidden_dim >= 128 (DSA_ERR_UNSUPPORTED otherwise). */
+
+/* dsa_indexer_project with FP8 outputs: key_cache_fp8 uint8 [cache_rows, head_dim]
+ * and key_scale fp32 [cache_rows] receive the token's key row; q_fp8 uint8
+ * [T, n_heads*head_dim] and q_scale fp32 [T, n_heads] the query; w_out as for
+ * dsa_indexer_project.  Other arguments and rules as for dsa_indexer_project. */
+dsa_status_t dsa_indexer_project_fp8(dsa_indexer_t h, int64_t T, const void* hidden, const void* q_latent,
+                                     const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                                     void* key_cache_fp8, float* key_scale, int64_t cache_rows,
+                                     const int64_t* cache_offsets, void* q_fp8, float* q_scale, float* w_out,
+                                     void* stream);
+
+/* FP8 codes and scales of n bf16 key rows keys [n, head_dim] (e.g. an existing
+ * bf16 cache, or the output of dsa_indexer_key_norm): key_cache_fp8 uint8
+ * [n, head_dim], key_scale fp32 [n]. */
+dsa_status_t dsa_indexer_quantize_keys_fp8(dsa_indexer_t h, int64_t n, const void* keys, void* key_cache_fp8,
+                                           float* key_scale, void* stream);
+
+/* dsa_indexer_topk over an FP8 cache: q_fp8 uint8 [T, n_heads, head_dim] with
+ * q_scale fp32 [T, n_heads], key_cache_fp8 uint8 [cache_rows, head_dim] with
+ * key_scale fp32 [cache_rows]; scores as above.  Every other argument, flag,
+ * output rule and error as for dsa_indexer_topk. */
+dsa_status_t dsa_indexer_topk_fp8(dsa_indexer_t h, int64_t T, const void* q_fp8, const float* q_scale, const float* w,
+                                  const int32_t* positions, const int32_t* q_seq_offsets, int32_t B,
+                                  const void* key_cache_fp8, const float* key_scale, int64_t cache_rows,
+                                  const int64_t* cache_offsets, int32_t* idx_out, float* score_out, uint32_t flags,
+                                  void* stream);
+
 /* Index reuse across speculative draft steps ('MTP' row of the page "Kimi K3.1
  * Pro vs GLM-5": GLM-5.2 reuses the first step's top-k indices in its later
  * draft steps).  Draft token d takes the selection of its anchor: row
