@@ -14,6 +14,7 @@ from .indexer_oracle import (  # noqa: F401
     parameter_count,
     layer_norm,
     key_norm,
+    rope,
     project,
     project_keys,
     index_scores,

@@ -129,15 +129,39 @@ def project_keys(hidden, W_k, gamma, beta, eps: float = LN_EPS) -> np.ndarray:
     return key_norm(np.asarray(hidden, np.float64) @ np.asarray(W_k, np.float64), gamma, beta, eps)
 
 
+def rope(x, positions, rope_dim: int, theta: float = 10000.0) -> np.ndarray:
+    """Rotary encoding of the first rope_dim dims of the last axis: for i < rope_dim / 2 the
+    pair (x[2i], x[2i+1]) is rotated by the angle p * theta^(-2i / rope_dim), p the row's
+    position; the other dims pass unchanged.  positions broadcast against x's leading axes
+    (one per row).  DeepSeek-V3.2's indexer rotates 64 of its 128 dims ('Partial RoPE /
+    NoPE' row, page "Kimi K3.1 Pro vs Gemma 4 31B"); Kimi K3.1's rotates none."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    if rope_dim == 0:
+        return x
+    i = np.arange(rope_dim // 2, dtype=np.float64)
+    inv_freq = theta ** (-2.0 * i / rope_dim)
+    ang = np.asarray(positions, np.float64)[..., None] * inv_freq
+    c, s = np.cos(ang), np.sin(ang)
+    a = x[..., 0:rope_dim:2].copy()
+    b = x[..., 1:rope_dim:2].copy()
+    x[..., 0:rope_dim:2] = a * c - b * s
+    x[..., 1:rope_dim:2] = a * s + b * c
+    return x
+
+
 def project(hidden, q_latent, W_q, W_k, W_w, gamma, beta, eps: float = LN_EPS,
-            n_heads: int = 32, head_dim: int = 128):
+            n_heads: int = 32, head_dim: int = 128, positions=None, rope_dim: int = 0,
+            rope_theta: float = 10000.0):
     """Indexer projections of T tokens.
 
-    q = bf16(q_latent @ W_q) viewed [T, n_heads, head_dim] (head h = columns
+    q = bf16(RoPE(q_latent @ W_q)) viewed [T, n_heads, head_dim] (head h = columns
         h*head_dim .. h*head_dim + head_dim - 1);
-    k = bf16(LayerNorm(hidden @ W_k));
+    k = bf16(RoPE(LayerNorm(hidden @ W_k)));
     w = fp32(hidden @ W_w).
-    All products and sums in float64; one rounding per output."""
+    RoPE (rope_dim > 0, the DeepSeek-V3.2 form; needs `positions`) rotates the first
+    rope_dim dims of every head of q and of k by the token's position; with rope_dim = 0
+    (Kimi K3.1) there is no rotary step.  All products and sums in float64; one rounding
+    per output."""
     hidden = np.asarray(hidden, np.float64)
     q_latent = np.asarray(q_latent, np.float64)
     shapes = parameter_shapes(hidden.shape[1], q_latent.shape[1], n_heads, head_dim)
@@ -145,8 +169,17 @@ def project(hidden, q_latent, W_q, W_k, W_w, gamma, beta, eps: float = LN_EPS,
         if tuple(np.shape(arr)) != shapes[name]:
             raise ValueError(f"{name} has shape {np.shape(arr)}, expected {shapes[name]}")
     T = hidden.shape[0]
-    q = bf16_round(q_latent @ np.asarray(W_q, np.float64)).reshape(T, n_heads, head_dim)
-    k = project_keys(hidden, W_k, gamma, beta, eps)
+    if rope_dim:
+        if positions is None:
+            raise ValueError("rope_dim > 0 needs the token positions")
+        pos = np.asarray(positions, np.float64)
+        q = bf16_round(rope((q_latent @ np.asarray(W_q, np.float64)).reshape(T, n_heads, head_dim),
+                            pos[:, None], rope_dim, rope_theta))
+        k = bf16_round(rope(layer_norm(hidden @ np.asarray(W_k, np.float64), gamma, beta, eps), pos, rope_dim,
+                            rope_theta))
+    else:
+        q = bf16_round(q_latent @ np.asarray(W_q, np.float64)).reshape(T, n_heads, head_dim)
+        k = project_keys(hidden, W_k, gamma, beta, eps)
     w = (hidden @ np.asarray(W_w, np.float64)).astype(np.float32).astype(np.float64)
     return q, k, w
 

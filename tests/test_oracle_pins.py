@@ -477,3 +477,64 @@ def test_fp8_selection_tracks_the_bf16_selection():
     idx_f, _ = oracle.topk_fp8(q8, sq, w, pos, np.array([0, T]), k8, sk, np.array([0, S]))
     for r in range(T):
         assert len(np.intersect1d(idx_b[r], idx_f[r])) / 2048 > 0.9
+
+
+# ---------------------------------------------------------------- DeepSeek-V3.2 form: 64 heads, RoPE on 64 dims
+
+def test_rope_identity_cases():
+    rng = np.random.default_rng(51)
+    x = rng.standard_normal((5, 128))
+    assert np.array_equal(oracle.rope(x, np.zeros(5), 64), x)            # position 0
+    assert np.array_equal(oracle.rope(x, np.arange(5), 0), x)            # no rotary dims
+    y = oracle.rope(x, np.arange(5) * 1000, 64)
+    assert np.array_equal(y[:, 64:], x[:, 64:])                          # only the first 64 dims move
+
+
+def test_rope_is_a_rotation_with_relative_positions():
+    rng = np.random.default_rng(52)
+    q = rng.standard_normal((7, 128))
+    k = rng.standard_normal((7, 128))
+    p = rng.integers(0, 100_000, 7).astype(np.float64)
+    s = rng.integers(0, 100_000, 7).astype(np.float64)
+    rq = oracle.rope(q, p, 64)
+    # each rotated pair keeps its length
+    assert np.allclose(np.hypot(rq[:, 0:64:2], rq[:, 1:64:2]), np.hypot(q[:, 0:64:2], q[:, 1:64:2]), rtol=1e-12)
+    # composition: rotating by p1 then p2 is rotating by p1 + p2
+    assert np.allclose(oracle.rope(oracle.rope(q, p, 64), s, 64), oracle.rope(q, p + s, 64), atol=1e-9)
+    # the dot product depends on the positions only through their difference
+    d = 12345.0
+    a = np.sum(oracle.rope(q, p, 64) * oracle.rope(k, s, 64), axis=1)
+    b = np.sum(oracle.rope(q, p + d, 64) * oracle.rope(k, s + d, 64), axis=1)
+    assert np.allclose(a, b, rtol=1e-9, atol=1e-9)
+    # the lowest pair turns by one radian per position, the highest by theta^(-62/64) of one
+    e = np.zeros((1, 128))
+    e[0, 0] = 1.0
+    e[0, 62] = 1.0
+    r = oracle.rope(e, np.array([3.0]), 64)
+    assert np.isclose(np.arctan2(r[0, 1], r[0, 0]), 3.0 - 0.0)
+    assert np.isclose(np.arctan2(r[0, 63], r[0, 62]), 3.0 * 10000.0 ** (-62 / 64))
+
+
+def test_project_64_heads_with_rope():
+    # the 64-head form: W_q 1,536 -> 8,192, W_w 7,168 -> 64 (shapes scaled down here), rotary
+    # step on the first 64 dims of q (every head) and of the normalised key
+    rng = np.random.default_rng(53)
+    T, hd, ql, H, D = 6, 32, 16, 4, 128
+    shapes = oracle.parameter_shapes(hd, ql, H, D)
+    ws = {k_: rng.standard_normal(s_) * 0.3 for k_, s_ in shapes.items()}
+    x, xq = rng.standard_normal((T, hd)), rng.standard_normal((T, ql))
+    pos = np.array([0, 1, 7, 100, 5000, 70000])
+    q0, k0, w0 = oracle.project(x, xq, ws["W_q"], ws["W_k"], ws["W_w"], ws["ln_gamma"], ws["ln_beta"],
+                                n_heads=H, head_dim=D)
+    q1, k1, w1 = oracle.project(x, xq, ws["W_q"], ws["W_k"], ws["W_w"], ws["ln_gamma"], ws["ln_beta"],
+                                n_heads=H, head_dim=D, positions=pos, rope_dim=64)
+    assert np.array_equal(w0, w1)
+    assert np.array_equal(q0[0], q1[0]) and np.array_equal(k0[0], k1[0])       # position 0
+    assert np.array_equal(q0[:, :, 64:], q1[:, :, 64:]) and np.array_equal(k0[:, 64:], k1[:, 64:])
+    assert not np.allclose(q0[3:, :, :64], q1[3:, :, :64])
+    # the rotated values are the rounding of the rotated unrounded projection
+    raw = (xq @ ws["W_q"]).reshape(T, H, D)
+    assert np.array_equal(q1, oracle.bf16_round(oracle.rope(raw, pos[:, None], 64)))
+    with pytest.raises(ValueError):
+        oracle.project(x, xq, ws["W_q"], ws["W_k"], ws["W_w"], ws["ln_gamma"], ws["ln_beta"], n_heads=H,
+                       head_dim=D, rope_dim=64)
