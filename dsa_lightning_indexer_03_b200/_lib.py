@@ -35,6 +35,8 @@ class Config(ctypes.Structure):
         ("top_k", ctypes.c_int32),
         ("ln_eps", ctypes.c_float),
         ("max_tokens", ctypes.c_int64),
+        ("rope_dim", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
     ]
 
 

@@ -73,6 +73,7 @@ struct dsa_indexer {
   __nv_bfloat16* WkwT = nullptr;  // [head_dim + n_heads, hidden_dim]
   float* gamma = nullptr;         // [head_dim]
   float* beta = nullptr;
+  double* inv_freq = nullptr;     // [32] rotary frequencies (rope_dim > 0)
   CUtensorMap tm_WqT, tm_WkwT;
   TopkWorkspace ws{};
   std::vector<void*> allocs;
@@ -108,6 +109,8 @@ void dsa_indexer_default_config(dsa_indexer_config_t* cfg) {
   cfg->top_k = 2048;
   cfg->ln_eps = 1e-6f;
   cfg->max_tokens = 131072;
+  cfg->rope_dim = 0;
+  cfg->rope_theta = 10000.f;
 }
 
 int32_t dsa_indexer_abi_version(void) { return DSA_INDEXER_ABI_VERSION; }
@@ -136,7 +139,11 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
     return DSA_ERR_INVALID_ARG;
   if (cfg->hidden_dim % 64 || cfg->q_latent_dim % 64) return DSA_ERR_INVALID_ARG;
   if (cfg->max_tokens > (int64_t(1) << 26)) return DSA_ERR_INVALID_ARG;
-  if (cfg->n_heads != kHeads || cfg->head_dim != kHeadDim || cfg->top_k != kTopK) return DSA_ERR_UNSUPPORTED;
+  if ((cfg->n_heads != 32 && cfg->n_heads != 64) || cfg->head_dim != kHeadDim || cfg->top_k != kTopK ||
+      (cfg->rope_dim != 0 && cfg->rope_dim != 64))
+    return DSA_ERR_UNSUPPORTED;
+  if (cfg->rope_dim > 0 && !(cfg->rope_theta > 1.f && std::isfinite(cfg->rope_theta))) return DSA_ERR_INVALID_ARG;
+  if ((cfg->n_heads == 64 || cfg->rope_dim > 0) && cfg->hidden_dim < 128) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(W_q) || !aligned16(W_k) || !aligned16(W_w) || !aligned16(ln_gamma) || !aligned16(ln_beta))
     return DSA_ERR_INVALID_ARG;
   if (!load_encode()) return DSA_ERR_CUDA;
@@ -148,10 +155,10 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
     delete h;
     return DSA_ERR_CUDA;
   }
-  const int H = kHeads, D = kHeadDim, HD = cfg->hidden_dim, QL = cfg->q_latent_dim;
+  const int H = cfg->n_heads, D = kHeadDim, HD = cfg->hidden_dim, QL = cfg->q_latent_dim;
   const int64_t T = cfg->max_tokens;
   bool ok = h->alloc(&h->WqT, size_t(H) * D * QL) && h->alloc(&h->WkwT, size_t(D + H) * HD) &&
-            h->alloc(&h->gamma, D) && h->alloc(&h->beta, D);
+            h->alloc(&h->gamma, D) && h->alloc(&h->beta, D) && h->alloc(&h->inv_freq, 32);
   TopkWorkspace& ws = h->ws;
   ws.part_tokens = static_cast<int>(T < kSplitMaxTokens ? T : kSplitMaxTokens);
   ws.max_items = static_cast<int>(T > ws.part_tokens * kMaxChunks ? T : ws.part_tokens * kMaxChunks) + 16;
@@ -196,12 +203,19 @@ dsa_status_t dsa_indexer_create(const dsa_indexer_config_t* cfg, const void* W_q
       if (e == cudaSuccess) e = cudaMemcpy(h->beta, gf + D, D * 4, cudaMemcpyHostToDevice);
     }
   }
+  if (e == cudaSuccess) {
+    // rotary frequencies theta^(-2i / rope_dim), in double precision
+    double f[32] = {};
+    for (int i = 0; i < 32 && cfg->rope_dim > 0; ++i)
+      f[i] = std::pow(static_cast<double>(cfg->rope_theta), -2.0 * i / cfg->rope_dim);
+    e = cudaMemcpy(h->inv_freq, f, sizeof(f), cudaMemcpyHostToDevice);
+  }
   if (e != cudaSuccess) {
     delete h;
     return DSA_ERR_CUDA;
   }
   if (!make_tmap(&h->tm_WqT, h->WqT, QL, uint64_t(H) * D, 64, 256) ||
-      !make_tmap(&h->tm_WkwT, h->WkwT, HD, uint64_t(D + H), 64, 160)) {
+      !make_tmap(&h->tm_WkwT, h->WkwT, HD, uint64_t(D + H), 64, D + H)) {
     delete h;
     return DSA_ERR_CUDA;
   }
@@ -240,7 +254,8 @@ dsa_status_t project_impl(dsa_indexer_t h, int64_t T, const void* hidden, const 
     return DSA_ERR_INVALID_ARG;
   if (cache_rows < 1 || cache_rows > (int64_t(1) << 31) - (int64_t(1) << 20)) return DSA_ERR_INVALID_ARG;
   const dsa_indexer_config_t& c = h->cfg;
-  if (fp8 && c.hidden_dim < 128) return DSA_ERR_UNSUPPORTED;   // the FP8 key epilogue is the split-K one
+  // FP8: the K3.1 form (32 heads, no rotary step), whose key epilogue is the split-K one
+  if (fp8 && (c.hidden_dim < 128 || c.n_heads != 32 || c.rope_dim != 0)) return DSA_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   CUtensorMap tmX, tmQL;
   if (!make_tmap(&tmX, hidden, c.hidden_dim, uint64_t(T), 64, 128) ||
@@ -257,6 +272,9 @@ dsa_status_t project_impl(dsa_indexer_t h, int64_t T, const void* hidden, const 
   e.q_seq_offsets = q_seq_offsets;
   e.B = B;
   e.cache_offsets = cache_offsets;
+  e.n_heads = c.n_heads;
+  e.rope_dim = c.rope_dim;
+  e.inv_freq = h->inv_freq;
   e.gamma = h->gamma;
   e.beta = h->beta;
   e.eps = c.ln_eps;
@@ -270,8 +288,9 @@ dsa_status_t project_impl(dsa_indexer_t h, int64_t T, const void* hidden, const 
   const cudaError_t eq =
       fp8 ? launch_proj_q8(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
                            static_cast<uint8_t*>(q_out), q_scale, h->ws.err, timeout_ns(), s)
-          : launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, kHeads * kHeadDim,
-                          static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s);
+          : launch_proj_q(tmQL, h->tm_WqT, static_cast<int>(T), c.q_latent_dim, c.n_heads * kHeadDim,
+                          static_cast<__nv_bfloat16*>(q_out), h->ws.err, timeout_ns(), s, positions, h->inv_freq,
+                          c.rope_dim);
   // join even if a launch failed, so that the side stream never runs ahead unordered
   if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess || cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess)
     return DSA_ERR_CUDA;
@@ -294,6 +313,8 @@ dsa_status_t topk_impl(dsa_indexer_t h, int64_t T, const void* q, const float* q
   if (fp8 && (!q_scale || !key_scale || (reinterpret_cast<uintptr_t>(q_scale) & 3) ||
               (reinterpret_cast<uintptr_t>(key_scale) & 3)))
     return DSA_ERR_INVALID_ARG;
+  const int H = h->cfg.n_heads;
+  if (fp8 && H != 32) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(w) || !aligned16(key_cache) || !aligned16(idx_out) ||
       (score_out && !aligned16(score_out)) || (reinterpret_cast<uintptr_t>(positions) & 3) ||
       (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7))
@@ -309,8 +330,9 @@ dsa_status_t topk_impl(dsa_indexer_t h, int64_t T, const void* q, const float* q
   // a box row is 128 bytes: 64 bf16 (two boxes per 128-dim row) or 128 FP8 codes (one)
   const uint32_t bi = fp8 ? 128 : 64;
   CUtensorMap tmQ1, tmQ8, tmK;
-  if (!make_tmap(&tmQ1, q, kHeadDim, uint64_t(T) * kHeads, bi, kHeads, fp8) ||
-      !make_tmap(&tmQ8, q, kHeadDim, uint64_t(T) * kHeads, bi, kHeads * kPrefillQ, fp8) ||
+  // an item of the prefill path holds 256 (query, head) rows: 8 queries of 32 heads or 4 of 64
+  if (!make_tmap(&tmQ1, q, kHeadDim, uint64_t(T) * H, bi, H, fp8) ||
+      !make_tmap(&tmQ8, q, kHeadDim, uint64_t(T) * H, bi, 256, fp8) ||
       !make_tmap(&tmK, key_cache, kHeadDim, uint64_t(cache_rows), bi, kKeyTile, fp8))
     return DSA_ERR_INVALID_ARG;
   TopkArgs a{};
@@ -328,6 +350,7 @@ dsa_status_t topk_impl(dsa_indexer_t h, int64_t T, const void* q, const float* q
   a.split = split;
   a.sorted = (flags & DSA_TOPK_SORTED) != 0;
   a.fp8 = fp8;
+  a.heads = H;
   a.q_scale = fp8 ? q_scale : nullptr;
   a.key_scale = fp8 ? key_scale : nullptr;
   a.timeout_ns = timeout_ns();

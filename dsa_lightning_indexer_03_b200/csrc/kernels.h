@@ -22,6 +22,9 @@ struct ProjKwEpilogue {
   const int64_t* cache_offsets;   // [B+1]
   uint8_t* key8;                  // FP8 cache instead of key_cache when set: e4m3 codes [cache_rows, 128]
   float* key_scale;               // FP8 cache: [cache_rows] scale of each row
+  int n_heads;                    // 32 or 64: head-weight columns after the 128 key columns
+  int rope_dim;                   // rotated dims at the start of the key (0: none)
+  const double* inv_freq;         // rotary frequencies, rope_dim / 2 of them
   const float* gamma;             // [128]
   const float* beta;              // [128]
   float eps;
@@ -29,11 +32,14 @@ struct ProjKwEpilogue {
   uint64_t timeout_ns;
 };
 
-// q_out[M, 4096] = bf16(A[M,K] * Bt[4096,K]^T); tmA box {64,128}, tmB box {64,256}
+// q_out[M, N] = bf16(RoPE(A[M,K] * Bt[N,K]^T)); tmA box {64,128}, tmB box {64,256}; with
+// rope_dim > 0 the first rope_dim dims of every 128-dim head turn by positions[m] * inv_freq[i]
 cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N,
-                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s);
+                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s,
+                          const int32_t* positions = nullptr, const double* inv_freq = nullptr, int rope_dim = 0);
 
-// [k~ | w] = A[M,K] * Bt[160,K]^T with the key LayerNorm / scatter epilogue; tmB box {64,160}
+// [k~ | w] = A[M,K] * Bt[128+H,K]^T with the key LayerNorm (+ RoPE) / scatter epilogue;
+// tmB box {64, 128+H}
 cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K, const ProjKwEpilogue& e,
                            cudaStream_t s);
 
@@ -61,7 +67,7 @@ constexpr int kCandStride = 2 * kTopK + 4 * kWarpApp;  // keep 0 | keep 1 | area
 constexpr int kMaxChunks = 16;                 // key chunks per query on the split-key path
 constexpr int kMinChunk = 4096;                // shortest key chunk on the split-key path
 constexpr int kSplitMaxTokens = 256;           // split-key path is offered up to this many queries
-constexpr int kPrefillQ = 8;                   // queries per work item on the prefill path
+constexpr int kPrefillQ = 8;                   // queries per work item on the prefill path (32 heads)
 
 struct WorkItem {
   int32_t t0;       // first query token
@@ -103,6 +109,7 @@ struct TopkArgs {
   float* score_out;
   bool split;
   bool sorted;       // order each row by (score desc, position asc); short rows stay [0..p, -1...]
+  int heads;         // 32, or 64 (bf16 only)
   bool fp8;          // q and key_cache hold FP8 e4m3 codes with the scales below
   const float* q_scale;    // FP8: [T, 32] per query head
   const float* key_scale;  // FP8: [cache_rows] per key row

@@ -140,6 +140,7 @@ extern "C" dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const
   a.split = false;
   a.sorted = false;
   a.fp8 = false;
+  a.heads = kHeads;
   a.timeout_ns = wait_timeout_ns();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the error word keeps the previous call's bits: start each call from zero

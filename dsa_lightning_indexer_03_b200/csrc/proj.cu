@@ -37,6 +37,9 @@ struct ProjParams {
   int ldq;
   uint8_t* q8_out;       // EPI_Q8: FP8 e4m3 codes [M, ldq]
   float* q_scale;        // EPI_Q8: [M, ldq / 128], one scale per query head
+  const int32_t* positions;   // EPI_Q with rope_dim > 0: token positions [M]
+  const double* inv_freq;     // rotary frequencies theta^(-2i / rope_dim), i < rope_dim / 2
+  int rope_dim;               // rotated dims at the start of each 128-dim head (0: none)
   ProjKwEpilogue kw;     // EPI_KW
   int* err;
   uint64_t timeout_ns;
@@ -58,6 +61,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 }
 
 __device__ __forceinline__ float round_bf16(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+// cos and sin of the rotary angle pos * inv_freq: the angle is formed and reduced to
+// [-pi, pi] in double precision (positions reach 10^6 radians), then sincosf.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
+  const double ang = static_cast<double>(pos) * inv_freq;
+  const double r = ang - 6.283185307179586 * rint(ang * 0.15915494309189535);
+  sincosf(static_cast<float>(r), s, c);
+}
+
+// Rotates the pairs (x[2m], x[2m+1]) of a run of N values that starts at dim d0 of a head:
+// pair i = d0/2 + m turns by pos * inv_freq[i] when 2i < rope_dim.
+template <int N>
+__device__ __forceinline__ void rope_rotate(float (&x)[N], int d0, int pos, const double* inv_freq, int rope_dim) {
+#pragma unroll
+  for (int m = 0; m < N / 2; ++m) {
+    const int i = d0 / 2 + m;
+    if (2 * i < rope_dim) {
+      float c, sn;
+      rope_cos_sin(pos, inv_freq[i], &c, &sn);
+      const float a = x[2 * m], b = x[2 * m + 1];
+      x[2 * m] = a * c - b * sn;
+      x[2 * m + 1] = a * sn + b * c;
+    }
+  }
+}
 
 // FP8 e4m3 codes of four values (round to nearest even, saturating at +-448), first value
 // in the lowest byte.
@@ -183,6 +211,15 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t r[32];
           tmem_ld_32cols(tbase + c * 32, r);
           tmem_ld_wait(r);
+          const int hd0 = (n0 + c * 32) & 127;   // first dim of this chunk inside its head
+          if (p.rope_dim > 0 && hd0 < p.rope_dim && row < p.M) {
+            float x[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(r[i]);
+            rope_rotate<32>(x, hd0, p.positions[row], p.inv_freq, p.rope_dim);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(x[i]);
+          }
           if (row < p.M) {
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
@@ -317,7 +354,6 @@ __global__ void __launch_bounds__(192, 1)
 // scatter to those rows and stores their head weights.  Each row is handled by CS threads
 // (128/CS key columns and 32/CS weight columns each); the LayerNorm's sums over the row are
 // shuffles inside those CS lanes.
-constexpr int kPartStride = 164;   // floats per row of the partial tile (conflict-free float4 stores)
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -341,18 +377,20 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
-template <int CS, int STAGES>
+template <int CS, int STAGES, int H>
 __global__ void __launch_bounds__(192, 1)
     proj_kw_cluster_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            ProjParams p) {
-  constexpr int BN = 160;
+  constexpr int BN = 128 + H;              // key columns, then the H head-weight columns
+  constexpr int kPartStride = BN + 4;      // floats per row of the partial tile (conflict-free float4 stores)
   constexpr int kRows = kBM / CS;        // rows of the tile this CTA finishes
   constexpr int kKeyCols = 128 / CS;     // key columns per thread
-  constexpr int kWCols = 32 / CS;        // weight columns per thread
+  constexpr int kWCols = H / CS;         // weight columns per thread
   static_assert(CS == 2 || CS == 4 || CS == 8, "cluster of 2, 4 or 8");
   static_assert(kBM * kPartStride * 4 <= STAGES * ProjSmem<BN, STAGES>::kStageBytes, "partial fits the ring");
   using L = ProjSmem<BN, STAGES>;
   constexpr uint32_t kTmemCols = 256;
+  static_assert(BN <= 256 && BN % 16 == 0, "one MMA covers the key and weight columns");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -507,24 +545,30 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
     for (int o = 1; o < CS; o <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float rstd = rsqrtf(ss * (1.0f / 128.0f) + p.kw.eps);
-    // FP8 cache: k = bf16(LayerNorm), then e4m3 codes with the row's scale (the shuffles run
-    // on every lane, before the per-token branch)
+    // the key: y = LayerNorm (fp32), rotary step on its first rope_dim dims, then bf16; the
+    // FP8 cache stores e4m3 codes of the bf16 key with the row's scale (the shuffles run on
+    // every lane, before the per-token branch)
+    const int tok = m0 + trow;
+    float y[kKeyCols];
+#pragma unroll
+    for (int i = 0; i < kKeyCols; ++i) {
+      const int d = t * kKeyCols + i;
+      y[i] = fmaf((xk[i] - mean) * rstd, s_gamma[d], s_beta[d]);
+    }
+    if (p.kw.rope_dim > 0 && tok < p.M)
+      rope_rotate<kKeyCols>(y, t * kKeyCols, p.kw.positions[tok], p.kw.inv_freq, p.kw.rope_dim);
+#pragma unroll
+    for (int i = 0; i < kKeyCols; ++i) y[i] = round_bf16(y[i]);
     const bool fp8 = p.kw.key8 != nullptr;
-    float y8[kKeyCols];
     float scale8 = 0.f, inv8 = 0.f;
     if (fp8) {
       float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < kKeyCols; ++i) {
-        const int d = t * kKeyCols + i;
-        y8[i] = round_bf16(fmaf((xk[i] - mean) * rstd, s_gamma[d], s_beta[d]));
-        amax = fmaxf(amax, fabsf(y8[i]));
-      }
+      for (int i = 0; i < kKeyCols; ++i) amax = fmaxf(amax, fabsf(y[i]));
 #pragma unroll
       for (int o = 1; o < CS; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       fp8_row_scale(amax, &scale8, &inv8);
     }
-    const int tok = m0 + trow;
     if (tok < p.M) {
       const int pos = p.kw.positions[tok];
       int lo = 0, hi = p.kw.B - 1;   // sequence of the token: the last b with q_seq_offsets[b] <= tok
@@ -536,40 +580,30 @@ __global__ void __launch_bounds__(192, 1)
       const int64_t cb = p.kw.cache_offsets[lo];
       const int64_t len = p.kw.cache_offsets[lo + 1] - cb;
       const bool in_cache = pos >= 0 && pos < len && cb >= 0 && cb + pos < p.kw.cache_rows;
-      if (fp8) {
-        if (in_cache) {
-          uint32_t* d32 = reinterpret_cast<uint32_t*>(p.kw.key8 + static_cast<size_t>(cb + pos) * kHeadDim +
-                                                      t * kKeyCols);
+      if (!in_cache) {
+        if (t == 0) atomicOr(p.err, kErrBounds);
+      } else if (fp8) {
+        uint32_t* d32 = reinterpret_cast<uint32_t*>(p.kw.key8 + static_cast<size_t>(cb + pos) * kHeadDim +
+                                                    t * kKeyCols);
 #pragma unroll
-          for (int v = 0; v < kKeyCols / 4; ++v)
-            d32[v] = pack_e4m3x4(__fmul_rn(y8[4 * v], inv8), __fmul_rn(y8[4 * v + 1], inv8),
-                                 __fmul_rn(y8[4 * v + 2], inv8), __fmul_rn(y8[4 * v + 3], inv8));
-          if (t == 0) p.kw.key_scale[cb + pos] = scale8;
-        } else if (t == 0) {
-          atomicOr(p.err, kErrBounds);
-        }
-      } else if (in_cache) {
+        for (int v = 0; v < kKeyCols / 4; ++v)
+          d32[v] = pack_e4m3x4(__fmul_rn(y[4 * v], inv8), __fmul_rn(y[4 * v + 1], inv8),
+                               __fmul_rn(y[4 * v + 2], inv8), __fmul_rn(y[4 * v + 3], inv8));
+        if (t == 0) p.kw.key_scale[cb + pos] = scale8;
+      } else {
         uint4* d4 = reinterpret_cast<uint4*>(p.kw.key_cache + static_cast<size_t>(cb + pos) * kHeadDim +
                                              t * kKeyCols);
 #pragma unroll
         for (int v = 0; v < kKeyCols / 8; ++v) {
-          float y[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int d = t * kKeyCols + 8 * v + i;
-            y[i] = fmaf((xk[8 * v + i] - mean) * rstd, s_gamma[d], s_beta[d]);
-          }
           uint4 pk;
-          pk.x = pack_bf16x2(y[0], y[1]);
-          pk.y = pack_bf16x2(y[2], y[3]);
-          pk.z = pack_bf16x2(y[4], y[5]);
-          pk.w = pack_bf16x2(y[6], y[7]);
+          pk.x = pack_bf16x2(y[8 * v], y[8 * v + 1]);
+          pk.y = pack_bf16x2(y[8 * v + 2], y[8 * v + 3]);
+          pk.z = pack_bf16x2(y[8 * v + 4], y[8 * v + 5]);
+          pk.w = pack_bf16x2(y[8 * v + 6], y[8 * v + 7]);
           d4[v] = pk;
         }
-      } else if (t == 0) {
-        atomicOr(p.err, kErrBounds);
       }
-      float4* w4 = reinterpret_cast<float4*>(p.kw.w_out + static_cast<size_t>(tok) * kHeads + t * kWCols);
+      float4* w4 = reinterpret_cast<float4*>(p.kw.w_out + static_cast<size_t>(tok) * H + t * kWCols);
 #pragma unroll
       for (int v = 0; v < kWCols / 4; ++v)
         w4[v] = make_float4(xw[4 * v], xw[4 * v + 1], xw[4 * v + 2], xw[4 * v + 3]);
@@ -663,8 +697,12 @@ cudaError_t launch_proj(const CUtensorMap& tmA, const CUtensorMap& tmB, const Pr
 }  // namespace
 
 cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N,
-                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s) {
+                          __nv_bfloat16* q_out, int* err, uint64_t timeout_ns, cudaStream_t s,
+                          const int32_t* positions, const double* inv_freq, int rope_dim) {
   ProjParams p{};
+  p.positions = positions;
+  p.inv_freq = inv_freq;
+  p.rope_dim = rope_dim;
   p.M = M;
   p.K = K;
   p.q_out = q_out;
@@ -674,10 +712,10 @@ cudaError_t launch_proj_q(const CUtensorMap& tmA, const CUtensorMap& tmB, int M,
   return launch_proj<256, 4, EPI_Q>(tmA, tmB, p, N / 256, s);
 }
 
-template <int CS>
+template <int CS, int H>
 cudaError_t launch_kw_cluster(const CUtensorMap& tmA, const CUtensorMap& tmB, const ProjParams& p, cudaStream_t s) {
-  using L = ProjSmem<160, 5>;
-  auto kern = proj_kw_cluster_kernel<CS, 5>;
+  using L = ProjSmem<128 + H, 5>;
+  auto kern = proj_kw_cluster_kernel<CS, 5, H>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -705,9 +743,15 @@ cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K
   p.timeout_ns = e.timeout_ns;
   const int nk = K / kBK;
   // the contraction is split over a cluster of CTAs when it is long enough to share
-  if (nk >= 8) return launch_kw_cluster<8>(tmA, tmB, p, s);
-  if (nk >= 4) return launch_kw_cluster<4>(tmA, tmB, p, s);
-  if (nk >= 2) return launch_kw_cluster<2>(tmA, tmB, p, s);
+  if (e.n_heads == 64) {
+    if (nk >= 8) return launch_kw_cluster<8, 64>(tmA, tmB, p, s);
+    if (nk >= 4) return launch_kw_cluster<4, 64>(tmA, tmB, p, s);
+    if (nk >= 2) return launch_kw_cluster<2, 64>(tmA, tmB, p, s);
+    return cudaErrorInvalidValue;
+  }
+  if (nk >= 8) return launch_kw_cluster<8, 32>(tmA, tmB, p, s);
+  if (nk >= 4) return launch_kw_cluster<4, 32>(tmA, tmB, p, s);
+  if (nk >= 2) return launch_kw_cluster<2, 32>(tmA, tmB, p, s);
   return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
 }
 

@@ -599,13 +599,13 @@ __device__ void sort_stage_and_emit(uint2* stage, int tid, int bar, int32_t* oi,
 }
 
 // ------------------------------------------------------------------------------------------
-template <int QPW>
+template <int QPW, int H>
 struct WGState {
   uint32_t hist[QPW][kBins1 / 2];  // per query: first-level counts of its candidates (packed)
   uint32_t rhist[kBins1 / 2];      // resolution scratch
   uint2 list[kListCap];            // boundary-bin candidates of one resolution
   uint32_t small[kSmallRank];      // keys of the boundary sub-bin
-  float w[QPW][kHeads];
+  float w[QPW][H];
   int cnt_w[QPW][4];               // per-warp append counts, published at check points
   int cnt_k[QPW];                  // entries in the current keep set
   int kcur[QPW];                   // which keep set is current
@@ -625,8 +625,11 @@ struct WGState {
 // queries (ALT = false) or, with ALT, take whole items in turn (group g takes the items
 // the CTA receives at positions g, g + 2, ...): one group's end-of-item selection then
 // overlaps the other group's tiles.
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, int EB = 2>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, int EB = 2, int H = kHeads>
 struct ScoreCfg {
+  // H = indexer heads (32, or 64 for the DeepSeek-V3.2 form); a query's H columns of the
+  // accumulator are H / 32 blocks of 32.
+  static constexpr int kHB = H / 32;
   // EB = bytes per element of q and of the keys: 2 (bf16, kind::f16 MMA) or 1 (FP8 e4m3,
   // kind::f8f6f4 MMA).  A 128-dim row is EB 128-byte swizzle rows ("halves") wide.
   static constexpr int kHalves = EB;
@@ -639,18 +642,18 @@ struct ScoreCfg {
   static constexpr bool kRegSplit = EW == 8;
   static constexpr int kCtrlRegs = 32;                // per thread of warps 0-3 after the split
   static constexpr int kEpiRegs = 112;                // per epilogue thread after the split
-  static constexpr int kAccCols = QMAX * kHeads;
+  static constexpr int kAccCols = QMAX * H;
   static constexpr int kTotalBufs = ALT ? NWG * ACC_BUFS : ACC_BUFS;  // with ALT each group has its own
   static constexpr int kTmemNeed = kTotalBufs * kAccCols;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kQHalf = QMAX * kHeads * 128;  // bytes of one 128-byte-wide half of the Q tile
+  static constexpr int kQHalf = QMAX * H * 128;       // bytes of one 128-byte-wide half of the Q tile
   static constexpr int kKHalf = kKeyTile * 128;       // 16 KB
   static constexpr int kKStage = kHalves * kKHalf;
   static constexpr int kQOff = 0;
   static constexpr int kKOff = kHalves * kQHalf;
   static constexpr int kWGOff = kKOff + STAGES * kKStage;
-  static constexpr int kWGBytes = (static_cast<int>(sizeof(WGState<kQPW>)) + 15) / 16 * 16;
+  static constexpr int kWGBytes = (static_cast<int>(sizeof(WGState<kQPW, H>)) + 15) / 16 * 16;
   static constexpr int kBarOff = kWGOff + NWG * kWGBytes;
   static constexpr int kNumBars = 2 * STAGES + 2 * kTotalBufs + 2 + 4 + 1;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;
@@ -661,6 +664,7 @@ struct ScoreCfg {
   static_assert(kQPH >= 1 && kQPH * (EW / 4) == kQPW, "queries split evenly over a quadrant's warps");
   static_assert(kCtrlRegs % 8 == 0 && kEpiRegs % 8 == 0, "setmaxnreg takes multiples of 8");
   static_assert(!ALT || NWG == 2, "alternating items need two epilogue groups");
+  static_assert(H % 32 == 0 && QMAX * H <= 256, "an item's (query, head) columns fit one MMA");
 };
 
 // The four threads t, t^1, t^2, t^3 hold partial sums over disjoint head sets for the same
@@ -686,11 +690,12 @@ __device__ __forceinline__ void sum_over_quad(const float (&part)[4 * QPH], floa
   }
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB>
-__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>::kThreads, 1)
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB, int H>
+__global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB, H>::kThreads, 1)
     score_topk_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       ScoreParams p) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB, H>;
+  constexpr int HB = C::kHB;
   constexpr bool kFp8 = EB == 1;
   constexpr int QPW = C::kQPW;
   constexpr int QPH = C::kQPH;
@@ -785,8 +790,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         if (kt1 <= kt0) continue;
         if (qloads > 0 && !mbar_wait(q_empty, (qloads - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(q_full, C::kHalves * C::kQHalf);
-        tma_load_2d_hint(sQ, &tmQ, q_full, 0, wi.t0 * kHeads, pol_q);
-        if constexpr (!kFp8) tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * kHeads, pol_q);
+        tma_load_2d_hint(sQ, &tmQ, q_full, 0, wi.t0 * H, pol_q);
+        if constexpr (!kFp8) tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * H, pol_q);
         ++qloads;
         const int row0 = static_cast<int>(p.cache_offsets[wi.b]);
         bool ok = true;
@@ -827,7 +832,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         if (!mbar_wait(q_full, qloads & 1, wc)) break;
         ++qloads;
         tc_fence_after();
-        const uint32_t idesc = kFp8 ? umma_idesc_e4m3(kKeyTile, wi.nq * kHeads) : umma_idesc_bf16(kKeyTile, wi.nq * kHeads);
+        const uint32_t idesc = kFp8 ? umma_idesc_e4m3(kKeyTile, wi.nq * H) : umma_idesc_bf16(kKeyTile, wi.nq * H);
         const bool second = ALT && (local & 1);   // with ALT, the CTA's odd items go to group 1
         bool ok = true;
         for (int kt = kt0; kt < kt1; ++kt, ++kstage) {
@@ -870,7 +875,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
     // key row of this thread inside a tile (the row whose scores it holds after sum_over_quad)
     const int r = qd * 32 + (lane >> 2) + 8 * ((lane >> 1) & 1) + 16 * (lane & 1);
     const uint32_t lt = lanemask_lt();
-    WGState<QPW>& st = *reinterpret_cast<WGState<QPW>*>(smem + C::kWGOff + g * C::kWGBytes);
+    WGState<QPW, H>& st = *reinterpret_cast<WGState<QPW, H>*>(smem + C::kWGOff + g * C::kWGBytes);
     const uint32_t tlane = tmem + (static_cast<uint32_t>(qd * 32) << 16);
     const int j0 = hq * QPH;                 // first of this warp's queries inside the group
     // candidates of query jj of this group start at qcand + jj * kCandStride
@@ -919,11 +924,11 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         for (int w = 0; w < 4; ++w) st.cnt_w[gtid][w] = 0;
       }
       if (it >= 0) {
-        for (int i = gtid; i < QPW * kHeads; i += NTG) {
-          const int jj = i / kHeads, j = qbase + jj;
-          const size_t wix = static_cast<size_t>(wi.t0 + j) * kHeads + (i % kHeads);
+        for (int i = gtid; i < QPW * H; i += NTG) {
+          const int jj = i / H, j = qbase + jj;
+          const size_t wix = static_cast<size_t>(wi.t0 + j) * H + (i % H);
           // FP8: the query head's scale joins its weight (sum_h w_h s_h ReLU(q8_h . k8))
-          st.w[jj][i % kHeads] = (j < wi.nq) ? (kFp8 ? p.w[wix] * p.q_scale[wix] : p.w[wix]) : 0.f;
+          st.w[jj][i % H] = (j < wi.nq) ? (kFp8 ? p.w[wix] * p.q_scale[wix] : p.w[wix]) : 0.f;
         }
       }
       if (named_bar_or(bar, NTG, it < 0)) break;   // every thread of the group leaves together
@@ -942,47 +947,56 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         thr_r[j] = 0u;
         pos_r[j] = (j < nmine) ? min(st.pos[j0 + j], wi.k_end - 1) : -2;   // last key position scored
       }
-      // this thread's head weights: heads 8 blk + 2 (lane % 4) + {0, 1} of each of its queries
-      float2 w2[QPH][4];
+      // this thread's head weights: heads 32 hb + 8 blk + 2 (lane % 4) + {0, 1} of each of its
+      // queries (hb = head block)
+      float2 w2[QPH * HB][4];
 #pragma unroll
       for (int j = 0; j < QPH; ++j)
 #pragma unroll
-        for (int blk = 0; blk < 4; ++blk)
-          w2[j][blk] = *reinterpret_cast<const float2*>(&st.w[j0 + j][8 * blk + 2 * (lane & 3)]);
+        for (int hb = 0; hb < HB; ++hb)
+#pragma unroll
+          for (int blk = 0; blk < 4; ++blk)
+            w2[j * HB + hb][blk] = *reinterpret_cast<const float2*>(&st.w[j0 + j][32 * hb + 8 * blk + 2 * (lane & 3)]);
       bool failed = false;
       for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
         const int ab = (ALT ? g * ACC_BUFS : 0) + acc_ctr % ACC_BUFS;   // this group's ring
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (acc_ctr / ACC_BUFS) & 1, wc));
         tc_fence_after();
         const int s_pos = kt * kKeyTile + r;
-        const uint32_t tcol = tlane + ab * C::kAccCols + (qbase + j0) * kHeads;
+        const uint32_t tcol = tlane + ab * C::kAccCols + (qbase + j0) * H;
         if (ok) {
-          // this warp's columns of the tile, as 16x256b blocks: one TMEM round trip per tile
-          uint32_t v[2 * QPH][16];   // [lane half h][query j] at h * QPH + j
+          // this warp's columns of the tile, as 16x256b blocks of 32 columns (CB of them: its
+          // queries' head blocks, contiguous): one TMEM round trip per tile
+          constexpr int CB = QPH * HB;
+          uint32_t v[2 * CB][16];   // [lane half h][column block cb] at h * CB + cb
           constexpr uint32_t kHalf16 = 16u << 16;   // lane offset of the quadrant's upper half
-          if constexpr (QPH == 2) {
-            tmem_ld4_16x256b_x4_wait(tcol, tcol + kHeads, tcol + kHalf16, tcol + kHalf16 + kHeads, v);
+          if constexpr (CB == 2) {
+            tmem_ld4_16x256b_x4_wait(tcol, tcol + 32, tcol + kHalf16, tcol + kHalf16 + 32, v);
           } else {
-            static_assert(QPH == 1, "one or two queries per epilogue warp");
+            static_assert(CB == 1, "one or two column blocks per epilogue warp");
             tmem_ld2_16x256b_x4_wait(tcol, tcol + kHalf16, v);
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
-          // partial sums over this thread's 8 heads, for its two rows of each lane half
+          // partial sums over this thread's 8 heads of each head block, for its two rows of
+          // each lane half
           float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
-              const uint32_t(&x)[16] = v[h * QPH + j];
               float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
 #pragma unroll
-              for (int blk = 0; blk < 4; ++blk) {
-                a = ffma2(w2[j][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
-                                                  fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
-                b = ffma2(w2[j][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
-                                                  fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
+              for (int hb = 0; hb < HB; ++hb) {
+                const uint32_t(&x)[16] = v[h * CB + j * HB + hb];
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                  a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
+                                                              fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
+                  b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
+                                                              fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
+                }
               }
               part[(2 * h) * QPH + j] = a.x + a.y;
               part[(2 * h + 1) * QPH + j] = b.x + b.y;
@@ -1372,6 +1386,7 @@ struct PrepParams {
   const int64_t* cache_offsets;
   int split;
   int num_sms;
+  int qpi;            // queries per work item on the prefill path (256 / heads)
   int32_t* idx_out;   // [T, kTopK]: every row is padded when the offsets are malformed
   float* score_out;   // [T, kTopK] or null
   TopkWorkspace ws;
@@ -1521,7 +1536,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       ws.tok_nchunks[o] = c;
     } else {
       const int nq = qoff[o + 1] - qoff[o];
-      c = (nq + kPrefillQ - 1) / kPrefillQ;
+      c = (nq + p.qpi - 1) / p.qpi;
     }
     base[o] = c;
   }
@@ -1552,8 +1567,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       wi.chunk = (nch > 1) ? local : -1;
     } else {
       const int b = o;
-      const int t0 = qoff[b] + local * kPrefillQ;
-      const int nq = min(kPrefillQ, qoff[b + 1] - t0);
+      const int t0 = qoff[b] + local * p.qpi;
+      const int nq = min(p.qpi, qoff[b + 1] - t0);
       int kend = 0;
       for (int j = 0; j < nq; ++j) kend = max(kend, ws.pos_eff[t0 + j] + 1);
       wi.t0 = t0;
@@ -1582,11 +1597,11 @@ __global__ void wait_timeout_selftest_kernel(int* status, uint64_t timeout_ns) {
   *status = ok ? 0 : ((err & kErrTimeout) ? 2 : 1);
 }
 
-template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB>
+template <int QMAX, int STAGES, int ACC_BUFS, int NWG, int EW, bool ALT, bool SORTED, int EB, int H = kHeads>
 cudaError_t launch_score(const CUtensorMap& tmQ, const CUtensorMap& tmK, const ScoreParams& p, int grid,
                          cudaStream_t s) {
-  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB>;
-  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, SORTED, EB>;
+  using C = ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, EB, H>;
+  auto kern = score_topk_kernel<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT, SORTED, EB, H>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   if (C::kRegSplit) {
@@ -1628,6 +1643,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   pp.cache_offsets = a.cache_offsets;
   pp.split = a.split ? 1 : 0;
   pp.num_sms = num_sms;
+  pp.qpi = 256 / a.heads;
   pp.idx_out = a.idx_out;
   pp.score_out = a.score_out;
   pp.ws = ws;
@@ -1654,7 +1670,10 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
   sp.timeout_ns = a.timeout_ns;
   const int grid = num_sms < ws.cand_slots ? num_sms : ws.cand_slots;
   if (a.split) {
-    if (a.fp8)   // 16 KB key tiles: twice the stages keep the same bytes in flight
+    if (a.heads == 64)
+      e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true, 2, 64>(tmQ1, tmK, sp, grid, s)
+                   : launch_score<1, 5, 4, 2, 4, true, false, 2, 64>(tmQ1, tmK, sp, grid, s);
+    else if (a.fp8)   // 16 KB key tiles: twice the stages keep the same bytes in flight
       e = a.sorted ? launch_score<1, 10, 4, 2, 4, true, true, 1>(tmQ1, tmK, sp, grid, s)
                    : launch_score<1, 10, 4, 2, 4, true, false, 1>(tmQ1, tmK, sp, grid, s);
     else
@@ -1680,6 +1699,9 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
                               static_cast<const int32_t*>(ws.part_idx), static_cast<const int*>(ws.tok_nchunks),
                               ws.part_hist, a.idx_out, a.score_out, a.sorted ? 1 : 0);
   }
+  if (a.heads == 64)   // four queries x 64 heads per item
+    return a.sorted ? launch_score<4, 3, 2, 2, 8, false, true, 2, 64>(tmQ8, tmK, sp, grid, s)
+                    : launch_score<4, 3, 2, 2, 8, false, false, 2, 64>(tmQ8, tmK, sp, grid, s);
   if (a.fp8)
     return a.sorted ? launch_score<kPrefillQ, 6, 2, 2, 8, false, true, 1>(tmQ8, tmK, sp, grid, s)
                     : launch_score<kPrefillQ, 6, 2, 2, 8, false, false, 1>(tmQ8, tmK, sp, grid, s);

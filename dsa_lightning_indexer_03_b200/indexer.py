@@ -38,7 +38,10 @@ class Indexer:
     """One layer's DSA lightning indexer (owns a C handle)."""
 
     def __init__(self, W_q: torch.Tensor, W_k: torch.Tensor, W_w: torch.Tensor, ln_gamma: torch.Tensor,
-                 ln_beta: torch.Tensor, *, ln_eps: float = 1e-6, max_tokens: int = 131072):
+                 ln_beta: torch.Tensor, *, ln_eps: float = 1e-6, max_tokens: int = 131072, rope_dim: int = 0,
+                 rope_theta: float = 10000.0):
+        """The head count comes from W_w ([hidden, n_heads]: 32, or 64 for the DeepSeek-V3.2
+        form); rope_dim = 64 adds that form's rotary step on the first 64 dims of q and k."""
         self._lib = _lib.load()
         dev = W_q.device
         if dev.type != "cuda":
@@ -53,6 +56,8 @@ class Indexer:
         cfg.head_dim = W_k.shape[1]
         cfg.ln_eps = float(ln_eps)
         cfg.max_tokens = int(max_tokens)
+        cfg.rope_dim = int(rope_dim)
+        cfg.rope_theta = float(rope_theta)
         self.cfg = cfg
         self.device = dev
         self.n_heads = cfg.n_heads

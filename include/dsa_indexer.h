@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define DSA_INDEXER_ABI_VERSION 1
+#define DSA_INDEXER_ABI_VERSION 2
 
 typedef enum {
   DSA_OK = 0,
@@ -62,26 +62,34 @@ typedef enum {
 
 typedef struct dsa_indexer* dsa_indexer_t;
 
-/* Create-time configuration.  Only n_heads = 32, head_dim = 128 and
- * top_k = 2048 are implemented (other values: DSA_ERR_UNSUPPORTED);
- * hidden_dim and q_latent_dim must be positive multiples of 64. */
+/* Create-time configuration.  head_dim = 128 and top_k = 2048; n_heads = 32
+ * (Kimi K3.1 Pro) or 64 (the DeepSeek-V3.2 form: 'Sparse / compressed attn'
+ * row, "DeepSeek-V3.2's indexer has 64 heads"); rope_dim = 0 (Kimi K3.1 Pro:
+ * index_rope_dim = 0) or 64 ('Partial RoPE / NoPE' row of the page "Kimi K3.1
+ * Pro vs Gemma 4 31B": DeepSeek-V3.2's indexer rotates 64 of its 128 dims).
+ * Other values: DSA_ERR_UNSUPPORTED.  hidden_dim and q_latent_dim must be
+ * positive multiples of 64 (hidden_dim >= 128 for n_heads = 64 or rope_dim > 0). */
 typedef struct {
   int32_t hidden_dim;    /* 7168: width of the hidden state feeding W_k and W_w */
   int32_t q_latent_dim;  /* 1536: width of the MLA query latent feeding W_q */
-  int32_t n_heads;       /* 32 */
+  int32_t n_heads;       /* 32 (64: DeepSeek-V3.2 form) */
   int32_t head_dim;      /* 128 */
   int32_t top_k;         /* 2048 */
   float ln_eps;          /* LayerNorm epsilon of the key norm; 1e-6 by default */
   int64_t max_tokens;    /* largest T passed to _topk; sizes the handle's workspace */
+  int32_t rope_dim;      /* 0, or 64: rotated dims at the start of q's heads and of k */
+  float rope_theta;      /* rotary base: pair i of a token at position p turns by
+                            p * rope_theta^(-2i / rope_dim); 10000 by default */
 } dsa_indexer_config_t;
 
-/* Fills *cfg with the Kimi K3.1 Pro indexer dimensions (above) and
- * max_tokens = 131072. */
+/* Fills *cfg with the Kimi K3.1 Pro indexer dimensions (above), rope_dim = 0,
+ * rope_theta = 10000 and max_tokens = 131072. */
 void dsa_indexer_default_config(dsa_indexer_config_t* cfg);
 
 /* Creates a handle for one layer's indexer on the current CUDA device.
  * Weight pointers are device bf16 tensors stored (in x out), row-major:
  *   W_q [q_latent_dim, n_heads*head_dim]   (head h = columns h*128 .. h*128+127)
+ *   (n_heads = 64: W_q [q_latent_dim, 8192], W_w [hidden_dim, 64])
  *   W_k [hidden_dim, head_dim], W_w [hidden_dim, n_heads],
  *   ln_gamma [head_dim], ln_beta [head_dim].
  * The weights are copied (re-laid out for the tensor cores) into memory the
@@ -111,7 +119,10 @@ dsa_status_t dsa_indexer_destroy(dsa_indexer_t h);
  *   q_out         bf16 [T, n_heads*head_dim] = bf16(q_latent W_q), fp32 accumulate
  *   w_out         fp32 [T, n_heads]          = hidden W_w, fp32 accumulate
  * The key is k = bf16(gamma * (x - mean) / sqrt(var + eps) + beta) with
- * x = hidden W_k kept in fp32 and the biased variance.  A token whose position
+ * x = hidden W_k kept in fp32 and the biased variance.  With rope_dim > 0 the
+ * first rope_dim dims of every query head and of the normalised key turn, pair
+ * (2i, 2i+1) by the angle positions[t] * rope_theta^(-2i / rope_dim), before
+ * the bf16 rounding.  A token whose position
  * lies outside [0, rows of its sequence) gets no key row and sets
  * DSA_ERR_DEVICE_BOUNDS.  T = 0 is a no-op.  One call covers at most
  * 8,388,480 tokens (65,535 tiles of 128 rows): a larger T is refused at launch
@@ -170,7 +181,8 @@ dsa_status_t dsa_indexer_topk(dsa_indexer_t h, int64_t T, const void* q, const f
  *     I[t,s] = key_scale[s] * sum_h (w[t,h] * q_scale[t,h]) * ReLU(q8[t,h] . k8[s])
  * (the positive scales factor out of the ReLU), computed on the tensor cores
  * with kind::f8f6f4 MMAs; decode reads 132 bytes per cached key instead of 256.
- * Requires hidden_dim >= 128 (DSA_ERR_UNSUPPORTED otherwise). */
+ * Requires hidden_dim >= 128, n_heads = 32 and rope_dim = 0 (the Kimi K3.1 form;
+ * DSA_ERR_UNSUPPORTED otherwise). */
 
 /* dsa_indexer_project with FP8 outputs: key_cache_fp8 uint8 [cache_rows, head_dim]
  * and key_scale fp32 [cache_rows] receive the token's key row; q_fp8 uint8
