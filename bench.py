@@ -760,9 +760,23 @@ def profile_call(d, spec, repeats):
     chunks up to CALL one at a time, so the device holds one chunk's tensors, the key
     cache and the workspace (well under 1 GB).  Prints the call's CUDA-event times."""
     name, _, call = spec.partition(":")
-    cfg = W.WORKLOADS[name]
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    if name in ("decode_64", "decode_64_fp8"):
+        fp8 = name.endswith("_fp8")
+        ds = setup_decode(d, 0, device, fp8)
+        spans = Spans()
+        decode_step(ds, spans)      # the projections write the new keys; then time the calls
+        torch.cuda.synchronize()
+        for i in range(repeats):
+            spans = Spans()
+            decode_step(ds, spans)
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for k, a, b in spans if k == "topk")
+            print(f"{spec} call {i}: {ms:.4f} ms, {ds['bytes'] / ms / 1e6:.1f} GB/s, 0 TFLOP/s", flush=True)
+        assert ds["ix"].device_error() == d.DSA_OK
+        return
+    cfg = W.WORKLOADS[name]
     wts = W.make_weights(cfg["weight_seed"])
     to = lambda t: t.to(device).contiguous()  # noqa: E731
     if cfg["kind"] == "chunked":

@@ -181,9 +181,26 @@ constexpr int kBins1 = 1 << (32 - kBinShift);  // 2,048 bins
 constexpr int kSubShift = kBinShift - 11;      // second-level bin = next 11 bits
 constexpr int kListCap = 1024;                 // boundary-bin candidates gathered in shared memory
 constexpr int kCheckTiles = 16;                // key tiles between threshold updates
-constexpr int kCapTiles = 16;                  // key tiles between capacity checks (long items)
+constexpr int kCapTiles = kCheckTiles;         // key tiles between capacity checks (long items)
 constexpr int kCheckMargin = kCapTiles * 32;   // appends one warp can make per query in that time
 constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
+constexpr int kSatBlocks = 2;                  // 8-head blocks (of 4) whose ReLU runs on the FMA pipe
+
+// An admission threshold held as a float, raised to the order-preserving key t if that is
+// higher.  Keys at or below that of -inf admit every finite score (-inf).
+__device__ __forceinline__ float raise_threshold(float thr, uint32_t t) {
+  const uint32_t u = max(float_to_ordered(thr), t);
+  return u <= float_to_ordered(-INFINITY) ? -INFINITY : ordered_to_float(u);
+}
+
+// ReLU of two values on the FMA pipe: x * sat(x * 2^64), sat clamping to [0, 1].  The mask is
+// 1 for x >= 2^-64 and 0 for x <= 0; in between (|x| < 5.5e-20) the result is x^2 2^64 < x.
+__device__ __forceinline__ float2 relu2_fma(float2 x) {
+  float m0, m1;
+  asm("mul.rn.sat.f32 %0, %1, 0f5F800000;" : "=f"(m0) : "f"(x.x));
+  asm("mul.rn.sat.f32 %0, %1, 0f5F800000;" : "=f"(m1) : "f"(x.y));
+  return __fmul2_rn(x, make_float2(m0, m1));
+}
 
 __device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
   atomicAdd(&h[bin >> 1], (bin & 1u) ? 0x10000u : 1u);
@@ -940,11 +957,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       // an item of at most kWarpApp / 32 tiles cannot fill an append area: no capacity checks
       const bool long_item = (kt1 - kt0) * 32 > kWarpApp;
       int cnt_r[QPH], pos_r[QPH];
-      uint32_t thr_r[QPH];
 #pragma unroll
       for (int j = 0; j < QPH; ++j) {
         cnt_r[j] = 0;
-        thr_r[j] = 0u;
         pos_r[j] = (j < nmine) ? min(st.pos[j0 + j], wi.k_end - 1) : -2;   // last key position scored
       }
       // this thread's head weights: heads 32 hb + 8 blk + 2 (lane % 4) + {0, 1} of each of its
@@ -958,12 +973,37 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           for (int blk = 0; blk < 4; ++blk)
             w2[j * HB + hb][blk] = *reinterpret_cast<const float2*>(&st.w[j0 + j][32 * hb + 8 * blk + 2 * (lane & 3)]);
       bool failed = false;
-      for (int kt = kt0; kt < kt1; ++kt, ++acc_ctr) {
-        const int ab = (ALT ? g * ACC_BUFS : 0) + acc_ctr % ACC_BUFS;   // this group's ring
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (acc_ctr / ACC_BUFS) & 1, wc));
+      // per-tile state kept incrementally: the group's accumulator slot and its phase, the
+      // TMEM column of this warp's first block in slot 0, this thread's key position, the
+      // admission thresholds as floats, and the tiles left until the next check point
+      int aslot = acc_ctr % ACC_BUFS;
+      uint32_t phase = static_cast<uint32_t>(acc_ctr / ACC_BUFS) & 1u;
+      const int slot0 = ALT ? g * ACC_BUFS : 0;
+      const uint32_t tcol0 = tlane + slot0 * C::kAccCols + (qbase + j0) * H;
+      int s_pos = kt0 * kKeyTile + r;
+      int to_check = kCheckTiles;
+      float thr_f[QPH];
+#pragma unroll
+      for (int j = 0; j < QPH; ++j) thr_f[j] = -INFINITY;
+      // FP8: the scales of this thread's key rows in the next kScalePrefetch tiles, loaded
+      // that many tiles ahead of their use (rows past the item's last scored key read as 0)
+      constexpr int kScalePrefetch = kFp8 ? 4 : 1;
+      float skq[kScalePrefetch];
+#pragma unroll
+      for (int i = 0; i < kScalePrefetch; ++i) {
+        const int sp = s_pos + i * kKeyTile;
+        skq[i] = (kFp8 && sp < wi.k_end) ? __ldg(p.key_scale + kbase + sp) : 0.f;
+      }
+      acc_ctr += kt1 - kt0;
+      for (int kt = kt0; kt < kt1; ++kt, s_pos += kKeyTile) {
+        const int ab = slot0 + aslot;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], phase, wc));
         tc_fence_after();
-        const int s_pos = kt * kKeyTile + r;
-        const uint32_t tcol = tlane + ab * C::kAccCols + (qbase + j0) * H;
+        const uint32_t tcol = tcol0 + aslot * C::kAccCols;
+        if (++aslot == ACC_BUFS) {
+          aslot = 0;
+          phase ^= 1u;
+        }
         if (ok) {
           // this warp's columns of the tile, as 16x256b blocks of 32 columns (CB of them: its
           // queries' head blocks, contiguous): one TMEM round trip per tile
@@ -980,7 +1020,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
           // partial sums over this thread's 8 heads of each head block, for its two rows of
-          // each lane half
+          // each lane half.  ReLU(x) w runs on two pipes: blocks below kSatBlocks form it on
+          // the FMA pipe as (x * sat(x * 2^64)) w, the others take max(x, 0) on the ALU pipe
           float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -992,10 +1033,15 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
                 const uint32_t(&x)[16] = v[h * CB + j * HB + hb];
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
-                  a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
-                                                              fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
-                  b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
-                                                              fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
+                  const float2 xa = make_float2(__uint_as_float(x[4 * blk]), __uint_as_float(x[4 * blk + 1]));
+                  const float2 xb = make_float2(__uint_as_float(x[4 * blk + 2]), __uint_as_float(x[4 * blk + 3]));
+                  if (blk < kSatBlocks) {
+                    a = ffma2(w2[j * HB + hb][blk], relu2_fma(xa), a);
+                    b = ffma2(w2[j * HB + hb][blk], relu2_fma(xb), b);
+                  } else {
+                    a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(xa.x, 0.f), fmaxf(xa.y, 0.f)), a);
+                    b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(xb.x, 0.f), fmaxf(xb.y, 0.f)), b);
+                  }
                 }
               }
               part[(2 * h) * QPH + j] = a.x + a.y;
@@ -1004,35 +1050,44 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           float score[QPH];
           sum_over_quad<QPH>(part, score, lane);
           if constexpr (kFp8) {
-            // the key row's scale (positive) multiplies every head's ReLU term; rows past the
-            // item's last scored key are masked and not read
-            const float sk = s_pos < wi.k_end ? __ldg(p.key_scale + kbase + s_pos) : 0.f;
+            // the key row's scale (positive) multiplies every head's ReLU term
 #pragma unroll
-            for (int j = 0; j < QPH; ++j) score[j] *= sk;
+            for (int j = 0; j < QPH; ++j) score[j] *= skq[0];
           }
           // admit (key, position) into this warp's area of each of its queries and count it;
-          // the append counts stay warp-uniform in registers
+          // the append counts stay warp-uniform in registers.  The float comparison with the
+          // threshold admits what the order-preserving key comparison admits (and -0 against
+          // a threshold of +0, a harmless extra candidate)
 #pragma unroll
           for (int j = 0; j < QPH; ++j) {
             if (j >= nmine) break;
-            const uint32_t u = float_to_ordered(score[j]);
-            const bool pass = (s_pos <= pos_r[j]) && (u >= thr_r[j]);
+            const bool pass = (s_pos <= pos_r[j]) && (score[j] >= thr_f[j]);
             const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-            if (pass) {
-              st_global_u2_hint(&my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)],
-                                make_uint2(u, static_cast<uint32_t>(s_pos)), pol_cand);
-              count_key(st.hist[j0 + j], u >> kBinShift);
+            if (bal) {
+              if (pass) {
+                const uint32_t u = float_to_ordered(score[j]);
+                st_global_u2_hint(&my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)],
+                                  make_uint2(u, static_cast<uint32_t>(s_pos)), pol_cand);
+                count_key(st.hist[j0 + j], u >> kBinShift);
+              }
+              cnt_r[j] += __popc(bal);
             }
-            cnt_r[j] += __popc(bal);
           }
         } else {
           failed = true;
         }
+        if constexpr (kFp8) {
+#pragma unroll
+          for (int i = 0; i + 1 < kScalePrefetch; ++i) skq[i] = skq[i + 1];
+          const int sp = s_pos + kScalePrefetch * kKeyTile;
+          skq[kScalePrefetch - 1] = sp < wi.k_end ? __ldg(p.key_scale + kbase + sp) : 0.f;
+        }
         // check point every kCheckTiles tiles (the same tiles for every warp of the group); a
         // long item also checks the append areas' capacity at every kCapTiles-th tile
-        if ((kt - kt0) % kCheckTiles == kCheckTiles - 1 && kt + 1 < kt1) {
+        if (--to_check == 0 && kt + 1 < kt1) {
+          to_check = kCheckTiles;
           bool need = false;
-          const bool cap_check = long_item && (kt - kt0) % kCapTiles == kCapTiles - 1;
+          const bool cap_check = long_item;   // every check point is a capacity point (kCapTiles == kCheckTiles)
           if (cap_check) {
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
@@ -1089,7 +1144,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
             for (int j = 0; j < QPH; ++j) {
               if (j < nmine) {
                 cnt_r[j] = st.cnt_w[j0 + j][qd];
-                thr_r[j] = max(thr_r[j], st.thr[j0 + j]);
+                thr_f[j] = raise_threshold(thr_f[j], st.thr[j0 + j]);
               }
             }
           }
@@ -1104,11 +1159,11 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
               const int jl = j0 + j;
               if ((jl & 3) == qd) {
                 const uint32_t t = static_cast<uint32_t>(scan_bins_warp(st.hist[jl], kTopK, lane)) << kBinShift;
-                thr_r[j] = max(thr_r[j], t);
+                thr_f[j] = raise_threshold(thr_f[j], t);
                 __syncwarp();
                 if (lane == 0) st.thr_bin[jl] = max(st.thr_bin[jl], t);
               } else {
-                thr_r[j] = max(thr_r[j], st.thr_bin[jl]);
+                thr_f[j] = raise_threshold(thr_f[j], st.thr_bin[jl]);
               }
             }
           }

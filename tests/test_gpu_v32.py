@@ -104,8 +104,11 @@ def test_v32_end_to_end(dsa):
     batch = W.make_prefill(67, [2500], start_positions=[100_000], cache_lens=[102_500])
     T = 2500
     ix = _indexer(dsa, wts, 4096)
-    # the keys of positions 0..99,999 are not part of this batch: zero rows score 0
+    # the keys of positions 0..99,999 are not part of this batch: seeded N(0,1) rows stand in
+    # for them (exactly tied zero rows would leave the selection free among ties)
+    prefix = W.make_scoring_inputs(68, 1, 100_000, n_heads=H)[1]
     cache = torch.zeros((102_500, 128), dtype=torch.bfloat16, device="cuda")
+    cache[:100_000] = _cuda(prefix)
     pos, qoff, coff = _cuda(batch.positions), _cuda(batch.q_seq_offsets), _cuda(batch.cache_offsets)
     q, w = ix.project(_cuda(batch.hidden), _cuda(batch.q_latent), pos, qoff, cache, coff)
     idx, sc = ix.topk(q, w, pos, qoff, cache, coff)
@@ -115,6 +118,7 @@ def test_v32_end_to_end(dsa):
     assert_proj_close(f64(q).reshape(T, -1), oq.reshape(T, -1), "q")
     assert_proj_close(f64(cache[100_000:]), ok_, "k")
     keys = np.zeros((102_500, 128))
+    keys[:100_000] = f64(prefix)
     keys[100_000:] = ok_
     rows = np.arange(0, T, 50)
     _, _, I, A = oracle.topk(oq, ow, batch.positions.numpy(), batch.q_seq_offsets.numpy(), keys,
