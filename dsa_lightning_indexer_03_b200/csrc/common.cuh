@@ -122,19 +122,30 @@ struct WaitCtl {
   uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
-  const uint32_t a = smem_u32(bar);
+// the CTA's abort flag, read with an explicit shared-memory volatile load
+__device__ __forceinline__ int read_abort(const WaitCtl& c) {
+  int v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(const_cast<int*>(c.abort_flag))) : "memory");
+  return v;
+}
+
+// bar is the barrier's shared-memory address
+__device__ __forceinline__ bool mbar_wait_addr(uint32_t a, uint32_t parity, const WaitCtl& c) {
   if (mbar_try_wait_sleep(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait_sleep(a, parity)) return true;
-    if (*c.abort_flag) return false;
+    if (read_abort(c)) return false;
     if (global_timer_ns() - t0 > c.timeout_ns) {
       atomicOr(c.err, kErrTimeout);
       *c.abort_flag = 1;
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& c) {
+  return mbar_wait_addr(smem_u32(bar), parity, c);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -184,7 +184,6 @@ constexpr int kCheckTiles = 16;                // key tiles between threshold up
 constexpr int kCapTiles = kCheckTiles;         // key tiles between capacity checks (long items)
 constexpr int kCheckMargin = kCapTiles * 32;   // appends one warp can make per query in that time
 constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
-constexpr int kSatBlocks = 2;                  // 8-head blocks (of 4) whose ReLU runs on the FMA pipe
 
 // An admission threshold held as a float, raised to the order-preserving key t if that is
 // higher.  Keys at or below that of -inf admit every finite score (-inf).
@@ -193,17 +192,11 @@ __device__ __forceinline__ float raise_threshold(float thr, uint32_t t) {
   return u <= float_to_ordered(-INFINITY) ? -INFINITY : ordered_to_float(u);
 }
 
-// ReLU of two values on the FMA pipe: x * sat(x * 2^64), sat clamping to [0, 1].  The mask is
-// 1 for x >= 2^-64 and 0 for x <= 0; in between (|x| < 5.5e-20) the result is x^2 2^64 < x.
-__device__ __forceinline__ float2 relu2_fma(float2 x) {
-  float m0, m1;
-  asm("mul.rn.sat.f32 %0, %1, 0f5F800000;" : "=f"(m0) : "f"(x.x));
-  asm("mul.rn.sat.f32 %0, %1, 0f5F800000;" : "=f"(m1) : "f"(x.y));
-  return __fmul2_rn(x, make_float2(m0, m1));
-}
-
+// h is shared memory: a fire-and-forget shared-memory reduction (the barrier that precedes
+// every read of the counts orders it)
 __device__ __forceinline__ void count_key(uint32_t* h, uint32_t bin) {
-  atomicAdd(&h[bin >> 1], (bin & 1u) ? 0x10000u : 1u);
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_u32(&h[bin >> 1])), "r"((bin & 1u) ? 0x10000u : 1u)
+               : "memory");
 }
 
 constexpr int kRoundU = 4;   // 16-byte loads (two candidates each) per thread and round
@@ -980,6 +973,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       uint32_t phase = static_cast<uint32_t>(acc_ctr / ACC_BUFS) & 1u;
       const int slot0 = ALT ? g * ACC_BUFS : 0;
       const uint32_t tcol0 = tlane + slot0 * C::kAccCols + (qbase + j0) * H;
+      const uint32_t afull0 = smem_u32(&acc_full[slot0]), aempty0 = smem_u32(&acc_empty[slot0]);
       int s_pos = kt0 * kKeyTile + r;
       int to_check = kCheckTiles;
       float thr_f[QPH];
@@ -996,8 +990,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       }
       acc_ctr += kt1 - kt0;
       for (int kt = kt0; kt < kt1; ++kt, s_pos += kKeyTile) {
-        const int ab = slot0 + aslot;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], phase, wc));
+        const uint32_t aoff = static_cast<uint32_t>(aslot) * 8u;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_addr(afull0 + aoff, phase, wc));
         tc_fence_after();
         const uint32_t tcol = tcol0 + aslot * C::kAccCols;
         if (++aslot == ACC_BUFS) {
@@ -1018,10 +1012,10 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);   // TMEM buffer free for the next MMA
+          if (lane == 0)   // TMEM buffer free for the next MMA
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(aempty0 + aoff) : "memory");
           // partial sums over this thread's 8 heads of each head block, for its two rows of
-          // each lane half.  ReLU(x) w runs on two pipes: blocks below kSatBlocks form it on
-          // the FMA pipe as (x * sat(x * 2^64)) w, the others take max(x, 0) on the ALU pipe
+          // each lane half
           float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
 #pragma unroll
           for (int h = 0; h < 2; ++h)
@@ -1033,15 +1027,10 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
                 const uint32_t(&x)[16] = v[h * CB + j * HB + hb];
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
-                  const float2 xa = make_float2(__uint_as_float(x[4 * blk]), __uint_as_float(x[4 * blk + 1]));
-                  const float2 xb = make_float2(__uint_as_float(x[4 * blk + 2]), __uint_as_float(x[4 * blk + 3]));
-                  if (blk < kSatBlocks) {
-                    a = ffma2(w2[j * HB + hb][blk], relu2_fma(xa), a);
-                    b = ffma2(w2[j * HB + hb][blk], relu2_fma(xb), b);
-                  } else {
-                    a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(xa.x, 0.f), fmaxf(xa.y, 0.f)), a);
-                    b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(xb.x, 0.f), fmaxf(xb.y, 0.f)), b);
-                  }
+                  a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
+                                                              fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
+                  b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
+                                                              fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
                 }
               }
               part[(2 * h) * QPH + j] = a.x + a.y;
