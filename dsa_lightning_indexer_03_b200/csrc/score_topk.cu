@@ -774,7 +774,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
     if (lane == 0) {
       int kstage = 0, qloads = 0;
       const uint64_t pol_q = l2_policy_evict_first();   // each Q tile is read once
-      const uint64_t pol_k = l2_policy_evict_last();    // key tiles are read by every item of a sequence
+      // prefill: key tiles are read by every item of a sequence; split path (decode): each key
+      // is read once, and should not push the partial lists out of L2
+      const uint64_t pol_k = ALT ? l2_policy_evict_first() : l2_policy_evict_last();
       for (int local = 0;; ++local) {
         const int slot = local & 1;
         if (local >= 2 && !mbar_wait(&sched_empty[slot], ((local >> 1) - 1) & 1, wc)) break;
@@ -815,6 +817,14 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           uint8_t* dst = sK + s * C::kKStage;
           tma_load_2d_hint(dst, &tmK, &full[s], 0, row0 + kt * kKeyTile, pol_k);
           if constexpr (!kFp8) tma_load_2d_hint(dst + C::kKHalf, &tmK, &full[s], 64, row0 + kt * kKeyTile, pol_k);
+          if constexpr (kFp8) {
+            // the tile's key scales, read by the epilogue threads once the tile is scored:
+            // bring their lines into L2 now (every prefetched address is a scale of the item)
+            const int nrows = min(kKeyTile, wi.k_end - kt * kKeyTile);
+            const float* sp = p.key_scale + row0 + kt * kKeyTile;
+            for (int i = 0; i < nrows; i += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(sp + i));
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(sp + nrows - 1));
+          }
         }
         if (!ok) break;
       }
@@ -979,17 +989,12 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       float thr_f[QPH];
 #pragma unroll
       for (int j = 0; j < QPH; ++j) thr_f[j] = -INFINITY;
-      // FP8: the scales of this thread's key rows in the next kScalePrefetch tiles, loaded
-      // that many tiles ahead of their use (rows past the item's last scored key read as 0)
-      constexpr int kScalePrefetch = kFp8 ? 4 : 1;
-      float skq[kScalePrefetch];
-#pragma unroll
-      for (int i = 0; i < kScalePrefetch; ++i) {
-        const int sp = s_pos + i * kKeyTile;
-        skq[i] = (kFp8 && sp < wi.k_end) ? __ldg(p.key_scale + kbase + sp) : 0.f;
-      }
       acc_ctr += kt1 - kt0;
       for (int kt = kt0; kt < kt1; ++kt, s_pos += kKeyTile) {
+        // FP8: this thread's key scale, requested before the accumulator wait (the producer
+        // brought its line into L2 when it loaded the tile); rows past the item's last scored
+        // key read as 0
+        const float sk = (kFp8 && s_pos < wi.k_end) ? __ldg(p.key_scale + kbase + s_pos) : 0.f;
         const uint32_t aoff = static_cast<uint32_t>(aslot) * 8u;
         const bool ok = __all_sync(0xffffffffu, mbar_wait_addr(afull0 + aoff, phase, wc));
         tc_fence_after();
@@ -1041,7 +1046,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           if constexpr (kFp8) {
             // the key row's scale (positive) multiplies every head's ReLU term
 #pragma unroll
-            for (int j = 0; j < QPH; ++j) score[j] *= skq[0];
+            for (int j = 0; j < QPH; ++j) score[j] *= sk;
           }
           // admit (key, position) into this warp's area of each of its queries and count it;
           // the append counts stay warp-uniform in registers.  The float comparison with the
@@ -1064,12 +1069,6 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           }
         } else {
           failed = true;
-        }
-        if constexpr (kFp8) {
-#pragma unroll
-          for (int i = 0; i + 1 < kScalePrefetch; ++i) skq[i] = skq[i + 1];
-          const int sp = s_pos + kScalePrefetch * kKeyTile;
-          skq[kScalePrefetch - 1] = sp < wi.k_end ? __ldg(p.key_scale + kbase + sp) : 0.f;
         }
         // check point every kCheckTiles tiles (the same tiles for every warp of the group); a
         // long item also checks the append areas' capacity at every kCapTiles-th tile
@@ -1256,12 +1255,14 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
 // merge of the split-key path: top-k over the partial lists of one query's key chunks.
 // Every chunk added the first-level bin counts of the entries it kept to the query's
 // histogram, so the bin b1 holding the kTopK-th largest entry is found from those counts
-// alone.  One pass over the partial lists then writes every entry above b1 to its output
-// slot and gathers b1's entries into shared memory, where the exact kTopK-th largest key K*
-// is found (kth_largest) and the entries of b1 above K*, then the first ties, are written.
-// The histogram is cleared after use, ready for the next call.
+// alone.  A first pass over the partial lists counts b1's entries by their next 11 bits; the
+// sub-bin b2 holding the kTopK-th largest follows.  A second pass writes every entry above
+// (b1, b2) to its output slot and gathers the entries of (b1, b2) -- a range of 2^10 keys --
+// into shared memory, where the exact kTopK-th largest key K* is found (kth_largest) and the
+// entries above K*, then the first ties, are written.  The histogram is cleared after use,
+// ready for the next call.
 constexpr int kMergeThreads = 1024;
-constexpr int kMergeList = 8192;   // boundary-bin entries held in shared memory
+constexpr int kMergeList = 8192;   // entries of the boundary sub-bin held in shared memory
 
 __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __restrict__ part_keys,
                                                               const int32_t* __restrict__ part_idx,
@@ -1269,10 +1270,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
                                                               uint32_t* __restrict__ part_hist,
                                                               int32_t* __restrict__ idx_out,
                                                               float* __restrict__ score_out, int sorted) {
-  extern __shared__ uint32_t msm[];   // list keys [kMergeList], list positions [kMergeList], stage [kTopK] pairs
+  // dynamic: list keys [kMergeList], list positions [kMergeList], stage [kTopK] pairs,
+  // second-level counts [kBins1]
+  extern __shared__ uint32_t msm[];
   uint32_t* const lkeys = msm;
   int32_t* const lidx = reinterpret_cast<int32_t*>(msm + kMergeList);
   uint2* const stage = reinterpret_cast<uint2*>(msm + 2 * kMergeList);
+  uint32_t* const hist2 = msm + 2 * kMergeList + 2 * kTopK;
   __shared__ uint32_t hist[kHistBins];
   __shared__ uint32_t scratch[kMergeThreads / 32];
   __shared__ int sh[8];
@@ -1299,6 +1303,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
     }
   };
   if (tid < 4) ctr[tid] = 0;
+  for (int i = tid; i < kBins1; i += kMergeThreads) hist2[i] = 0u;
   // 1. boundary bin from the counts (two bins per thread), then clear them
   constexpr int kBPT = kBins1 / kMergeThreads;
   static_assert(kBPT == 2, "two bins per thread");
@@ -1315,7 +1320,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
     sh[0] = 0;
     sh[1] = 0;
   }
-  const uint32_t above_t = group_suffix_excl<kMergeThreads>(csum, tid, scratch, 1);
+  uint32_t above_t = group_suffix_excl<kMergeThreads>(csum, tid, scratch, 1);
   if (above_t < static_cast<uint32_t>(kTopK) && static_cast<uint32_t>(kTopK) <= above_t + csum) {
     uint32_t cum = above_t;
 #pragma unroll
@@ -1331,7 +1336,47 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   named_bar_sync(1, kMergeThreads);
   const uint32_t b1 = static_cast<uint32_t>(min(max(sh[0], 0), kBins1 - 1));
   const int above = min(max(sh[1], 0), kTopK);
-  // 2. one pass: entries above b1 to their slots, b1's entries to the list
+  const int need = kTopK - above;
+  // 2. second-level counts of b1's entries
+#pragma unroll 4
+  for (int g = tid; g < n / 4; g += kMergeThreads) {
+    const uint4 kk = reinterpret_cast<const uint4*>(keys)[g];
+    const int4 ii = reinterpret_cast<const int4*>(pos)[g];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t key = u4_get(kk, j);
+      if (i4_get(ii, j) >= 0 && (key >> kBinShift) == b1)
+        asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(smem_u32(&hist2[(key >> kSubShift) & (kBins1 - 1)])) : "memory");
+    }
+  }
+  named_bar_sync(1, kMergeThreads);
+#pragma unroll
+  for (int i = 0; i < kBPT; ++i) {
+    c[i] = hist2[kBPT * tid + i];
+  }
+  csum = c[0] + c[1];
+  if (tid == 0) {
+    sh[2] = 0;
+    sh[3] = 0;
+  }
+  above_t = group_suffix_excl<kMergeThreads>(csum, tid, scratch, 1);
+  if (above_t < static_cast<uint32_t>(need) && static_cast<uint32_t>(need) <= above_t + csum) {
+    uint32_t cum = above_t;
+#pragma unroll
+    for (int i = kBPT - 1; i >= 0; --i) {
+      if (cum + c[i] >= static_cast<uint32_t>(need)) {
+        sh[2] = kBPT * tid + i;
+        sh[3] = static_cast<int>(cum);
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  named_bar_sync(1, kMergeThreads);
+  const uint32_t b2 = static_cast<uint32_t>(min(max(sh[2], 0), kBins1 - 1));
+  const int above2 = min(max(sh[3], 0), need);
+  const uint32_t lo = (b1 << kBinShift) | (b2 << kSubShift), hi = lo + ((1u << kSubShift) - 1u);
+  // 3. one pass: entries above lo to their slots, the entries of [lo, hi] to the list
   const uint32_t lt = lanemask_lt();
 #pragma unroll 2
   for (int base = 0; base < n / 4; base += kMergeThreads) {
@@ -1346,8 +1391,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
     for (int j = 0; j < 4; ++j) {
       const uint32_t key = u4_get(kk, j);
       const int p = i4_get(ii, j);
-      const uint32_t bin = key >> kBinShift;
-      const bool up = p >= 0 && bin > b1, mid = p >= 0 && bin == b1;
+      const bool up = p >= 0 && key > hi, mid = p >= 0 && key >= lo && key <= hi;
       const uint32_t bu = __ballot_sync(0xffffffffu, up), bm = __ballot_sync(0xffffffffu, mid);
       if (bu | bm) {
         int ou = 0, om = 0;
@@ -1367,23 +1411,24 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   }
   named_bar_sync(1, kMergeThreads);
   const int m = ctr[1];
-  const int need = kTopK - above;
-  const uint32_t lo = b1 << kBinShift, hi = lo + ((1u << kBinShift) - 1u);
+  const int base_slot = above + above2;   // slots taken by the entries above the sub-bin
+  const int need3 = need - above2;
   int n_above;
   uint32_t kth;
-  // 3. the exact need-th largest key of the boundary bin
+  // 4. the exact need3-th largest key of the sub-bin
   if (m <= kMergeList) {
-    kth = kth_largest<kMergeThreads>(lkeys, m, need, lo, hi, hist, scratch, sh, tid, 1, &n_above);
+    kth = kth_largest<kMergeThreads>(lkeys, m, need3, lo, hi, hist, scratch, sh, tid, 1, &n_above);
   } else {
-    // more boundary entries than the list holds: visit them in the partial lists
+    // more entries in the sub-bin than the list holds (many equal scores): visit them in the
+    // partial lists
     auto visit = [&](auto f) {
       for (int e = tid; e < n; e += kMergeThreads)
-        if (pos[e] >= 0 && (keys[e] >> kBinShift) == b1) f(keys[e]);
+        if (pos[e] >= 0 && keys[e] >= lo && keys[e] <= hi) f(keys[e]);
     };
-    kth = kth_window<kMergeThreads>(visit, need, lo, hi, hist, scratch, sh, tid, 1, &n_above);
+    kth = kth_window<kMergeThreads>(visit, need3, lo, hi, hist, scratch, sh, tid, 1, &n_above);
   }
-  // 4. the boundary bin's entries above K*, then the first ties
-  const int ties = need - n_above;
+  // 5. the sub-bin's entries above K*, then the first ties
+  const int ties = need3 - n_above;
   auto fin = [&](uint32_t key, int p, bool ok) {
     const bool gt = ok && key > kth, eq = ok && key == kth;
     const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
@@ -1395,8 +1440,8 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
       }
       og = __shfl_sync(0xffffffffu, og, 0) + __popc(bg & lt);
       oe = __shfl_sync(0xffffffffu, oe, 0) + __popc(be & lt);
-      if (gt && above + og < kTopK) out(above + og, key, p);
-      if (eq && oe < ties) out(above + n_above + oe, key, p);
+      if (gt && base_slot + og < kTopK) out(base_slot + og, key, p);
+      if (eq && oe < ties) out(base_slot + n_above + oe, key, p);
     }
   };
   if (m <= kMergeList) {
@@ -1408,7 +1453,7 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   } else {
     for (int base = 0; base < n; base += kMergeThreads) {
       const int e = base + tid;
-      const bool ok = e < n && pos[e] >= 0 && (keys[e] >> kBinShift) == b1;
+      const bool ok = e < n && pos[e] >= 0 && keys[e] >= lo && keys[e] <= hi;
       fin(ok ? keys[e] : 0u, ok ? pos[e] : -1, ok);
     }
   }
@@ -1504,21 +1549,33 @@ __device__ __forceinline__ int sequence_of_token(const int32_t* qoff, int B, int
   return lo;
 }
 
-constexpr int kPrepCopy = 4096;   // offset arrays up to this length are searched in shared memory
+constexpr int kPrepCopy = 2048;   // offset arrays up to this length are searched in shared memory
+constexpr int kPrepTok = 1024;    // validated positions and chunk counts of up to this many queries stay in shared memory
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __shared__ int warp_sums[32];
   __shared__ int bad;
   __shared__ unsigned long long total_keys;
   __shared__ int s_qoff[kPrepCopy + 1];   // copy of q_seq_offsets when B < kPrepCopy
+  __shared__ int64_t s_coff[kPrepCopy + 1];   // copy of cache_offsets when B < kPrepCopy
   __shared__ int s_base[kPrepCopy + 1];   // copy of the items' owner bases when n_owners < kPrepCopy
+  __shared__ int s_pe[kPrepTok];          // validated positions when T <= kPrepTok
+  __shared__ int s_nch[kPrepTok];         // key chunks per query when T <= kPrepTok
   const TopkWorkspace& ws = p.ws;
   // the score kernel may start its prologue now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // every input is read once, up front; later phases read the shared copies
   const bool qoff_in_smem = p.B < kPrepCopy;
   if (qoff_in_smem)
-    for (int b = threadIdx.x; b <= p.B; b += kPrepThreads) s_qoff[b] = p.q_seq_offsets[b];
+    for (int b = threadIdx.x; b <= p.B; b += kPrepThreads) {
+      s_qoff[b] = p.q_seq_offsets[b];
+      s_coff[b] = p.cache_offsets[b];
+    }
   const int32_t* qoff = qoff_in_smem ? s_qoff : p.q_seq_offsets;
+  const int64_t* coff = qoff_in_smem ? s_coff : p.cache_offsets;
+  const bool tok_in_smem = p.T <= kPrepTok;
+  int* const pe = tok_in_smem ? s_pe : ws.pos_eff;      // validated positions (also written to ws.pos_eff)
+  int* const nchk = tok_in_smem ? s_nch : ws.tok_nchunks;
   if (threadIdx.x == 0) {
     bad = 0;
     total_keys = 0;
@@ -1526,12 +1583,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __syncthreads();
   // 1. offsets
   for (int b = threadIdx.x; b <= p.B; b += kPrepThreads) {
-    const int qo = p.q_seq_offsets[b];
-    const int64_t co = p.cache_offsets[b];
+    const int qo = qoff[b];
+    const int64_t co = coff[b];
     bool ok = qo >= 0 && qo <= p.T && co >= 0 && co <= p.cache_rows;
     if (b == 0) ok = ok && qo == 0;
     if (b == p.B) ok = ok && qo == p.T;
-    if (b > 0) ok = ok && p.q_seq_offsets[b - 1] <= qo && p.cache_offsets[b - 1] <= co;
+    if (b > 0) ok = ok && qoff[b - 1] <= qo && coff[b - 1] <= co;
     if (!ok) bad = 1;
   }
   __syncthreads();
@@ -1553,11 +1610,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   // 2. validated positions
   for (int t = threadIdx.x; t < p.T; t += kPrepThreads) {
     const int lo = sequence_of_token(qoff, p.B, t);
-    const int64_t len = p.cache_offsets[lo + 1] - p.cache_offsets[lo];
+    const int64_t len = coff[lo + 1] - coff[lo];
     const int pos = p.positions[t];
     const bool ok = pos >= 0 && pos < len;
     if (!ok) atomicOr(ws.err, kErrBounds);
-    ws.pos_eff[t] = ok ? pos : -1;
+    pe[t] = ok ? pos : -1;
+    if (tok_in_smem) ws.pos_eff[t] = ok ? pos : -1;
     ws.tok_nchunks[t] = 0;
     if (p.split && ok) atomicAdd(&total_keys, static_cast<unsigned long long>(pos) + 1ull);
   }
@@ -1574,10 +1632,11 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   for (int o = threadIdx.x; o < n_owners; o += kPrepThreads) {
     int c;
     if (p.split) {
-      const int n = ws.pos_eff[o] + 1;
+      const int n = pe[o] + 1;
       const int cl = chunk_len_for(n, target);
       c = n > cl ? (n + cl - 1) / cl : 1;
-      ws.tok_nchunks[o] = c;
+      nchk[o] = c;
+      if (tok_in_smem) ws.tok_nchunks[o] = c;
     } else {
       const int nq = qoff[o + 1] - qoff[o];
       c = (nq + p.qpi - 1) / p.qpi;
@@ -1600,8 +1659,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     wi.pad0 = wi.pad1 = 0;
     if (p.split) {
       const int t = o;
-      const int n = ws.pos_eff[t] + 1;
-      const int nch = ws.tok_nchunks[t];
+      const int n = pe[t] + 1;
+      const int nch = nchk[t];
       const int cl = chunk_len_for(n, target);
       wi.t0 = t;
       wi.nq = 1;
@@ -1614,7 +1673,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       const int t0 = qoff[b] + local * p.qpi;
       const int nq = min(p.qpi, qoff[b + 1] - t0);
       int kend = 0;
-      for (int j = 0; j < nq; ++j) kend = max(kend, ws.pos_eff[t0 + j] + 1);
+      for (int j = 0; j < nq; ++j) kend = max(kend, pe[t0 + j] + 1);
       wi.t0 = t0;
       wi.nq = nq;
       wi.b = b;
@@ -1724,7 +1783,7 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
       e = a.sorted ? launch_score<1, 5, 4, 2, 4, true, true, 2>(tmQ1, tmK, sp, grid, s)
                    : launch_score<1, 5, 4, 2, 4, true, false, 2>(tmQ1, tmK, sp, grid, s);
     if (e != cudaSuccess) return e;
-    const int msmem = 2 * kMergeList * 4 + kTopK * 8;
+    const int msmem = 2 * kMergeList * 4 + kTopK * 8 + kBins1 * 4;
     e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem);
     if (e != cudaSuccess) return e;
     // programmatic dependent of the score kernel, whose CTAs release it when the work list
