@@ -361,7 +361,8 @@ __device__ __forceinline__ int scan_bins_warp(const uint32_t* hw, uint32_t need,
 
 struct ResolveSmem {
   uint32_t* rh;      // kBins1 / 2 words: second-level counts, then kth_window's bins
-  uint2* list;       // kListCap boundary-bin candidates
+  uint2* list;       // list_cap boundary-bin candidates
+  int list_cap;
   uint32_t* small;   // kSmallRank keys of the boundary sub-bin
   uint32_t* scratch;
   int* sh;
@@ -379,12 +380,15 @@ struct ResolveSmem {
 // 4. emit the keys of b1 greater than K* and the first kTopK - n_above keys equal to K*.
 // sink(slot, key, pos) is called once for each slot 0..kTopK-1.  With clear_h1 the words
 // of h1 are zeroed before the first sink call.  Returns K*.
+// With rs.rh == h1 the first-level counts are consumed (and cleared) by step 1 and their
+// words then hold the second-level counts (clear_h1 must be set).
 template <int NT, class Sink>
 __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1, const ResolveSmem& rs, int tid,
                                  int bar, Sink&& sink) {
   const int lane = tid & 31;
   const uint32_t lt = lanemask_lt();
-  for (int i = tid; i < kBins1 / 2; i += NT) rs.rh[i] = 0u;
+  if (rs.rh != h1)
+    for (int i = tid; i < kBins1 / 2; i += NT) rs.rh[i] = 0u;
   if (tid == 0) {
     rs.ctr[0] = 0;
     rs.ctr[1] = 0;
@@ -426,7 +430,7 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
       }
       ou += __popc(bu[e]);
       if (lim[e >> 1] > (e & 1) && (c.x >> kBinShift) == ub1) {
-        if (oa < kListCap) rs.list[oa] = c;
+        if (oa < rs.list_cap) rs.list[oa] = c;
         count_key(rs.rh, (c.x >> kSubShift) & (kBins1 - 1));
         ++oa;
       }
@@ -442,7 +446,7 @@ __device__ uint32_t resolve_topk(const CandView& v, uint32_t* h1, bool clear_h1,
   const uint32_t hi = lo + ((1u << kSubShift) - 1u);
   const int need3 = static_cast<int>(need2 - above2);
   const int m2 = static_cast<int>((rs.rh[b2 >> 1] >> ((b2 & 1) * 16)) & 0xFFFFu);
-  const bool in_list = m <= kListCap;
+  const bool in_list = m <= rs.list_cap;
   int n3;
   uint32_t kth;
   if (in_list && m2 <= kSmallRank) {
@@ -590,8 +594,9 @@ __device__ __forceinline__ void bitonic_sort(uint64_t (&v)[kTopK / NT], int tid,
   if constexpr (K < kTopK) bitonic_sort<NT, 2 * K>(v, tid, s64, bar);
 }
 
+// not inlined: its 2,048 / NT 64-bit words per thread stay out of its callers' register allocation
 template <int NT>
-__device__ void sort_stage_and_emit(uint2* stage, int tid, int bar, int32_t* oi, float* os) {
+__device__ __noinline__ void sort_stage_and_emit(uint2* stage, int tid, int bar, int32_t* oi, float* os) {
   constexpr int E = kTopK / NT;
   static_assert(E >= 1 && (E & (E - 1)) == 0 && E * NT == kTopK, "power-of-two elements per thread");
   uint64_t* const s64 = reinterpret_cast<uint64_t*>(stage);
@@ -614,7 +619,7 @@ struct WGState {
   uint32_t hist[QPW][kBins1 / 2];  // per query: first-level counts of its candidates (packed)
   uint32_t rhist[kBins1 / 2];      // resolution scratch
   uint2 list[kListCap];            // boundary-bin candidates of one resolution
-  uint32_t small[kSmallRank];      // keys of the boundary sub-bin
+  uint32_t small[2 * kSmallRank];  // keys of the boundary sub-bin (per sub-group)
   float w[QPW][H];
   int cnt_w[QPW][4];               // per-warp append counts, published at check points
   int cnt_k[QPW];                  // entries in the current keep set
@@ -623,8 +628,8 @@ struct WGState {
   uint32_t thr_bin[QPW];           // admission threshold found by the query's scanning warp
   int pos[QPW];
   uint32_t scratch[64];
-  int sh[8];
-  int ctr[4];
+  int sh[16];                      // 8 per sub-group
+  int ctr[8];                      // 4 per sub-group
 };
 
 // Thread layout of the score kernel.  EW = epilogue warps per group: 4 (one warp per
@@ -903,7 +908,17 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
     uint2* const qcand =
         p.cand + (static_cast<size_t>(blockIdx.x) * (ALT ? QMAX * NWG : QMAX) + g * QPW) * kCandStride;
     uint2* const my_area = qcand + static_cast<size_t>(j0) * kCandStride + 2 * kTopK + qd * kWarpApp;
-    const ResolveSmem rs{st.rhist, st.list, st.small, st.scratch, st.sh, st.ctr};
+    const ResolveSmem rs{st.rhist, st.list, kListCap, st.small, st.scratch, st.sh, st.ctr};
+    // the prefill path's end-of-item selections run in sub-groups of NTS threads, one query
+    // each at a time, so that the latency of one query's passes overlaps another's; each
+    // sub-group has its own named barrier and its own share of the selection scratch, and
+    // the query's own first-level counts serve as its second-level counts
+    constexpr int kSub = (!ALT && QPW >= 2) ? 2 : 1;
+    constexpr int NTS = NTG / kSub;
+    const int sg = gtid / NTS, stid = gtid % NTS;
+    const int sbar = kSub == 1 ? bar : 3 + kSub * g + sg;
+    const ResolveSmem rsub{st.rhist, st.list + sg * (kListCap / kSub), kListCap / kSub, st.small + sg * kSmallRank,
+                           st.scratch + sg * 32, st.sh + sg * 8, st.ctr + sg * 4};
     const uint64_t pol_cand = l2_policy_evict_last();   // candidates are read back at the item's end
     int acc_ctr = 0;
 
@@ -1164,18 +1179,20 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
           if (j < nmine) st.cnt_w[j0 + j][qd] = cnt_r[j];
       }
       if (named_bar_or(bar, NTG, failed)) break;   // a failed wait ends every warp of the group
+      if (wi.chunk < 0) {
+        // output rows: query jj of the group is resolved by sub-group jj % kSub
 #pragma unroll 1
-      for (int jj = 0; jj < nloc; ++jj) {
-        const int t = wi.t0 + qbase + jj;
-        const CandView v = cands(jj);
-        const int n_valid = v.total();
-        if (wi.chunk < 0) {
+        for (int jj = sg; jj < nloc; jj += kSub) {
+          const int t = wi.t0 + qbase + jj;
+          const CandView v = cands(jj);
           int32_t* oi = p.idx_out + static_cast<size_t>(t) * kTopK;
           float* os = p.score_out ? p.score_out + static_cast<size_t>(t) * kTopK : nullptr;
           const int prefix = st.pos[jj] + 1;   // keys this query scores (<= 0 if invalid)
+          ResolveSmem rq = rsub;
+          if (kSub > 1) rq.rh = st.hist[jj];
           if (prefix <= kTopK) {
             // every position 0..prefix-1 is a candidate: place each at its own index
-            v.for_rounds<NTG>(gtid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
+            v.for_rounds<NTS>(stid, [&](const uint4 (&x)[kRoundU], const int (&lim)[kRoundU]) {
 #pragma unroll
               for (int e = 0; e < 2 * kRoundU; ++e) {
                 const uint2 c = round_entry(x, e);
@@ -1185,25 +1202,33 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
                 }
               }
             });
-            for (int s2 = max(prefix, 0) + gtid; s2 < kTopK; s2 += NTG) {
+            for (int s2 = max(prefix, 0) + stid; s2 < kTopK; s2 += NTS) {
               __stcs(oi + s2, -1);
               if (os) __stcs(os + s2, -INFINITY);
             }
           } else if constexpr (SORTED) {
             // the query's other keep set is not read by this selection: it stages the row
             uint2* const stage = qcand + static_cast<size_t>(jj) * kCandStride + (st.kcur[jj] ^ 1) * kTopK;
-            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+            resolve_topk<NTS>(v, st.hist[jj], kSub > 1, rq, stid, sbar, [&](int s2, uint32_t key, uint32_t pos) {
               stage[s2] = make_uint2(key, pos);
             });
-            named_bar_sync(bar, NTG);
-            sort_stage_and_emit<NTG>(stage, gtid, bar, oi, os);
+            named_bar_sync(sbar, NTS);
+            sort_stage_and_emit<NTS>(stage, stid, sbar, oi, os);
           } else {
-            resolve_topk<NTG>(v, st.hist[jj], false, rs, gtid, bar, [&](int s2, uint32_t key, uint32_t pos) {
+            resolve_topk<NTS>(v, st.hist[jj], kSub > 1, rq, stid, sbar, [&](int s2, uint32_t key, uint32_t pos) {
               __stcs(oi + s2, static_cast<int>(pos));
               if (os) __stcs(os + s2, ordered_to_float(key));
             });
           }
-        } else {
+          named_bar_sync(sbar, NTS);
+        }
+        if (kSub > 1) named_bar_sync(bar, NTG);   // every sub-group is done with the counts
+      } else {
+#pragma unroll 1
+        for (int jj = 0; jj < nloc; ++jj) {
+          const int t = wi.t0 + qbase + jj;
+          const CandView v = cands(jj);
+          const int n_valid = v.total();
           uint32_t* pk = p.part_keys + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
           int32_t* pi = p.part_idx + (static_cast<size_t>(t) * kMaxChunks + wi.chunk) * kTopK;
           uint32_t* const h = st.hist[jj];
@@ -1235,8 +1260,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
             if (wd & 0xFFFFu) atomicAdd(&qh[2 * i], wd & 0xFFFFu);
             if (wd >> 16) atomicAdd(&qh[2 * i + 1], wd >> 16);
           }
+          named_bar_sync(bar, NTG);
         }
-        named_bar_sync(bar, NTG);
       }
       // empty histograms for the next item
       for (int i = gtid; i < QPW * (kBins1 / 2); i += NTG) (&st.hist[0][0])[i] = 0u;
