@@ -762,6 +762,24 @@ def profile_call(d, spec, repeats):
     name, _, call = spec.partition(":")
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
+    if name == "project":
+        # the projections of one workload's first call (dsa_indexer_project), timed alone
+        st = setup_prefill(d, call, 0, device)
+        (a0, a1), qoff = st["bounds"][0], st["qoffs"][0]
+        ix = st["ix"]
+        for i in range(repeats + 1):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ix.project(st["hidden"][a0:a1], st["q_latent"][a0:a1], st["positions"][a0:a1], qoff, st["cache"],
+                       st["coff"], q_out=st["q"][a0:a1], w_out=st["w"][a0:a1])
+            e1.record()
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            r = projection_report(a1 - a0, ms, 1646.6, 6551.7)
+            print(f"{spec} call {i}: {ms:.4f} ms, {r['achieved_gbs']:.1f} GB/s, {r['achieved_tflops']:.1f} TFLOP/s",
+                  flush=True)
+        assert ix.device_error() == d.DSA_OK
+        return
     if name in ("decode_64", "decode_64_fp8"):
         fp8 = name.endswith("_fp8")
         ds = setup_decode(d, 0, device, fp8)

@@ -742,38 +742,28 @@ cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K
   p.err = e.err;
   p.timeout_ns = e.timeout_ns;
   const int nk = K / kBK;
-  // the contraction is split over a cluster of CTAs when it is long enough to share
-  if (e.n_heads == 64) {
-    if (nk >= 8) return launch_kw_cluster<8, 64>(tmA, tmB, p, s);
-    if (nk >= 4) return launch_kw_cluster<4, 64>(tmA, tmB, p, s);
-    if (nk >= 2) return launch_kw_cluster<2, 64>(tmA, tmB, p, s);
-    return cudaErrorInvalidValue;
+  const int tiles = (e.M + kBM - 1) / kBM;
+  // Few token tiles (decode): split the contraction over a cluster so that more SMs stream
+  // `hidden`.  Many tiles: the q GEMM runs next to this kernel, and one CTA per tile leaves it
+  // the most SMs (measured: 0.149 ms for both GEMMs at 8,192 tokens with one CTA per tile,
+  // 0.155 / 0.172 / 0.207 ms with clusters of 2 / 4 / 8).  The single-CTA kernel has the bf16,
+  // 32-head, no-rotary epilogue; the other forms use clusters of at least 2.
+  const bool plain = e.key8 == nullptr && e.rope_dim == 0 && e.n_heads == 32;
+  int cs = tiles <= 2 ? 8 : tiles <= 4 ? 4 : tiles <= 8 ? 2 : 1;
+  if (cs == 1 && !plain) cs = 2;
+  while (cs > 1 && nk < cs) cs >>= 1;   // at least one k-block per CTA of the cluster
+  if (cs == 1) {
+    if (!plain) return cudaErrorInvalidValue;
+    return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
   }
-  if (nk >= 8) return launch_kw_cluster<8, 32>(tmA, tmB, p, s);
-  if (nk >= 4) return launch_kw_cluster<4, 32>(tmA, tmB, p, s);
-  if (nk >= 2) return launch_kw_cluster<2, 32>(tmA, tmB, p, s);
-  return launch_proj<160, 5, EPI_KW>(tmA, tmB, p, 1, s);
-}
-
-cudaError_t launch_proj_q8(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N, uint8_t* q8_out,
-                           float* q_scale, int* err, uint64_t timeout_ns, cudaStream_t s) {
-  ProjParams p{};
-  p.M = M;
-  p.K = K;
-  p.q8_out = q8_out;
-  p.q_scale = q_scale;
-  p.ldq = N;
-  p.err = err;
-  p.timeout_ns = timeout_ns;
-  return launch_proj<256, 4, EPI_Q8>(tmA, tmB, p, N / 256, s);
-}
-
-cudaError_t launch_quantize_keys_fp8(int64_t n, const __nv_bfloat16* keys, uint8_t* out, float* scale,
-                                     cudaStream_t s) {
-  if (n <= 0) return cudaSuccess;
-  const int64_t blocks = (n + 7) / 8;
-  quantize_keys_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(n, keys, out, scale);
-  return cudaGetLastError();
+  if (e.n_heads == 64) {
+    if (cs == 8) return launch_kw_cluster<8, 64>(tmA, tmB, p, s);
+    if (cs == 4) return launch_kw_cluster<4, 64>(tmA, tmB, p, s);
+    return launch_kw_cluster<2, 64>(tmA, tmB, p, s);
+  }
+  if (cs == 8) return launch_kw_cluster<8, 32>(tmA, tmB, p, s);
+  if (cs == 4) return launch_kw_cluster<4, 32>(tmA, tmB, p, s);
+  return launch_kw_cluster<2, 32>(tmA, tmB, p, s);
 }
 
 cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,
