@@ -766,6 +766,27 @@ cudaError_t launch_proj_kw(const CUtensorMap& tmA, const CUtensorMap& tmB, int K
   return launch_kw_cluster<2, 32>(tmA, tmB, p, s);
 }
 
+cudaError_t launch_proj_q8(const CUtensorMap& tmA, const CUtensorMap& tmB, int M, int K, int N, uint8_t* q8_out,
+                           float* q_scale, int* err, uint64_t timeout_ns, cudaStream_t s) {
+  ProjParams p{};
+  p.M = M;
+  p.K = K;
+  p.q8_out = q8_out;
+  p.q_scale = q_scale;
+  p.ldq = N;
+  p.err = err;
+  p.timeout_ns = timeout_ns;
+  return launch_proj<256, 4, EPI_Q8>(tmA, tmB, p, N / 256, s);
+}
+
+cudaError_t launch_quantize_keys_fp8(int64_t n, const __nv_bfloat16* keys, uint8_t* out, float* scale,
+                                     cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = (n + 7) / 8;
+  quantize_keys_fp8_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(n, keys, out, scale);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_key_norm(int64_t n, const float* raw, __nv_bfloat16* out, const float* gamma,
                             const float* beta, float eps, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
