@@ -1329,6 +1329,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   };
   if (tid < 4) ctr[tid] = 0;
   for (int i = tid; i < kBins1; i += kMergeThreads) hist2[i] = 0u;
+  // every key this thread visits (entries 4 g .. 4 g + 3 for g = tid + kMergeThreads j), requested
+  // at once so that their latency overlaps the counts' (the lists hold at most kMaxChunks * kTopK
+  // entries: kMergeJ 16-byte words per thread); empty slots are 0 and below every score
+  constexpr int kMergeJ = kMaxChunks * kTopK / 4 / kMergeThreads;
+  uint4 kq[kMergeJ];
+#pragma unroll
+  for (int j = 0; j < kMergeJ; ++j) {
+    const int g = tid + kMergeThreads * j;
+    kq[j] = g < n / 4 ? reinterpret_cast<const uint4*>(keys)[g] : make_uint4(0u, 0u, 0u, 0u);
+  }
   // 1. boundary bin from the counts (two bins per thread), then clear them
   constexpr int kBPT = kBins1 / kMergeThreads;
   static_assert(kBPT == 2, "two bins per thread");
@@ -1362,18 +1372,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   const uint32_t b1 = static_cast<uint32_t>(min(max(sh[0], 0), kBins1 - 1));
   const int above = min(max(sh[1], 0), kTopK);
   const int need = kTopK - above;
-  // 2. second-level counts of b1's entries
-#pragma unroll 4
-  for (int g = tid; g < n / 4; g += kMergeThreads) {
-    const uint4 kk = reinterpret_cast<const uint4*>(keys)[g];
-    const int4 ii = reinterpret_cast<const int4*>(pos)[g];
+  // 2. second-level counts of b1's entries (a key of an empty slot is 0: never in b1, as b1
+  // holds the kTopK-th largest of at least kTopK valid entries)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t key = u4_get(kk, j);
-      if (i4_get(ii, j) >= 0 && (key >> kBinShift) == b1)
+  for (int j = 0; j < kMergeJ; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t key = u4_get(kq[j], e);
+      if (key != 0u && (key >> kBinShift) == b1)
         asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(smem_u32(&hist2[(key >> kSubShift) & (kBins1 - 1)])) : "memory");
     }
-  }
   named_bar_sync(1, kMergeThreads);
 #pragma unroll
   for (int i = 0; i < kBPT; ++i) {
@@ -1401,35 +1409,42 @@ __global__ void __launch_bounds__(kMergeThreads) merge_kernel(const uint32_t* __
   const uint32_t b2 = static_cast<uint32_t>(min(max(sh[2], 0), kBins1 - 1));
   const int above2 = min(max(sh[3], 0), need);
   const uint32_t lo = (b1 << kBinShift) | (b2 << kSubShift), hi = lo + ((1u << kSubShift) - 1u);
-  // 3. one pass: entries above lo to their slots, the entries of [lo, hi] to the list
+  // 3. entries above lo to their slots, the entries of [lo, hi] to the list; positions are
+  // read only for the 16-byte words that hold one of those (all such reads issued together)
   const uint32_t lt = lanemask_lt();
-#pragma unroll 2
-  for (int base = 0; base < n / 4; base += kMergeThreads) {
-    const int g = base + tid;
-    uint4 kk = make_uint4(0u, 0u, 0u, 0u);
-    int4 ii = make_int4(-1, -1, -1, -1);
-    if (g < n / 4) {
-      kk = reinterpret_cast<const uint4*>(keys)[g];
-      ii = reinterpret_cast<const int4*>(pos)[g];
+  constexpr int kHalfJ = kMergeJ / 2;   // positions are read for half of the words at a time (registers)
+#pragma unroll
+  for (int jh = 0; jh < kMergeJ; jh += kHalfJ) {
+    int4 iq[kHalfJ];
+#pragma unroll
+    for (int jj = 0; jj < kHalfJ; ++jj) {
+      const int j = jh + jj;
+      const int g = tid + kMergeThreads * j;
+      const bool any = u4_get(kq[j], 0) >= lo || u4_get(kq[j], 1) >= lo || u4_get(kq[j], 2) >= lo ||
+                       u4_get(kq[j], 3) >= lo;
+      iq[jj] = (any && g < n / 4) ? reinterpret_cast<const int4*>(pos)[g] : make_int4(-1, -1, -1, -1);
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t key = u4_get(kk, j);
-      const int p = i4_get(ii, j);
-      const bool up = p >= 0 && key > hi, mid = p >= 0 && key >= lo && key <= hi;
-      const uint32_t bu = __ballot_sync(0xffffffffu, up), bm = __ballot_sync(0xffffffffu, mid);
-      if (bu | bm) {
-        int ou = 0, om = 0;
-        if (lane == 0) {
-          if (bu) ou = atomicAdd(&ctr[0], __popc(bu));
-          if (bm) om = atomicAdd(&ctr[1], __popc(bm));
-        }
-        ou = __shfl_sync(0xffffffffu, ou, 0) + __popc(bu & lt);
-        om = __shfl_sync(0xffffffffu, om, 0) + __popc(bm & lt);
-        if (up && ou < kTopK) out(ou, key, p);
-        if (mid && om < kMergeList) {
-          lkeys[om] = key;
-          lidx[om] = p;
+    for (int jj = 0; jj < kHalfJ; ++jj) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t key = u4_get(kq[jh + jj], e);
+        const int p = i4_get(iq[jj], e);
+        const bool up = p >= 0 && key > hi, mid = p >= 0 && key >= lo && key <= hi;
+        const uint32_t bu = __ballot_sync(0xffffffffu, up), bm = __ballot_sync(0xffffffffu, mid);
+        if (bu | bm) {
+          int ou = 0, om = 0;
+          if (lane == 0) {
+            if (bu) ou = atomicAdd(&ctr[0], __popc(bu));
+            if (bm) om = atomicAdd(&ctr[1], __popc(bm));
+          }
+          ou = __shfl_sync(0xffffffffu, ou, 0) + __popc(bu & lt);
+          om = __shfl_sync(0xffffffffu, om, 0) + __popc(bm & lt);
+          if (up && ou < kTopK) out(ou, key, p);
+          if (mid && om < kMergeList) {
+            lkeys[om] = key;
+            lidx[om] = p;
+          }
         }
       }
     }
