@@ -758,7 +758,7 @@ def profile_call(d, spec, repeats):
     """A small case for ncu captures: one dsa_indexer_topk call of a workload, repeated.
     spec is WORKLOAD[:CALL]; for the chunked prefill the cache is filled by projecting the
     chunks up to CALL one at a time, so the device holds one chunk's tensors, the key
-    cache and the workspace (well under 1 GB).  Prints the call's CUDA-event times."""
+    cache and the workspace (well under 1 GB); CALL "all" runs every chunk's call.  Prints the call's CUDA-event times."""
     name, _, call = spec.partition(":")
     device = torch.device("cuda", 0)
     torch.cuda.set_device(device)
@@ -797,9 +797,27 @@ def profile_call(d, spec, repeats):
     cfg = W.WORKLOADS[name]
     wts = W.make_weights(cfg["weight_seed"])
     to = lambda t: t.to(device).contiguous()  # noqa: E731
+    def run_calls(label, ix, q, w, pos, qoff, cache, coff, pairs):
+        idx = torch.empty((q.shape[0], 2048), dtype=torch.int32, device=device)
+        sc = torch.empty((q.shape[0], 2048), dtype=torch.float32, device=device)
+        torch.cuda.synchronize()
+        for i in range(repeats):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ix.topk(q, w, pos, qoff, cache, coff, idx_out=idx, score_out=sc)
+            e1.record()
+            e1.synchronize()
+            ms = e0.elapsed_time(e1)
+            print(f"{label} call {i}: {ms:.4f} ms, {pairs / ms / 1e6:.2f} Gpairs/s, "
+                  f"{pairs * FLOP_PER_PAIR / ms / 1e9:.1f} TFLOP/s", flush=True)
+        assert ix.device_error() == d.DSA_OK
+
     if cfg["kind"] == "chunked":
+        # CALL = one chunk's call (the earlier chunks only fill the cache), or "all": every
+        # chunk's call in order, each right after its chunk was projected
         S, C = cfg["seq_len"], cfg["chunk"]
-        c_last = int(call or S // C - 1)
+        every = call == "all"
+        c_last = S // C - 1 if (every or not call) else int(call)
         ix = _make_indexer(d, wts, device, C)
         cache = torch.zeros((S, 128), dtype=torch.bfloat16, device=device)
         coff = to(torch.tensor([0, S], dtype=torch.int64))
@@ -808,6 +826,10 @@ def profile_call(d, spec, repeats):
             b = W.make_prefill(cfg["act_seed"], [C], start_positions=[c * C], cache_lens=[S], sub=c)
             pos = to(b.positions)
             q, w = ix.project(to(b.hidden), to(b.q_latent), pos, qoff, cache, coff)
+            if every:
+                run_calls(f"{name}:{c}", ix, q, w, pos, qoff, cache, coff, W.causal_pairs(b.positions))
+        if every:
+            return
         pairs = W.causal_pairs(b.positions)
     else:
         b = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
@@ -818,19 +840,7 @@ def profile_call(d, spec, repeats):
         if "heavy_frac" in cfg:
             cache[to(W.heavy_hitter_rows(cfg["act_seed"], b.cache_offsets, cfg["heavy_frac"]))] *= 4
         pairs = W.causal_pairs(b.positions)
-    idx = torch.empty((q.shape[0], 2048), dtype=torch.int32, device=device)
-    sc = torch.empty((q.shape[0], 2048), dtype=torch.float32, device=device)
-    torch.cuda.synchronize()
-    for i in range(repeats):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        ix.topk(q, w, pos, qoff, cache, coff, idx_out=idx, score_out=sc)
-        e1.record()
-        e1.synchronize()
-        ms = e0.elapsed_time(e1)
-        print(f"{spec} call {i}: {ms:.4f} ms, {pairs / ms / 1e6:.2f} Gpairs/s, "
-              f"{pairs * FLOP_PER_PAIR / ms / 1e9:.1f} TFLOP/s", flush=True)
-    assert ix.device_error() == d.DSA_OK
+    run_calls(spec, ix, q, w, pos, qoff, cache, coff, pairs)
 
 
 # ------------------------------------------------------------------------------------------ main
