@@ -665,12 +665,19 @@ struct ScoreCfg {
   static constexpr int kQHalf = QMAX * H * 128;       // bytes of one 128-byte-wide half of the Q tile
   static constexpr int kKHalf = kKeyTile * 128;       // 16 KB
   static constexpr int kKStage = kHalves * kKHalf;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kHalves * kQHalf;
-  static constexpr int kWGOff = kKOff + STAGES * kKStage;
+  static constexpr int kQBytes = kHalves * kQHalf;   // one item's Q tile
   static constexpr int kWGBytes = (static_cast<int>(sizeof(WGState<kQPW, H>)) + 15) / 16 * 16;
+  // small Q tiles (the split path: one query per item) are double-buffered where shared memory
+  // allows, so that the next item's tile loads while this item's last key tiles are scored
+  static constexpr int kQBufs =
+      (kQBytes <= 16384 &&
+       2 * kQBytes + STAGES * kKStage + NWG * kWGBytes + 8 * (2 * STAGES + 2 * kTotalBufs + 9) + 1088 <= 232448)
+          ? 2 : 1;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQBufs * kQBytes;
+  static constexpr int kWGOff = kKOff + STAGES * kKStage;
   static constexpr int kBarOff = kWGOff + NWG * kWGBytes;
-  static constexpr int kNumBars = 2 * STAGES + 2 * kTotalBufs + 2 + 4 + 1;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kTotalBufs + 2 * kQBufs + 4 + 1;
   static constexpr int kMiscOff = kBarOff + 8 * kNumBars;
   static constexpr int kSmemBytes = kMiscOff + 64 + 1024;
   static_assert(kTmemNeed <= 512, "TMEM holds 512 columns");
@@ -724,9 +731,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + C::kTotalBufs;
-  uint64_t* q_full = acc_empty + C::kTotalBufs;
-  uint64_t* q_empty = q_full + 1;
-  uint64_t* sched_full = q_empty + 1;
+  uint64_t* q_full = acc_empty + C::kTotalBufs;   // [kQBufs]
+  uint64_t* q_empty = q_full + C::kQBufs;         // [kQBufs]
+  uint64_t* sched_full = q_empty + C::kQBufs;
   uint64_t* sched_empty = sched_full + 2;
   uint64_t* mma_done = sched_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
@@ -744,8 +751,10 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], C::kConsumers);
     }
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    for (int b = 0; b < C::kQBufs; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sched_full[i], 1);
       mbar_init(&sched_empty[i], 1 + C::kConsumers);
@@ -805,10 +814,12 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         const WorkItem wi = p.items[it];
         const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
         if (kt1 <= kt0) continue;
-        if (qloads > 0 && !mbar_wait(q_empty, (qloads - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(q_full, C::kHalves * C::kQHalf);
-        tma_load_2d_hint(sQ, &tmQ, q_full, 0, wi.t0 * H, pol_q);
-        if constexpr (!kFp8) tma_load_2d_hint(sQ + C::kQHalf, &tmQ, q_full, 64, wi.t0 * H, pol_q);
+        const int qb = qloads % C::kQBufs;
+        if (qloads >= C::kQBufs && !mbar_wait(&q_empty[qb], ((qloads / C::kQBufs) - 1) & 1, wc)) break;
+        uint8_t* const dq = sQ + qb * C::kQBytes;
+        mbar_arrive_expect_tx(&q_full[qb], C::kQBytes);
+        tma_load_2d_hint(dq, &tmQ, &q_full[qb], 0, wi.t0 * H, pol_q);
+        if constexpr (!kFp8) tma_load_2d_hint(dq + C::kQHalf, &tmQ, &q_full[qb], 64, wi.t0 * H, pol_q);
         ++qloads;
         const int row0 = static_cast<int>(p.cache_offsets[wi.b]);
         bool ok = true;
@@ -836,7 +847,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       if (*abort_flag) {
         for (int ks = (kstage > STAGES ? kstage - STAGES : 0); ks < kstage; ++ks)
           drain_wait(&full[ks % STAGES], (ks / STAGES) & 1);
-        if (qloads > 0) drain_wait(q_full, (qloads - 1) & 1);
+        for (int ql = (qloads > C::kQBufs ? qloads - C::kQBufs : 0); ql < qloads; ++ql)
+          drain_wait(&q_full[ql % C::kQBufs], (ql / C::kQBufs) & 1);
       }
     }
   } else if (warp == 1) {
@@ -844,7 +856,6 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
     if (lane == 0) {
       int kstage = 0, qloads = 0;
       int acc0 = 0, acc1 = 0;   // tiles given to group 0 / group 1 (one shared ring without ALT)
-      const uint32_t qa = smem_u32(sQ);
       for (int local = 0;; ++local) {
         const int slot = local & 1;
         if (!mbar_wait(&sched_full[slot], (local >> 1) & 1, wc)) break;
@@ -854,8 +865,10 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         const WorkItem wi = p.items[it];
         const int kt0 = wi.k_begin / kKeyTile, kt1 = (wi.k_end + kKeyTile - 1) / kKeyTile;
         if (kt1 <= kt0) continue;
-        if (!mbar_wait(q_full, qloads & 1, wc)) break;
+        const int qb = qloads % C::kQBufs;
+        if (!mbar_wait(&q_full[qb], (qloads / C::kQBufs) & 1, wc)) break;
         ++qloads;
+        const uint32_t qa = smem_u32(sQ + qb * C::kQBytes);
         tc_fence_after();
         const uint32_t idesc = kFp8 ? umma_idesc_e4m3(kKeyTile, wi.nq * H) : umma_idesc_bf16(kKeyTile, wi.nq * H);
         const bool second = ALT && (local & 1);   // with ALT, the CTA's odd items go to group 1
@@ -879,7 +892,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
             umma_tile_k128<C::kKHalf, C::kQHalf>(tmem + ab * C::kAccCols, smem_u32(sK + s * C::kKStage), qa, idesc,
                                                 &empty[s], &acc_full[ab]);
         }
-        umma_commit(q_empty);
+        umma_commit(&q_empty[qb]);
         if (!ok) break;
       }
       umma_commit(mma_done);
@@ -1005,81 +1018,106 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
 #pragma unroll
       for (int j = 0; j < QPH; ++j) thr_f[j] = -INFINITY;
       acc_ctr += kt1 - kt0;
-      for (int kt = kt0; kt < kt1; ++kt, s_pos += kKeyTile) {
-        // FP8: this thread's key scale, requested before the accumulator wait (the producer
-        // brought its line into L2 when it loaded the tile); rows past the item's last scored
-        // key read as 0
-        const float sk = (kFp8 && s_pos < wi.k_end) ? __ldg(p.key_scale + kbase + s_pos) : 0.f;
-        const uint32_t aoff = static_cast<uint32_t>(aslot) * 8u;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait_addr(afull0 + aoff, phase, wc));
-        tc_fence_after();
-        const uint32_t tcol = tcol0 + aslot * C::kAccCols;
-        if (++aslot == ACC_BUFS) {
-          aslot = 0;
-          phase ^= 1u;
+      // a warp that holds one 32-column block per tile (one query of 32 heads: the split path)
+      // takes two tiles per iteration, so that the two tiles' loads and arithmetic overlap
+      constexpr int CB = QPH * HB;
+      constexpr int TPI = CB == 1 ? 2 : 1;
+      for (int kt = kt0; kt < kt1; kt += TPI, s_pos += TPI * kKeyTile) {
+        const int ntile = (TPI == 2 && kt + 1 < kt1) ? 2 : 1;
+        // FP8: this thread's key scales, requested before the accumulator waits (the producer
+        // brought their lines into L2 when it loaded the tiles); rows past the item's last
+        // scored key read as 0
+        float sk[TPI];
+        uint32_t tcol[TPI], aoff[TPI];
+        bool ok = true;
+#pragma unroll
+        for (int u = 0; u < TPI; ++u) {
+          if (u < ntile) {
+            const int sp = s_pos + u * kKeyTile;
+            sk[u] = (kFp8 && sp < wi.k_end) ? __ldg(p.key_scale + kbase + sp) : 0.f;
+            aoff[u] = static_cast<uint32_t>(aslot) * 8u;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait_addr(afull0 + aoff[u], phase, wc));
+            tcol[u] = tcol0 + aslot * C::kAccCols;
+            if (++aslot == ACC_BUFS) {
+              aslot = 0;
+              phase ^= 1u;
+            }
+          }
         }
+        tc_fence_after();
         if (ok) {
-          // this warp's columns of the tile, as 16x256b blocks of 32 columns (CB of them: its
-          // queries' head blocks, contiguous): one TMEM round trip per tile
-          constexpr int CB = QPH * HB;
-          uint32_t v[2 * CB][16];   // [lane half h][column block cb] at h * CB + cb
+          // this warp's columns of the tiles, as 16x256b blocks of 32 columns (CB per tile: its
+          // queries' head blocks, contiguous): one TMEM round trip per iteration
+          uint32_t v[TPI][2 * CB][16];   // [tile][lane half h][column block cb] at [u][h * CB + cb]
           constexpr uint32_t kHalf16 = 16u << 16;   // lane offset of the quadrant's upper half
           if constexpr (CB == 2) {
-            tmem_ld4_16x256b_x4_wait(tcol, tcol + 32, tcol + kHalf16, tcol + kHalf16 + 32, v);
+            tmem_ld4_16x256b_x4_wait(tcol[0], tcol[0] + 32, tcol[0] + kHalf16, tcol[0] + kHalf16 + 32, v[0]);
           } else {
             static_assert(CB == 1, "one or two column blocks per epilogue warp");
-            tmem_ld2_16x256b_x4_wait(tcol, tcol + kHalf16, v);
+            if (ntile == 2)
+              tmem_ld4_16x256b_x4_wait(tcol[0], tcol[0] + kHalf16, tcol[1], tcol[1] + kHalf16,
+                                       reinterpret_cast<uint32_t(&)[4][16]>(v));
+            else
+              tmem_ld2_16x256b_x4_wait(tcol[0], tcol[0] + kHalf16, v[0]);
           }
           tc_fence_before();
           __syncwarp();
-          if (lane == 0)   // TMEM buffer free for the next MMA
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(aempty0 + aoff) : "memory");
-          // partial sums over this thread's 8 heads of each head block, for its two rows of
-          // each lane half
-          float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
+          if (lane == 0) {   // TMEM buffers free for the next MMAs
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+            for (int u = 0; u < TPI; ++u)
+              if (u < ntile) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(aempty0 + aoff[u]) : "memory");
+          }
+#pragma unroll
+          for (int u = 0; u < TPI; ++u) {
+            if (u >= ntile) break;
+            const int sp = s_pos + u * kKeyTile;   // this thread's key position in tile u
+            // partial sums over this thread's 8 heads of each head block, for its two rows of
+            // each lane half
+            float part[4 * QPH];   // [2 h + row][query j] at (2 h + row) * QPH + j
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int j = 0; j < QPH; ++j) {
+                float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int hb = 0; hb < HB; ++hb) {
+                  const uint32_t(&x)[16] = v[u][h * CB + j * HB + hb];
+#pragma unroll
+                  for (int blk = 0; blk < 4; ++blk) {
+                    a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
+                                                                fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
+                    b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
+                                                                fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
+                  }
+                }
+                part[(2 * h) * QPH + j] = a.x + a.y;
+                part[(2 * h + 1) * QPH + j] = b.x + b.y;
+              }
+            float score[QPH];
+            sum_over_quad<QPH>(part, score, lane);
+            if constexpr (kFp8) {
+              // the key row's scale (positive) multiplies every head's ReLU term
+#pragma unroll
+              for (int j = 0; j < QPH; ++j) score[j] *= sk[u];
+            }
+            // admit (key, position) into this warp's area of each of its queries and count it;
+            // the append counts stay warp-uniform in registers.  The float comparison with the
+            // threshold admits what the order-preserving key comparison admits (and -0 against
+            // a threshold of +0, a harmless extra candidate)
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
-              float2 a = make_float2(0.f, 0.f), b = make_float2(0.f, 0.f);
-#pragma unroll
-              for (int hb = 0; hb < HB; ++hb) {
-                const uint32_t(&x)[16] = v[h * CB + j * HB + hb];
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                  a = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk]), 0.f),
-                                                              fmaxf(__uint_as_float(x[4 * blk + 1]), 0.f)), a);
-                  b = ffma2(w2[j * HB + hb][blk], make_float2(fmaxf(__uint_as_float(x[4 * blk + 2]), 0.f),
-                                                              fmaxf(__uint_as_float(x[4 * blk + 3]), 0.f)), b);
+              if (j >= nmine) break;
+              const bool pass = (sp <= pos_r[j]) && (score[j] >= thr_f[j]);
+              const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+              if (bal) {
+                if (pass) {
+                  const uint32_t uk = float_to_ordered(score[j]);
+                  st_global_u2_hint(&my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)],
+                                    make_uint2(uk, static_cast<uint32_t>(sp)), pol_cand);
+                  count_key(st.hist[j0 + j], uk >> kBinShift);
                 }
+                cnt_r[j] += __popc(bal);
               }
-              part[(2 * h) * QPH + j] = a.x + a.y;
-              part[(2 * h + 1) * QPH + j] = b.x + b.y;
-            }
-          float score[QPH];
-          sum_over_quad<QPH>(part, score, lane);
-          if constexpr (kFp8) {
-            // the key row's scale (positive) multiplies every head's ReLU term
-#pragma unroll
-            for (int j = 0; j < QPH; ++j) score[j] *= sk;
-          }
-          // admit (key, position) into this warp's area of each of its queries and count it;
-          // the append counts stay warp-uniform in registers.  The float comparison with the
-          // threshold admits what the order-preserving key comparison admits (and -0 against
-          // a threshold of +0, a harmless extra candidate)
-#pragma unroll
-          for (int j = 0; j < QPH; ++j) {
-            if (j >= nmine) break;
-            const bool pass = (s_pos <= pos_r[j]) && (score[j] >= thr_f[j]);
-            const uint32_t bal = __ballot_sync(0xffffffffu, pass);
-            if (bal) {
-              if (pass) {
-                const uint32_t u = float_to_ordered(score[j]);
-                st_global_u2_hint(&my_area[static_cast<size_t>(j) * kCandStride + cnt_r[j] + __popc(bal & lt)],
-                                  make_uint2(u, static_cast<uint32_t>(s_pos)), pol_cand);
-                count_key(st.hist[j0 + j], u >> kBinShift);
-              }
-              cnt_r[j] += __popc(bal);
             }
           }
         } else {
@@ -1087,7 +1125,8 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         }
         // check point every kCheckTiles tiles (the same tiles for every warp of the group); a
         // long item also checks the append areas' capacity at every kCapTiles-th tile
-        if (--to_check == 0 && kt + 1 < kt1) {
+        to_check -= ntile;
+        if (to_check <= 0 && kt + ntile < kt1) {
           to_check = kCheckTiles;
           bool need = false;
           const bool cap_check = long_item;   // every check point is a capacity point (kCapTiles == kCheckTiles)
