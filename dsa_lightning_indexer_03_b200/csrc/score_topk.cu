@@ -1630,6 +1630,7 @@ __device__ __forceinline__ int sequence_of_token(const int32_t* qoff, int B, int
 
 constexpr int kPrepCopy = 2048;   // offset arrays up to this length are searched in shared memory
 constexpr int kPrepTok = 1024;    // validated positions and chunk counts of up to this many queries stay in shared memory
+constexpr int kLenBuckets = 1024; // item lengths in key tiles (longer items share the last bucket)
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __shared__ int warp_sums[32];
@@ -1640,6 +1641,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
   __shared__ int s_base[kPrepCopy + 1];   // copy of the items' owner bases when n_owners < kPrepCopy
   __shared__ int s_pe[kPrepTok];          // validated positions when T <= kPrepTok
   __shared__ int s_nch[kPrepTok];         // key chunks per query when T <= kPrepTok
+  __shared__ int s_len[kLenBuckets];      // split path: items per length bucket, then bucket starts
   const TopkWorkspace& ws = p.ws;
   // the score kernel may start its prologue now; it waits for this grid's results
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -1730,25 +1732,50 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
     *ws.work_counter = 0;
   }
   __syncthreads();
-  // 4. items, written in reverse order of (owner, tile) so the longest prefixes come first
-  for (int i = threadIdx.x; i < total; i += kPrepThreads) {
-    const int o = owner_of(base, n_owners, i);
-    const int local = i - base[o];
+  // 4. items.  Split path: item i is chunk `local` of query o; the items are written longest
+  // first (a counting sort by length in key tiles, buckets in descending order), so that the
+  // dynamically scheduled CTAs end on the shortest chunks and finish together.  Prefill path:
+  // reverse order of (sequence, query group), which puts each sequence's longest prefixes
+  // first.
+  auto split_item = [&](int i) {
+    const int t = owner_of(base, n_owners, i);
+    const int local = i - base[t];
+    const int n = pe[t] + 1;
+    const int nch = nchk[t];
+    const int cl = chunk_len_for(n, target);
     WorkItem wi;
     wi.pad0 = wi.pad1 = 0;
-    if (p.split) {
-      const int t = o;
-      const int n = pe[t] + 1;
-      const int nch = nchk[t];
-      const int cl = chunk_len_for(n, target);
-      wi.t0 = t;
-      wi.nq = 1;
-      wi.b = sequence_of_token(qoff, p.B, t);
-      wi.k_begin = (nch > 1) ? local * cl : 0;
-      wi.k_end = (nch > 1) ? min(n, (local + 1) * cl) : n;
-      wi.chunk = (nch > 1) ? local : -1;
-    } else {
-      const int b = o;
+    wi.t0 = t;
+    wi.nq = 1;
+    wi.b = sequence_of_token(qoff, p.B, t);
+    wi.k_begin = (nch > 1) ? local * cl : 0;
+    wi.k_end = (nch > 1) ? min(n, (local + 1) * cl) : n;
+    wi.chunk = (nch > 1) ? local : -1;
+    return wi;
+  };
+  // bucket of an item: kLenBuckets - 1 - (length in tiles, capped), so ascending buckets hold
+  // descending lengths
+  auto len_bucket = [](const WorkItem& wi) {
+    const int tiles = (wi.k_end - wi.k_begin + kKeyTile - 1) / kKeyTile;
+    return kLenBuckets - 1 - (tiles < kLenBuckets - 1 ? tiles : kLenBuckets - 1);
+  };
+  if (p.split) {
+    for (int b = threadIdx.x; b < kLenBuckets; b += kPrepThreads) s_len[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < total; i += kPrepThreads) atomicAdd(&s_len[len_bucket(split_item(i))], 1);
+    __syncthreads();
+    block_exclusive_scan(s_len, kLenBuckets, warp_sums);
+    __syncthreads();
+    for (int i = threadIdx.x; i < total; i += kPrepThreads) {
+      const WorkItem wi = split_item(i);
+      ws.items[atomicAdd(&s_len[len_bucket(wi)], 1)] = wi;
+    }
+  } else {
+    for (int i = threadIdx.x; i < total; i += kPrepThreads) {
+      const int b = owner_of(base, n_owners, i);
+      const int local = i - base[b];
+      WorkItem wi;
+      wi.pad0 = wi.pad1 = 0;
       const int t0 = qoff[b] + local * p.qpi;
       const int nq = min(p.qpi, qoff[b + 1] - t0);
       int kend = 0;
@@ -1759,8 +1786,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(PrepParams p) {
       wi.k_begin = 0;
       wi.k_end = kend;
       wi.chunk = -1;
+      ws.items[total - 1 - i] = wi;
     }
-    ws.items[total - 1 - i] = wi;
   }
 }
 
