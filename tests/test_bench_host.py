@@ -105,13 +105,20 @@ def test_time_steps_splits_projection_and_topk(monkeypatch):
 
 
 def test_prefill_roofline_arithmetic():
-    peaks = dict(bf16_tflops=1650.0, source="measured")
+    peaks = dict(bf16_tflops=1650.0, bf16_tflops_sustained=1400.0, source="measured")
     r = bench.prefill_roofline(8_590_000_128, 100.0, peaks, None)
     tflops = 8_590_000_128 * 8192 / 0.1 / 1e12
     assert abs(r["achieved"] - tflops) < 0.01
-    assert abs(r["frac"] - tflops / 1650.0) < 1e-4
+    assert abs(r["frac"] - tflops / 1650.0) < 1e-4      # short timed region: burst peak
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["gpairs_score_topk"] - 85.9) < 0.001
+    # a timed region of seconds of back-to-back launches is held to the sustained peak
+    r = bench.prefill_roofline(8_590_000_128, 100.0, peaks, None, timed_s=2.0)
+    assert r["peak"] == 1400.0 and abs(r["frac"] - tflops / 1400.0) < 1e-4
+    assert abs(r["frac_burst"] - tflops / 1650.0) < 1e-4 and "sustained" in r["peak_source"]
+    # FP8 operands: the nominal 2x of the bf16 figure
+    r = bench.prefill_roofline(8_590_000_128, 100.0, peaks, None, fp8=True, timed_s=0.1)
+    assert r["peak"] == 3300.0
 
 
 def test_headline_is_the_long_context_chunked_prefill():
