@@ -476,8 +476,8 @@ def run_prefill(d, name, rank, device, steps, warmup, flush, peaks, mx, clk=None
     rec = {"workload": name + ("_fp8" if fp8 else ""), "metric": "indexer score+top-2048 Gpairs/s (prefill)",
            "value": None, "unit": "Gpairs/s", "ms_per_step": round(ms, 4), "causal_pairs": st["pairs"],
            "tokens": st["T"], "calls_per_step": n_calls,
-           "roofline": prefill_roofline(st["pairs"], topk_avg, peaks, _profile_traffic(f"score_topk:{name}"), fp8,
-                                        timed_s),
+           "roofline": prefill_roofline(st["pairs"], topk_avg, peaks,
+                                        _profile_traffic(f"score_topk:{name}" + ("_fp8" if fp8 else "")), fp8, timed_s),
            "projections": projection_report(st["T"], proj_avg, tensor_peak(peaks, timed_s)[0], peaks["hbm_gbs"]),
            "device_error": err, "gpu_launches_per_step": n_calls * (LAUNCHES["project"] + LAUNCHES["topk"])}
     rec["roofline"]["ms_per_launch"] = round(topk_avg / n_calls, 4)
