@@ -26,8 +26,9 @@
 //              key reaches the query's admission threshold: the pair goes to the warp's own
 //              append area (warp ballot, warp-uniform counts in registers, no atomics) and
 //              the key is counted in the query's first-level histogram in shared memory.
-//              Every kCheckTiles tiles the threshold rises to the lowest bin that still
-//              holds the query's best 2,048 counted keys (a warp scan of the histogram);
+//              Every 16 tiles (24 in items of more than 512 tiles) the threshold rises to
+//              the lowest bin that still holds the query's best 2,048 counted keys (a warp
+//              scan of the histogram);
 //              in long items a nearly full append area is compacted to the exact best
 //              2,048.  At the end of the item each query's candidates are reduced to
 //              exactly the top 2,048 in one pass (resolve_topk) and written out.
@@ -180,9 +181,13 @@ constexpr int kBinShift = 21;                  // first-level bin = key >> kBinS
 constexpr int kBins1 = 1 << (32 - kBinShift);  // 2,048 bins
 constexpr int kSubShift = kBinShift - 11;      // second-level bin = next 11 bits
 constexpr int kListCap = 1024;                 // boundary-bin candidates gathered in shared memory
-constexpr int kCheckTiles = 16;                // key tiles between threshold updates
-constexpr int kCapTiles = kCheckTiles;         // key tiles between capacity checks (long items)
-constexpr int kCheckMargin = kCapTiles * 32;   // appends one warp can make per query in that time
+constexpr int kCheckTiles = 16;                // key tiles between threshold updates (and capacity checks)
+// items of more than kLongCheckItem tiles space their check points kLongCheckTiles apart: late in
+// a long prefix the threshold moves slowly, and the check points (a scan of the counts, a group
+// barrier, the capacity test) cost more than the extra admissions they save (measured on 96 K to
+// 128 K-key items: 3-5 % faster; on 32 K to 64 K-key items 1-2 % slower, so those keep 16)
+constexpr int kLongCheckItem = 512;
+constexpr int kLongCheckTiles = 24;
 constexpr int kSmallRank = 32;                 // boundary sub-bins up to this size are ranked by one warp
 
 // An admission threshold held as a float, raised to the order-preserving key t if that is
@@ -1013,7 +1018,9 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
       const uint32_t tcol0 = tlane + slot0 * C::kAccCols + (qbase + j0) * H;
       const uint32_t afull0 = smem_u32(&acc_full[slot0]), aempty0 = smem_u32(&acc_empty[slot0]);
       int s_pos = kt0 * kKeyTile + r;
-      int to_check = kCheckTiles;
+      const int check_tiles = (kt1 - kt0 > kLongCheckItem) ? kLongCheckTiles : kCheckTiles;
+      const int check_margin = check_tiles * 32;   // appends one warp can make per query between checks
+      int to_check = check_tiles;
       float thr_f[QPH];
 #pragma unroll
       for (int j = 0; j < QPH; ++j) thr_f[j] = -INFINITY;
@@ -1123,18 +1130,18 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
         } else {
           failed = true;
         }
-        // check point every kCheckTiles tiles (the same tiles for every warp of the group); a
-        // long item also checks the append areas' capacity at every kCapTiles-th tile
+        // check point every check_tiles tiles (the same tiles for every warp of the group); in
+        // a long item every check point also checks the append areas' capacity
         to_check -= ntile;
         if (to_check <= 0 && kt + ntile < kt1) {
-          to_check = kCheckTiles;
+          to_check = check_tiles;
           bool need = false;
-          const bool cap_check = long_item;   // every check point is a capacity point (kCapTiles == kCheckTiles)
+          const bool cap_check = long_item;
           if (cap_check) {
 #pragma unroll
             for (int j = 0; j < QPH; ++j) {
               if (j < nmine) {
-                need |= cnt_r[j] > kWarpApp - kCheckMargin;
+                need |= cnt_r[j] > kWarpApp - check_margin;
                 if (lane == 0) st.cnt_w[j0 + j][qd] = cnt_r[j];
               }
             }
@@ -1145,7 +1152,7 @@ __global__ void __launch_bounds__(ScoreCfg<QMAX, STAGES, ACC_BUFS, NWG, EW, ALT,
             for (int jj = 0; jj < nloc; ++jj) {
               // st.*[jj] is read by every thread here and written only after the barriers below
               const CandView v = cands(jj);
-              if (max(max(v.n0, v.n1), max(v.n2, v.n3)) <= kWarpApp - kCheckMargin) continue;
+              if (max(max(v.n0, v.n1), max(v.n2, v.n3)) <= kWarpApp - check_margin) continue;
               uint2* const q = qcand + static_cast<size_t>(jj) * kCandStride;
               const int kc = st.kcur[jj];
               const int n_valid = v.total();
