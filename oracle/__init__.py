@@ -29,3 +29,9 @@ from .indexer_oracle import (  # noqa: F401
     fp8_index_scores,
     topk_fp8,
 )
+from .sparse_mla_oracle import (  # noqa: F401
+    MLA_HEADS,
+    MLA_DIM,
+    MLA_LATENT,
+    sparse_mla,
+)

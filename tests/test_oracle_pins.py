@@ -538,3 +538,93 @@ def test_project_64_heads_with_rope():
     with pytest.raises(ValueError):
         oracle.project(x, xq, ws["W_q"], ws["W_k"], ws["W_w"], ws["ln_gamma"], ws["ln_beta"], n_heads=H,
                        head_dim=D, rope_dim=64)
+
+
+# ---------------------------------------------------------------- sparse MLA over the selection
+
+def _mla_case(seed=0, T=3, H=4, n_rows=(40, 30), K=16, pad=4):
+    rng = np.random.default_rng(seed)
+    co = np.concatenate([[0], np.cumsum(n_rows)])
+    qo = np.array([0, 2, T])                      # queries 0,1 in sequence 0; the rest in sequence 1
+    kv = rng.standard_normal((int(co[-1]), oracle.MLA_DIM))
+    q = rng.standard_normal((T, H, oracle.MLA_DIM)) * 0.1
+    idx = np.full((T, K), -1, np.int64)
+    for t in range(T):
+        b = 0 if t < 2 else 1
+        idx[t, : K - pad] = rng.choice(n_rows[b], K - pad, replace=False)
+    return q, kv, co, qo, idx
+
+
+def test_sparse_mla_matches_torch_attention():
+    import torch
+    q, kv, co, qo, idx = _mla_case()
+    scale = 1.0 / np.sqrt(192.0)
+    o, lse = oracle.sparse_mla(q, kv, co, qo, idx, scale)
+    for t in range(q.shape[0]):
+        b = 0 if t < 2 else 1
+        rows = torch.tensor(kv[co[b] + idx[t][idx[t] >= 0]])
+        qt = torch.tensor(q[t])[None]                        # [1, H, 576] as (batch, len, dim)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            qt, rows[None], rows[None, :, : oracle.MLA_LATENT], scale=scale)[0]
+        assert np.allclose(o[t], ref.numpy(), rtol=1e-10, atol=1e-12)
+        s = scale * (torch.tensor(q[t]) @ rows.T)
+        assert np.allclose(lse[t], torch.logsumexp(s, dim=1).numpy(), rtol=1e-12)
+
+
+def test_sparse_mla_brute_force_loops():
+    q, kv, co, qo, idx = _mla_case(seed=3, T=2, H=2, n_rows=(9, 7), K=5, pad=1)
+    scale = 0.7
+    o, lse = oracle.sparse_mla(q, kv, co, qo, idx, scale)
+    import math
+    for t in range(2):
+        base = 0                                   # both queries are in sequence 0
+        for h in range(2):
+            sc = []
+            for j in idx[t]:
+                if j < 0:
+                    continue
+                row = kv[base + j]
+                sc.append((scale * sum(q[t, h, d] * row[d] for d in range(oracle.MLA_DIM)), row))
+            mx = max(s for s, _ in sc)
+            z = sum(math.exp(s - mx) for s, _ in sc)
+            for d in (0, 100, 511):
+                want = sum(math.exp(s - mx) / z * row[d] for s, row in sc)
+                assert abs(o[t, h, d] - want) < 1e-12
+            assert abs(lse[t, h] - (mx + math.log(z))) < 1e-12
+
+
+def test_sparse_mla_special_cases():
+    q, kv, co, qo, idx = _mla_case(seed=5)
+    scale = 0.3
+    # one selected token: the output is that token's latent, lse its score
+    one = np.full_like(idx, -1)
+    one[:, 0] = 7
+    o, lse = oracle.sparse_mla(q, kv, co, qo, one, scale)
+    for t in range(q.shape[0]):
+        row = kv[co[0 if t < 2 else 1] + 7]
+        assert np.allclose(o[t], np.broadcast_to(row[: oracle.MLA_LATENT], o[t].shape))
+        assert np.allclose(lse[t], scale * q[t] @ row)
+    # identical rows: the output is the row whatever the query; lse = score + log(count)
+    kv2 = np.tile(kv[:1], (kv.shape[0], 1))
+    o, lse = oracle.sparse_mla(q, kv2, co, qo, idx, scale)
+    n = (idx >= 0).sum(axis=1)
+    assert np.allclose(o, kv2[0, : oracle.MLA_LATENT])
+    assert np.allclose(lse, scale * (q @ kv2[0]) + np.log(n)[:, None])
+    # -1 entries are no token: dropping them changes nothing
+    comp = np.array([np.concatenate([r[r >= 0], r[r < 0]]) for r in idx])
+    o1, l1 = oracle.sparse_mla(q, kv, co, qo, idx, scale)
+    o2, l2 = oracle.sparse_mla(q, kv, co, qo, comp, scale)
+    assert np.allclose(o1, o2) and np.allclose(l1, l2)
+    # nothing selected: zeros and -inf
+    o, lse = oracle.sparse_mla(q, kv, co, qo, np.full_like(idx, -1), scale)
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+
+
+def test_sparse_mla_reads_the_query_sequence_rows():
+    # a planted difference in sequence 1's rows changes only sequence 1's queries
+    q, kv, co, qo, idx = _mla_case(seed=7)
+    o1, _ = oracle.sparse_mla(q, kv, co, qo, idx, 0.5)
+    kv2 = kv.copy()
+    kv2[co[1]:] += 1.0
+    o2, _ = oracle.sparse_mla(q, kv2, co, qo, idx, 0.5)
+    assert np.allclose(o1[:2], o2[:2]) and not np.allclose(o1[2:], o2[2:])
