@@ -48,7 +48,11 @@ ALL_WORKLOADS = PREFILL_WORKLOADS + ["decode_64"]
 # kernels of this library launched by one call of each entry point (the timed region holds
 # nothing else of ours): project = q GEMM + k|w GEMM with the LayerNorm epilogue;
 # topk = prep + score kernel, plus the merge on the split-key path
-LAUNCHES = {"project": 2, "topk": 2, "topk_split": 3}
+LAUNCHES = {"project": 2, "topk": 2, "topk_split": 3, "sparse_mla": 1}
+
+# sparse MLA over the selection ('Latent attention (MLA)' row): 96 heads, 576 cached values
+# per token (512 latent + 64 rope), 2,048 selected tokens per query, scale 1/sqrt(192)
+MLA_SCALE = 192 ** -0.5
 
 
 # ------------------------------------------------------------------------------------------ helpers
@@ -507,6 +511,51 @@ def run_decode(d, rank, device, steps, warmup, flush, peaks, mx, fp8=False):
     return ds, rec, gbs
 
 
+def setup_mla_decode(seed_offset, device, small=False):
+    """The decode step's sparse MLA: 64 sequences of 16,384..131,072 cached 576-value rows,
+    one query of 96 heads each, 2,048 selected positions per query (distinct, uniform over
+    the sequence: the access pattern of an unsorted top-k row).  small: sequences of 2,048
+    rows (every row selected once, in random order; a 151 MB cache for profiler captures)."""
+    cfg = W.WORKLOADS["decode_64"]
+    lengths = W.decode_lengths(cfg["act_seed"] + seed_offset, cfg["batch"], cfg["L_min"], cfg["L_max"])
+    if small:
+        lengths = torch.full_like(lengths, 2048)
+    b = W.make_mla(cfg["act_seed"] + seed_offset, lengths.tolist(), [1] * cfg["batch"], device=str(device))
+    to = lambda t: t.to(device).contiguous()  # noqa: E731
+    T, H, k = b.q.shape[0], b.q.shape[1], b.idx.shape[1]
+    ms = dict(q=to(b.q), kv=b.kv, coff=to(b.cache_offsets), qoff=to(b.q_seq_offsets), idx=to(b.idx),
+              out=torch.empty((T, H, 512), dtype=torch.bfloat16, device=device),
+              lse=torch.empty((T, H), dtype=torch.float32, device=device), T=T, H=H, k=k)
+    # algorithmic bytes: every selected row once, q, the index rows, out and lse
+    ms["bytes"] = T * k * 576 * 2 + T * H * 576 * 2 + T * k * 4 + T * H * (512 * 2 + 4)
+    # useful flops: q . row over 576 values and p . latent over 512, per head and token
+    ms["flops"] = 2 * T * H * k * (576 + 512)
+    torch.cuda.synchronize()
+    return ms
+
+
+def mla_call(ix, ms):
+    ix.sparse_mla(ms["q"], ms["kv"], ms["coff"], ms["qoff"], ms["idx"], MLA_SCALE, out=ms["out"], lse=ms["lse"])
+
+
+def run_mla_decode(d, ix, rank, device, steps, warmup, flush, peaks, mx):
+    ms = setup_mla_decode(rank, device)
+    fn = lambda spans: spans.span("topk", lambda: mla_call(ix, ms))  # noqa: E731
+    _time_steps(fn, warmup, flush)
+    _, t, _ = _time_steps(fn, steps, flush)
+    dms = mx(statistics.mean(t))
+    gbs = ms["bytes"] / (dms * 1e-3) / 1e9
+    rec = {"workload": "sparse_mla_decode_64", "metric": "sparse MLA decode GB/s", "value": None, "unit": "GB/s",
+           "queries": ms["T"], "heads": ms["H"], "selected": ms["k"], "ms_per_step": round(dms, 4),
+           "tflops": round(ms["flops"] / (dms * 1e-3) / 1e12, 2), "algorithmic_bytes": ms["bytes"],
+           "roofline": {"bound": "hbm", "achieved": round(gbs, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": _profile_traffic("sparse_mla:decode_64"),
+                        "kernel": "sparse_mla_kernel (dsa_indexer_sparse_mla)", "ms_per_launch": round(dms, 4),
+                        "peak_source": peaks["source"] + " HBM copy"},
+           "device_error": ix.device_error(), "gpu_launches_per_step": LAUNCHES["sparse_mla"]}
+    return ms, rec, gbs
+
+
 def gpu_arm(args, rank, world, local_rank, dist):
     import dsa_lightning_indexer_03_b200 as d
     from dsa_lightning_indexer_03_b200 import build as B
@@ -561,6 +610,15 @@ def gpu_arm(args, rank, world, local_rank, dist):
             subs[rec["workload"]] = rec
             del ds
             torch.cuda.empty_cache()
+        # the consumer of the selection: sparse MLA attention of the decode batch
+        ix = _make_indexer(d, W.make_weights(W.WORKLOADS["decode_64"]["weight_seed"], hidden_dim=256,
+                                             q_latent_dim=128), device, 256)
+        ms, rec, gbs = run_mla_decode(d, ix, rank, device, n, args.warmup, flush, peaks, mx)
+        rec["value"] = round(gbs * world, 2)
+        rec["steps"] = n
+        subs[rec["workload"]] = rec
+        del ms, ix
+        torch.cuda.empty_cache()
         # the FP8 cache on the 8,192-token prefill (FP8 tensor-core scoring)
         s2, rec, ms2 = run_prefill(d, "prefill_8k", rank, device, n, args.warmup, flush, peaks, mx, fp8=True)
         rec["value"] = round(whole_job_rate(s2["pairs"], world, ms2) / 1e9, 3)
@@ -811,6 +869,20 @@ def profile_call(d, spec, repeats):
             ms = sum(a.elapsed_time(b) for k, a, b in spans if k == "topk")
             print(f"{spec} call {i}: {ms:.4f} ms, {ds['bytes'] / ms / 1e6:.1f} GB/s, 0 TFLOP/s", flush=True)
         assert ds["ix"].device_error() == d.DSA_OK
+        return
+    if name in ("sparse_mla_decode_64", "sparse_mla_small"):
+        ix = _make_indexer(d, W.make_weights(0, hidden_dim=256, q_latent_dim=128), device, 256)
+        ms = setup_mla_decode(0, device, small=name == "sparse_mla_small")
+        for i in range(repeats):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mla_call(ix, ms)
+            e1.record()
+            e1.synchronize()
+            t = e0.elapsed_time(e1)
+            print(f"{spec} call {i}: {t:.4f} ms, {ms['bytes'] / t / 1e6:.1f} GB/s, "
+                  f"{ms['flops'] / t / 1e9:.1f} TFLOP/s", flush=True)
+        assert ix.device_error() == d.DSA_OK
         return
     cfg = W.WORKLOADS[name]
     wts = W.make_weights(cfg["weight_seed"])

@@ -60,6 +60,8 @@ SIGNATURES = {
     "dsa_indexer_topk_fp8": (ctypes.c_int, [_vp, _i64, _vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _i64, _vp, _vp, _vp,
                                              _u32, _vp]),
     "dsa_indexer_topk_reuse": (ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "dsa_indexer_sparse_mla": (ctypes.c_int, [_vp, _i64, _vp, _i32, _vp, _i64, _vp, _vp, _i32, _vp, _i32,
+                                              ctypes.c_float, _vp, _vp, _vp]),
     "dsa_indexer_device_error": (ctypes.c_int, [_vp]),
     "dsa_indexer_noalloc_device_error": (ctypes.c_int, [_vp]),
     "dsa_indexer_selftest_wait_timeout": (ctypes.c_int, [_i64, _vp]),

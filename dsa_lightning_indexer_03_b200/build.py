@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG_DIR, "csrc")
 ROOT = os.path.dirname(PKG_DIR)
 LIB_NAME = "libdsa_indexer.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
-SOURCES = ["api.cu", "proj.cu", "score_topk.cu", "noalloc.cu", "reuse.cu"]
+SOURCES = ["api.cu", "proj.cu", "score_topk.cu", "noalloc.cu", "reuse.cu", "sparse_mla.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", os.path.join(ROOT, "include")]

@@ -438,6 +438,41 @@ dsa_status_t dsa_indexer_topk_reuse(dsa_indexer_t h, int64_t n_draft, const int3
   return DSA_OK;
 }
 
+dsa_status_t dsa_indexer_sparse_mla(dsa_indexer_t h, int64_t T, const void* q, int32_t n_heads, const void* kv_cache,
+                                    int64_t cache_rows, const int64_t* cache_offsets, const int32_t* q_seq_offsets,
+                                    int32_t B, const int32_t* idx, int32_t k_sel, float scale, void* out, float* lse,
+                                    void* stream) {
+  if (!h || T < 0 || B < 1 || k_sel < 0) return DSA_ERR_INVALID_ARG;
+  if (n_heads < 1 || n_heads > 96 || !(scale > 0.f) || !std::isfinite(scale)) return DSA_ERR_INVALID_ARG;
+  if (k_sel > 2048) return DSA_ERR_UNSUPPORTED;
+  if (T == 0) return DSA_OK;
+  if (T > (int64_t(1) << 31) - 1 || cache_rows < 1 || cache_rows > (int64_t(1) << 40)) return DSA_ERR_INVALID_ARG;
+  if (!q || !kv_cache || !cache_offsets || !q_seq_offsets || (!idx && k_sel > 0) || !out || !lse)
+    return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out) || (reinterpret_cast<uintptr_t>(idx) & 3) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3) || (reinterpret_cast<uintptr_t>(cache_offsets) & 7) ||
+      (reinterpret_cast<uintptr_t>(q_seq_offsets) & 3))
+    return DSA_ERR_INVALID_ARG;
+  SparseMlaArgs a;
+  a.T = static_cast<int>(T);
+  a.B = B;
+  a.H = n_heads;
+  a.k_sel = k_sel;
+  a.cache_rows = cache_rows;
+  a.q = q;
+  a.kv_cache = kv_cache;
+  a.cache_offsets = cache_offsets;
+  a.q_seq_offsets = q_seq_offsets;
+  a.idx = idx;
+  a.scale = scale;
+  a.out = out;
+  a.lse = lse;
+  a.err = h->ws.err;
+  a.timeout_ns = timeout_ns();
+  if (launch_sparse_mla(a, static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 dsa_status_t dsa_indexer_device_error(dsa_indexer_t h) {
   if (!h) return DSA_ERR_INVALID_ARG;
   if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;

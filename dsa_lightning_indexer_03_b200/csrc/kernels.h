@@ -124,6 +124,27 @@ cudaError_t launch_topk(const TopkArgs& a, const TopkWorkspace& ws, const CUtens
 cudaError_t launch_reuse_rows(int n, const int32_t* anchor, int n_src, const int32_t* src_idx, const float* src_score,
                               int32_t* dst_idx, float* dst_score, int* err, int num_sms, cudaStream_t s);
 
+// ---------------------------------------------------------------- sparse MLA
+// Attention of T queries (H <= 96 heads of 576 values) over the k_sel cache rows each query's
+// idx row selects (positions inside its sequence, -1 = none); out bf16 [T, H, 512], lse
+// fp32 [T, H] (natural log; -inf and zeros for a query with no token).
+struct SparseMlaArgs {
+  int T, B, H, k_sel;
+  int64_t cache_rows;
+  const void* q;                  // bf16 [T, H, 576]
+  const void* kv_cache;           // bf16 [cache_rows, 576]
+  const int64_t* cache_offsets;   // [B+1]
+  const int32_t* q_seq_offsets;   // [B+1]
+  const int32_t* idx;             // [T, k_sel]
+  float scale;
+  void* out;                      // bf16 [T, H, 512]
+  float* lse;                     // [T, H]
+  int* err;
+  uint64_t timeout_ns;
+};
+
+cudaError_t launch_sparse_mla(const SparseMlaArgs& a, cudaStream_t s);
+
 cudaError_t launch_wait_timeout_selftest(int* status, uint64_t timeout_ns, cudaStream_t s);
 
 // Limit of every bounded pipeline wait in the library's kernels: 2 s, or

@@ -247,6 +247,34 @@ class Indexer:
               "dsa_indexer_topk_reuse")
         return idx_out, score_out
 
+    def sparse_mla(self, q, kv_cache, cache_offsets, q_seq_offsets, idx, scale, out=None, lse=None, stream=None):
+        """Attention of each query (q bf16 [T, H, 576]) over the kv_cache rows (bf16 [rows, 576])
+        its idx row selects (int32 [T, k_sel], positions in its sequence, -1 = none), latent
+        form: returns out bf16 [T, H, 512] and lse fp32 [T, H]."""
+        dev = self.device
+        _need(q, "q", torch.bfloat16, dev)
+        _need(kv_cache, "kv_cache", torch.bfloat16, dev)
+        _need(cache_offsets, "cache_offsets", torch.int64, dev)
+        _need(q_seq_offsets, "q_seq_offsets", torch.int32, dev)
+        _need(idx, "idx", torch.int32, dev)
+        if q.dim() != 3 or q.shape[2] != 576 or kv_cache.dim() != 2 or kv_cache.shape[1] != 576:
+            raise ValueError("q must be [T, H, 576] and kv_cache [rows, 576]")
+        T, H = q.shape[0], q.shape[1]
+        if idx.dim() != 2 or idx.shape[0] != T:
+            raise ValueError("idx must be [T, k_sel]")
+        if out is None:
+            out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=dev)
+        if lse is None:
+            lse = torch.empty((T, H), dtype=torch.float32, device=dev)
+        _need(out, "out", torch.bfloat16, dev)
+        _need(lse, "lse", torch.float32, dev)
+        check(self._lib.dsa_indexer_sparse_mla(self._h, T, _ptr(q), H, _ptr(kv_cache), kv_cache.shape[0],
+                                               _ptr(cache_offsets), _ptr(q_seq_offsets), cache_offsets.numel() - 1,
+                                               _ptr(idx), idx.shape[1], float(scale), _ptr(out), _ptr(lse),
+                                               _stream(stream)),
+              "dsa_indexer_sparse_mla")
+        return out, lse
+
     def device_error(self) -> int:
         """Synchronises and returns (then clears) the handle's device error status."""
         with torch.cuda.device(self.device):

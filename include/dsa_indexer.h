@@ -261,6 +261,34 @@ dsa_status_t dsa_indexer_topk_noalloc(int64_t T, const void* q, const float* w, 
  * counterpart on the pages, as for dsa_indexer_topk_noalloc). */
 dsa_status_t dsa_indexer_noalloc_device_error(void* stream);
 
+/* Sparse MLA attention over the indexer's selection ('Latent attention (MLA)' row of
+ * the pages "Qwen3.5-397B-A17B vs Kimi K3.1 Pro" and "Kimi K3.1 Pro vs Gemma 4 31B":
+ * 96 heads; keys and values come from a 512-dim latent plus a 64-dim shared key slot, 576
+ * cached values per token; each query attends only to the 2,048 tokens the indexer
+ * selects).  It runs in the latent ("absorbed") form: a head's query is 576 values (its
+ * no-rope part already taken into the latent space), the score of a selected token s is
+ *     x[h,s] = scale * (q[t,h] . kv[s])          over all 576 values,
+ * and the value is the row's first 512 values (the latent):
+ *     out[t,h] = sum_s softmax_s(x[h,.]) * kv[s][0..511],   lse[t,h] = ln sum_s exp(x[h,s]).
+ *   q             bf16 [T, n_heads, 576], n_heads in 1..96
+ *   kv_cache      bf16 [cache_rows, 576]; token s of sequence b is row cache_offsets[b] + s
+ *   cache_offsets int64 [B+1], q_seq_offsets int32 [B+1]: as for dsa_indexer_project
+ *   idx           int32 [T, k_sel]: positions inside the query's sequence, -1 = no token
+ *                 (the idx_out of dsa_indexer_topk, k_sel = top_k); a position may repeat
+ *                 and then counts once per entry; k_sel <= 2,048 (larger:
+ *                 DSA_ERR_UNSUPPORTED); k_sel = 0 (idx may be NULL) gives every query no token
+ *   scale         > 0 (e.g. 1/sqrt(192) for 128 + 64-dim query/key heads)
+ *   out           bf16 [T, n_heads, 512];  lse fp32 [T, n_heads]
+ * A query with no valid entry gets out = 0 and lse = -inf.  An entry at or past its
+ * sequence's row count is skipped and sets DSA_ERR_DEVICE_BOUNDS; malformed offsets set it
+ * too and give the affected queries no token.  Scores and the softmax weights' sum are
+ * fp32; the weights multiply the latent as bf16 (fp32 accumulate).  T = 0 is a no-op;
+ * asynchronous on `stream`. */
+dsa_status_t dsa_indexer_sparse_mla(dsa_indexer_t h, int64_t T, const void* q, int32_t n_heads, const void* kv_cache,
+                                    int64_t cache_rows, const int64_t* cache_offsets, const int32_t* q_seq_offsets,
+                                    int32_t B, const int32_t* idx, int32_t k_sel, float scale, void* out, float* lse,
+                                    void* stream);
+
 /* Synchronises the device, then returns DSA_OK or the first device-side error
  * recorded since the last call (DSA_ERR_DEVICE_BOUNDS, DSA_ERR_DEVICE_TIMEOUT)
  * and clears the error word. */

@@ -93,6 +93,8 @@ def test_argument_validation_without_a_gpu(lib):
     assert lib.dsa_indexer_topk_fp8(None, 1, *([None] * 5), 1, None, None, 1, None, None, None, 0, None) == 1
     assert lib.dsa_indexer_quantize_keys_fp8(None, 1, None, None, None, None) == 1
     assert lib.dsa_indexer_topk_reuse(None, 1, None, 1, None, None, None, None, None) == 1
+    assert lib.dsa_indexer_sparse_mla(None, 1, None, 96, None, 1, None, None, 1, None, 2048, 0.07, None, None,
+                                      None) == 1
     assert lib.dsa_indexer_destroy(None) == 1
     assert lib.dsa_indexer_device_error(None) == 1
     assert lib.dsa_indexer_selftest_wait_timeout(0, None) == 1

@@ -25,4 +25,7 @@ from .generate import (  # noqa: F401
     causal_pairs,
     make_scoring_inputs,
     stratified_rows,
+    MLA_DIMS,
+    MlaBatch,
+    make_mla,
 )

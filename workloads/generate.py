@@ -39,6 +39,11 @@ WORKLOADS = {
 # stream ids: one per tensor kind
 _S_WQ, _S_WK, _S_WW, _S_GAMMA, _S_BETA = 1, 2, 3, 4, 5
 _S_HIDDEN, _S_QLAT, _S_LENS, _S_RAWK, _S_HEAVY = 11, 12, 13, 14, 15
+_S_MLA_Q, _S_MLA_KV, _S_MLA_IDX = 21, 22, 23
+
+# Sparse MLA consumer ('Latent attention (MLA)' row): 96 heads, 576 cached values per token
+# (512 latent + 64 rope key), 2,048 selected tokens per query.
+MLA_DIMS = dict(n_heads=96, dim=576, latent=512, k_sel=2048)
 
 
 def _gen(seed: int, stream: int, sub: int = 0) -> torch.Generator:
@@ -212,3 +217,48 @@ def stratified_rows(q_seq_offsets, n: int, seed: int = 0, chunk: int | None = No
     while len(picked) < min(n, T):   # a draw that hit an included row: draw again
         picked.add(int(torch.randint(0, T, (1,), generator=g)))
     return torch.tensor(sorted(picked), dtype=torch.int64)
+
+
+@dataclass
+class MlaBatch:
+    q: torch.Tensor              # bf16 [T, H, 576]
+    kv: torch.Tensor             # bf16 [rows, 576]
+    cache_offsets: torch.Tensor  # int64 [B+1]
+    q_seq_offsets: torch.Tensor  # int32 [B+1]
+    idx: torch.Tensor            # int32 [T, k_sel], positions in the query's sequence, -1 = none
+
+
+def make_mla(seed: int, lengths, queries_per_seq, n_heads: int = 96, k_sel: int = 2048, q_std: float = 1.0,
+             pad: int = 0, device: str = "cpu") -> MlaBatch:
+    """Inputs of the sparse MLA step: sequence b holds lengths[b] cached 576-value rows (bf16
+    N(0, 1): the normalised latent and rope key) and queries_per_seq[b] queries (bf16
+    N(0, q_std^2) per value).  Each query selects min(k_sel - pad, L_b) distinct positions of
+    its sequence in random order (as an unsorted top-k row would hold them); the rest of the
+    row is -1.  The cache is drawn on `device` (a large decode cache is drawn on the GPU with
+    a seeded CUDA generator); everything else on the CPU."""
+    lengths = [int(v) for v in lengths]
+    qps = [int(v) for v in queries_per_seq]
+    B = len(lengths)
+    T = sum(qps)
+    cache_offsets = torch.zeros(B + 1, dtype=torch.int64)
+    cache_offsets[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0)
+    q_seq_offsets = torch.zeros(B + 1, dtype=torch.int32)
+    q_seq_offsets[1:] = torch.cumsum(torch.tensor(qps, dtype=torch.int64), 0).to(torch.int32)
+    rows = int(cache_offsets[-1])
+    q = _normal(_gen(seed, _S_MLA_Q), (T, n_heads, MLA_DIMS["dim"]), q_std).to(torch.bfloat16)
+    if device == "cpu":
+        kv = _normal(_gen(seed, _S_MLA_KV), (rows, MLA_DIMS["dim"])).to(torch.bfloat16)
+    else:
+        g = torch.Generator(device=device)
+        g.manual_seed((int(seed) * 1_000_003 + _S_MLA_KV * 7919) & 0x7FFF_FFFF_FFFF)
+        kv = torch.randn((rows, MLA_DIMS["dim"]), generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
+    idx = torch.full((T, k_sel), -1, dtype=torch.int32)
+    g = _gen(seed, _S_MLA_IDX)
+    t = 0
+    for b in range(B):
+        n = min(k_sel - pad, lengths[b])
+        for _ in range(qps[b]):
+            if n > 0:
+                idx[t, :n] = torch.randperm(lengths[b], generator=g)[:n].to(torch.int32)
+            t += 1
+    return MlaBatch(q, kv, cache_offsets, q_seq_offsets, idx)
