@@ -120,3 +120,20 @@ def check_sorted(gpu_idx: np.ndarray, gpu_score: np.ndarray, rows, positions, I_
         assert np.all(I[a] >= I[b] - band), f"row {rows[r]}: order contradicts the oracle outside the band"
         open_pairs += int(np.sum(np.abs(I[a] - I[b]) <= band))
     return open_pairs
+
+
+def mla_tolerances(q_t, rows, o_ref_t, scale):
+    """Bounds of the sparse MLA check for one query (q_t [H, 576], the selected rows [n, 576]
+    in float64, the oracle's o [H, 512]): per value, |o - o_ref| <= 1.01 U (spread + |o_ref|)
+    + e_s spread + 1e-5 with U = 2^-8 (bf16 unit roundoff: the weights enter P.V as bf16 and
+    o is written as bf16), spread = max_j |v_jd - o_d| over the selected latents and
+    e_s = 6 sqrt(576) 2^-24 scale |q_h| max_j |row_j| (a six-sigma random-walk allowance for
+    the fp32 score sums); per head, |lse - lse_ref| <= 1.01 U + e_s + 1e-5."""
+    U = 2.0 ** -8
+    if rows.shape[0] == 0:
+        return np.full(o_ref_t.shape, 1e-5), np.full(o_ref_t.shape[0], 1e-5)
+    v = rows[:, :512]
+    spread = np.maximum(v.max(0)[None, :] - o_ref_t, o_ref_t - v.min(0)[None, :])
+    e_s = 6 * np.sqrt(576) * 2.0 ** -24 * scale * np.linalg.norm(q_t, axis=1) * np.linalg.norm(rows, axis=1).max()
+    o_tol = 1.01 * U * (spread + np.abs(o_ref_t)) + e_s[:, None] * spread + 1e-5
+    return o_tol, 1.01 * U + e_s + 1e-5

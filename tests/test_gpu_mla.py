@@ -16,7 +16,7 @@ import torch
 
 import oracle
 import workloads as W
-from _parity import f64
+from _parity import f64, mla_tolerances
 
 pytestmark = pytest.mark.gpu
 
@@ -61,13 +61,7 @@ def _selected_rows(batch, t):
 
 def _tolerances(q_t, rows, o_ref_t, scale=SCALE):
     """Per-value bound on |o - o_ref| and per-head bound on |lse - lse_ref| of one query."""
-    if rows.shape[0] == 0:
-        return np.full(o_ref_t.shape, 1e-5), np.full(o_ref_t.shape[0], 1e-5)
-    v = rows[:, :512]
-    spread = np.maximum(v.max(0)[None, :] - o_ref_t, o_ref_t - v.min(0)[None, :])
-    e_s = 6 * np.sqrt(576) * 2.0 ** -24 * scale * np.linalg.norm(q_t, axis=1) * np.linalg.norm(rows, axis=1).max()
-    o_tol = 1.01 * U * (spread + np.abs(o_ref_t)) + e_s[:, None] * spread + 1e-5
-    return o_tol, 1.01 * U + e_s + 1e-5
+    return mla_tolerances(q_t, rows, o_ref_t, scale)
 
 
 def _ref(batch, scale=SCALE, rows=None):
