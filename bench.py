@@ -511,6 +511,14 @@ def run_decode(d, rank, device, steps, warmup, flush, peaks, mx, fp8=False):
     return ds, rec, gbs
 
 
+def mla_bytes_flops(T, H, k):
+    """Algorithmic bytes of a sparse MLA call (every selected 1,152-byte row once, q, the index
+    rows, out and lse) and its useful flops (q . row over 576 values and p . latent over 512,
+    per head and selected token)."""
+    return (T * k * 576 * 2 + T * H * 576 * 2 + T * k * 4 + T * H * (512 * 2 + 4),
+            2 * T * H * k * (576 + 512))
+
+
 def setup_mla_decode(seed_offset, device, small=False):
     """The decode step's sparse MLA: 64 sequences of 16,384..131,072 cached 576-value rows,
     one query of 96 heads each, 2,048 selected positions per query (distinct, uniform over
@@ -526,10 +534,7 @@ def setup_mla_decode(seed_offset, device, small=False):
     ms = dict(q=to(b.q), kv=b.kv, coff=to(b.cache_offsets), qoff=to(b.q_seq_offsets), idx=to(b.idx),
               out=torch.empty((T, H, 512), dtype=torch.bfloat16, device=device),
               lse=torch.empty((T, H), dtype=torch.float32, device=device), T=T, H=H, k=k)
-    # algorithmic bytes: every selected row once, q, the index rows, out and lse
-    ms["bytes"] = T * k * 576 * 2 + T * H * 576 * 2 + T * k * 4 + T * H * (512 * 2 + 4)
-    # useful flops: q . row over 576 values and p . latent over 512, per head and token
-    ms["flops"] = 2 * T * H * k * (576 + 512)
+    ms["bytes"], ms["flops"] = mla_bytes_flops(T, H, k)
     torch.cuda.synchronize()
     return ms
 

@@ -144,3 +144,28 @@ def test_stratified_rows_cover_chunk_edges_and_the_topk_boundary():
         assert p in r
     # every 1/64 of the range holds a sampled row
     assert len({t * 64 // S for t in r}) == 64
+
+
+def test_mla_inputs_are_seeded_distinct_selections_padded_with_minus_one():
+    import torch
+    import workloads as W
+    a = W.make_mla(3, [5000, 100], [2, 3], n_heads=8, k_sel=256, pad=6)
+    b = W.make_mla(3, [5000, 100], [2, 3], n_heads=8, k_sel=256, pad=6)
+    assert torch.equal(a.idx, b.idx) and torch.equal(a.q.view(torch.int16), b.q.view(torch.int16))
+    assert a.q.shape == (5, 8, 576) and a.kv.shape == (5100, 576) and a.idx.shape == (5, 256)
+    assert a.cache_offsets.tolist() == [0, 5000, 5100] and a.q_seq_offsets.tolist() == [0, 2, 5]
+    for t in range(5):
+        L = 5000 if t < 2 else 100
+        row = a.idx[t]
+        n = min(256 - 6, L)
+        assert torch.all(row[n:] == -1)
+        sel = row[:n]
+        assert torch.all((sel >= 0) & (sel < L)) and sel.unique().numel() == n
+
+
+def test_mla_decode_record_bytes_and_flops():
+    # the decode batch (64 queries x 96 heads x 2,048 rows): 2,048 rows x 1,152 B + q 96 x 1,152 B
+    # + idx 8 KB + out 96 x 1,024 B + lse 384 B per query; 2 x 96 x 2,048 x 1,088 flop per query
+    per_query = 2048 * 1152 + 96 * 1152 + 8192 + 96 * 1024 + 384
+    assert bench.mla_bytes_flops(64, 96, 2048) == (64 * per_query, 64 * 2 * 96 * 2048 * 1088)
+    assert bench.mla_bytes_flops(64, 96, 2048)[0] == 164_913_152
