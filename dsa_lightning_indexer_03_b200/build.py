@@ -37,12 +37,19 @@ def _inputs():
 
 
 def source_hash() -> str:
-    """Short hash of the CUDA sources: ties recorded profile figures to the kernels they measured."""
+    """Short hash of the CUDA sources' code: ties recorded profile figures to the kernels they
+    measured.  Comments and blank lines are left out, so editing a comment keeps the figures."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in sorted(SOURCES + HEADERS):
-        with open(os.path.join(CSRC, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(CSRC, f)) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        lines = [ln.rstrip() for ln in text.splitlines() if ln.strip()]
+        h.update(f.encode())
+        h.update("\n".join(lines).encode())
     return h.hexdigest()[:12]
 
 

@@ -13,13 +13,14 @@
 //              into a 3-stage ring, laid out as the MMA's 128-byte-swizzled tiles.
 //   warp 8     MMA issuer: S = Q . K^T (M = 128 head rows of which the first H are real,
 //              N = 32 tokens, K = 576 as 36 tcgen05.mma of K = 16) into one of two TMEM
-//              score buffers; then O += P . V for the previous tile (A = P, bf16 in TMEM;
-//              B = the same tile's latent half read in place as an MN-major operand).
+//              score buffers, and O += P . V of the previous tile (A = P, bf16 in TMEM;
+//              B = that tile's latent half read in place as an MN-major operand), issued
+//              between those MMAs as soon as its P is ready.
 //   warps 4-7  softmax, one thread per head row (the warp's TMEM lane quadrant): masks the
 //              tile's missing tokens, keeps the running maximum m (in log2 units) and sum l,
 //              writes P = 2^(s - m) as bf16 into TMEM, and rescales O in TMEM only when the
-//              maximum rises by more than 2^8 (so P stays below 256); at the end O / l is
-//              written out in bf16 and the half-0 CTA writes lse.
+//              maximum rises by more than 8 (log2 units, so P stays below 256); at the end
+//              O / l is written out in bf16 and the half-0 CTA writes lse.
 
 #include "kernels.h"
 
@@ -41,7 +42,8 @@ constexpr int kMlaThreads = 288;
 constexpr int kMlaMmaWarp = 8;
 // TMEM columns: O (256 fp32), two score buffers (32 each), two P buffers (16 each)
 constexpr uint32_t kMlaTmemO = 0, kMlaTmemS = 256, kMlaTmemP = 320;
-constexpr int kMlaNumBars = 3 * 2 + 2 * 4;              // kv_full/empty[3], s_full/empty, p_full, pv_done [2]
+constexpr int kMlaNumBars = 3 * 2 + 2 * 4 + 1;          // kv_full/empty[3], s_full/empty, p_full, pv_done [2], mma_done
+constexpr uint64_t kMlaDrainNs = 200ull * 1000 * 1000;   // limit of the final wait for this CTA's MMAs
 constexpr int kMlaMaxSel = 2048;                         // selected entries per query held in shared memory
 constexpr int kMlaSmem = kMlaQBytes + kMlaStages * kMlaStage + 4 * kMlaMaxSel + 8 * kMlaNumBars + 64 + 1024;
 static_assert(kMlaQChunk % 1024 == 0 && kMlaKvChunk % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
@@ -111,6 +113,8 @@ __device__ __forceinline__ void tmem_st_32(uint32_t taddr, const uint32_t (&r)[3
       : "memory");
 }
 
+// 2^x by the hardware's approximate base-2 exponential (relative error near 2^-22, far below
+// the bf16 rounding the weights then get); 2^-inf = 0.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -130,6 +134,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(MlaParams p)
   uint64_t* s_empty = s_full + 2;
   uint64_t* p_full = s_empty + 2;
   uint64_t* pv_done = p_full + 2;
+  uint64_t* mma_done = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kMlaNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -165,6 +170,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(MlaParams p)
       mbar_init(&p_full[b], 4);
       mbar_init(&pv_done[b], 1);
     }
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -391,6 +397,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(MlaParams p)
     }
     for (; ok && pv_next < ntiles; ++pv_next)
       if ((ok = mbar_wait(&p_full[pv_next & 1], (pv_next >> 1) & 1, wc))) issue_pv(pv_next);
+    // every MMA this thread issued has finished before TMEM is freed (on an early exit too);
+    // the wait is bounded
+    umma_commit(mma_done);
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(smem_u32(mma_done), 0) && global_timer_ns() - t0 <= kMlaDrainNs) {
+    }
   }
   tc_fence_before();
   __syncthreads();
