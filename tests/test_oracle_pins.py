@@ -571,6 +571,37 @@ def test_sparse_mla_matches_torch_attention():
         assert np.allclose(lse[t], torch.logsumexp(s, dim=1).numpy(), rtol=1e-12)
 
 
+def test_sparse_mla_latent_form_equals_the_per_head_192_128_form():
+    # The per-head form of the 'Latent attention (MLA)' row: q/k heads of 192 = 128 no-rope
+    # + 64 rope dims, v heads of 128; keys and values are up-projected from the 512-dim latent
+    # c (k_nope = W_UK c, v = W_UV c) and the 64-dim rope key is shared by the heads.  Taking
+    # q_nope into the latent space (W_UK^T q_nope) gives the 576-value query the oracle takes,
+    # and W_UV applied to its 512-dim output gives the 128-dim head output: checked here with
+    # torch's attention on the up-projected keys and values.
+    import torch
+    rng = np.random.default_rng(11)
+    H, n = 3, 20
+    c = rng.standard_normal((n, 512))
+    k_rope = rng.standard_normal((n, 64))
+    W_UK = rng.standard_normal((H, 128, 512)) / np.sqrt(512)
+    W_UV = rng.standard_normal((H, 128, 512)) / np.sqrt(512)
+    q_nope = rng.standard_normal((H, 128))
+    q_rope = rng.standard_normal((H, 64))
+    scale = 1.0 / np.sqrt(192.0)
+    kv = np.concatenate([c, k_rope], axis=1)                          # the cached 576-value rows
+    q_lat = np.concatenate([np.einsum("hdc,hd->hc", W_UK, q_nope), q_rope], axis=1)
+    o_lat, lse = oracle.sparse_mla(q_lat[None], kv, np.array([0, n]), np.array([0, 1]),
+                                   np.arange(n)[None], scale)
+    o_head = np.einsum("hdc,hc->hd", W_UV, o_lat[0])                  # [H, 128]
+    for h in range(H):
+        k_h = torch.tensor(np.concatenate([c @ W_UK[h].T, k_rope], axis=1))   # [n, 192]
+        v_h = torch.tensor(c @ W_UV[h].T)                                       # [n, 128]
+        q_h = torch.tensor(np.concatenate([q_nope[h], q_rope[h]]))[None, None]  # [1, 1, 192]
+        ref = torch.nn.functional.scaled_dot_product_attention(q_h, k_h[None], v_h[None], scale=scale)
+        assert np.allclose(o_head[h], ref[0, 0].numpy(), rtol=1e-10, atol=1e-12)
+        assert np.isclose(lse[0, h], torch.logsumexp(scale * (k_h @ q_h[0, 0]), 0).item(), rtol=1e-12)
+
+
 def test_sparse_mla_brute_force_loops():
     q, kv, co, qo, idx = _mla_case(seed=3, T=2, H=2, n_rows=(9, 7), K=5, pad=1)
     scale = 0.7
