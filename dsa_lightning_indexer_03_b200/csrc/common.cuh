@@ -129,8 +129,10 @@ __device__ __forceinline__ int read_abort(const WaitCtl& c) {
   return v;
 }
 
-// bar is the barrier's shared-memory address
+// bar is the barrier's shared-memory address.  A phase that has already completed is taken
+// with one plain try_wait: the suspend-hinted form costs about 200 cycles even then.
 __device__ __forceinline__ bool mbar_wait_addr(uint32_t a, uint32_t parity, const WaitCtl& c) {
+  if (mbar_try_wait(a, parity)) return true;
   if (mbar_try_wait_sleep(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
