@@ -388,9 +388,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(MlaParams p)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
           umma_bf16(tmem + kMlaTmemS + 32 * b, ad + 2 * ks, bd + 2 * ks, idesc_s, (c > 0 || ks > 0) ? 1u : 0u);
-        // one look per tile, after a third of the score MMAs (each look costs the issue slot
-        // of about half an MMA)
-        if (c == 2 && pv_next < tile && mbar_try_wait(smem_u32(&p_full[pv_next & 1]), (pv_next >> 1) & 1)) {
+        if (pv_next < tile && mbar_try_wait(smem_u32(&p_full[pv_next & 1]), (pv_next >> 1) & 1)) {
           issue_pv(pv_next);
           ++pv_next;
         }
