@@ -369,13 +369,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) sparse_mla_kernel(MlaParams p)
       umma_commit(&kv_empty[su]);
     };
     // The P . V of a tile is issued as soon as its P is ready, between the score MMAs of the
-    // next tile (the tensor pipe runs them in issue order), and no later than before the
-    // wait for the tile that reuses its ring stage.
+    // next tile (the tensor pipe runs them in issue order), and at the latest before the wait
+    // for tile + 2: the gather threads publish tile + 2 only after they have passed the wait
+    // for the ring stage of tile + 3, which this P . V frees.
     int pv_next = 0;
     bool ok = true;
     for (int tile = 0; tile < ntiles && ok; ++tile) {
       const int s = tile % kMlaStages, b = tile & 1;
-      for (; pv_next < tile - 2; ++pv_next)
+      for (; pv_next < tile - 1; ++pv_next)
         if (!(ok = mbar_wait(&p_full[pv_next & 1], (pv_next >> 1) & 1, wc))) break; else issue_pv(pv_next);
       if (!ok) break;
       if (!mbar_wait(&kv_full[s], (tile / kMlaStages) & 1, wc)) break;
