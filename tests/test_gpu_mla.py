@@ -208,3 +208,26 @@ def test_sparse_mla_decode_full_size(dsa, ix):
                                            np.arange(2048)[None, :], SCALE)
         o_tol, lse_tol = _tolerances(q_t, kv_t, o_ref[0])
         _check(o[t:t + 1], lse[t:t + 1], o_ref, lse_ref, o_tol[None], lse_tol[None])
+
+
+def test_sparse_mla_on_the_prefill_8k_selection_full_size(dsa):
+    # the bench's prefill_8k workload (full-size weights and activations) through project and
+    # top-k, its [8,192, 2,048] selection (rows of early queries padded with -1) feeding the
+    # attention with all 96 heads: 16,384 CTAs; 24 stratified queries against the oracle
+    cfg = W.WORKLOADS["prefill_8k"]
+    wts = W.make_weights(cfg["weight_seed"])
+    pre = W.make_prefill(cfg["act_seed"], cfg["seq_lens"])
+    dev = "cuda"
+    ix = dsa.Indexer(*(t.to(dev).contiguous() for t in (wts.W_q, wts.W_k, wts.W_w, wts.gamma, wts.beta)),
+                     max_tokens=8192)
+    T = pre.hidden.shape[0]
+    cache = torch.zeros((T, 128), dtype=torch.bfloat16, device=dev)
+    pos, qoff, coff = pre.positions.to(dev), pre.q_seq_offsets.to(dev), pre.cache_offsets.to(dev)
+    q, w = ix.project(pre.hidden.to(dev), pre.q_latent.to(dev), pos, qoff, cache, coff)
+    idx, _ = ix.topk(q, w, pos, qoff, cache, coff)
+    mla = W.make_mla(47, [T], [T], n_heads=96, k_sel=1)          # q and cache only; idx replaced
+    batch = W.MlaBatch(mla.q, mla.kv, mla.cache_offsets, mla.q_seq_offsets, idx.cpu())
+    o, lse = _run(dsa, ix, batch)
+    assert np.all(np.isfinite(lse)) and np.all(np.isfinite(o))
+    sample = W.stratified_rows(pre.q_seq_offsets, 24, seed=2, positions=pre.positions).numpy()
+    _check(o[sample], lse[sample], *_ref(batch, rows=sample))
