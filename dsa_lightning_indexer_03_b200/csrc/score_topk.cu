@@ -1568,7 +1568,10 @@ struct PrepParams {
 };
 
 __device__ int block_exclusive_scan(int* a, int n, int* warp_sums) {
-  // in-place exclusive scan of a[0..n) by kPrepThreads threads; returns the total
+  // in-place exclusive scan of a[0..n) by kPrepThreads threads; returns the total.  Warp 0
+  // scans all 32 warp sums, so the block must have exactly 32 warps (kPrepThreads = 1024):
+  // with fewer, stale sums would enter the totals and the item list would be written out of
+  // bounds.
   __shared__ int carry;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
